@@ -1,0 +1,234 @@
+/*
+ * mglu_oracle.c -- the CPU oracle for the Masked Gated Linear Unit forward.
+ *
+ * TEST INFRASTRUCTURE ONLY.  This file is the plain, slow, float64 statement
+ * of what the MGLU forward computes.  Only the test suite, the smoke check and
+ * the benchmark's CPU-baseline leg may load it.  It shares no code, header,
+ * table or packing routine with the CUDA library; neither side includes or
+ * links the other.
+ *
+ * Source of the method: "Masked Gated Linear Unit" (atlas.scime.ai summary
+ * page of the MGLU paper), sections "Approach" and "Key results", and the rows
+ * of its "Measured effects" table about summing all masks and about the
+ * GELU / ReLU gating activations.  The page gives no equation; the reading
+ * written out below is:
+ *
+ *     out[b,j] = sum_{i < n_m} act(g_i[b,j]) * v_i[b,j]
+ *     g_i[b,j] = sum_k x[b,k] * W[k,j] * M_i[k,j]          (gate subspace)
+ *     v_i[b,j] = sum_k x[b,k] * W[k,j] * (1 - M_i[k,j])    (value subspace)
+ *
+ * One shared weight W, n_m binary masks, each mask splitting W into
+ * complementary gate and value parts ("Approach"); the n_m gated products are
+ * summed, not averaged ("Measured effects": routing to 1 or 2 of 4 masks is
+ * compared against summing all 4).  act is Swish (beta = 1), exact-erf GELU or
+ * ReLU ("Measured effects": the GELU and ReLU gating-activation rows).
+ * Which side of a mask is the gate is not stated on the page; the reading
+ * here is bit = 1 -> gate.
+ *
+ * Storage: x is [T][d]; W is stored transposed as Ws[j][k] = W[k,j]
+ * (the nn.Linear(d, h).weight layout); masks unpacked are [n_m][h][d] bytes
+ * in {0,1} with masks[i][j][k] = M_i[k,j].
+ *
+ * Packed mask format (this library's own format; the page only says masks
+ * are binary and are unpacked inside the fused kernel, "Approach"): weight
+ * (j,k) owns n_m consecutive bits starting at bit offset (j*d + k)*n_m of a
+ * little-endian byte stream, bit i of that field is mask i, bits counted from
+ * the least significant bit of each byte.
+ *
+ * Every product and sum is taken in float64 from the exact input values the
+ * GPU also consumes (inputs are rounded to bf16 or fp32 before either side
+ * sees them).  v_i is summed from its own definition, not as D - g_i, so the
+ * oracle does not share the GPU's algebraic shortcut; the invariant
+ * g_i + v_i = D is measured and returned to the caller.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#define ORACLE_ACT_SWISH 0
+#define ORACLE_ACT_GELU 1
+#define ORACLE_ACT_RELU 2
+
+/* Gating activation ("Measured effects": Swish is the default, GELU and ReLU
+ * are the ablation rows).  Swish with beta = 1 (SiLU, as in SwiGLU); GELU in
+ * its exact form z * Phi(z), Phi the standard normal CDF written with erf. */
+static double oracle_act(int act, double z)
+{
+    switch (act) {
+    case ORACLE_ACT_SWISH:
+        return z / (1.0 + exp(-z));
+    case ORACLE_ACT_GELU:
+        return 0.5 * z * (1.0 + erf(z / sqrt(2.0)));
+    case ORACLE_ACT_RELU:
+        return z > 0.0 ? z : 0.0;
+    default:
+        return NAN;
+    }
+}
+
+double oracle_activation(int act, double z) { return oracle_act(act, z); }
+
+/* Bit i of weight (j,k) from the packed stream, read bit by bit. */
+static int oracle_bit(const uint8_t *packed, int n_m, int64_t d, int64_t j,
+                      int64_t k, int i)
+{
+    int64_t pos = (j * d + k) * (int64_t)n_m + i;
+    return (packed[pos >> 3] >> (pos & 7)) & 1;
+}
+
+int64_t oracle_packed_bytes(int n_m, int64_t d, int64_t h)
+{
+    return (h * d * (int64_t)n_m + 7) / 8;
+}
+
+/* masks[i][j][k] in {0,1}  ->  packed stream.  One bit at a time. */
+void oracle_pack_masks(const uint8_t *masks, int n_m, int64_t d, int64_t h,
+                       uint8_t *packed)
+{
+    int64_t nbytes = oracle_packed_bytes(n_m, d, h);
+    memset(packed, 0, (size_t)nbytes);
+    for (int i = 0; i < n_m; ++i)
+        for (int64_t j = 0; j < h; ++j)
+            for (int64_t k = 0; k < d; ++k) {
+                if (masks[((int64_t)i * h + j) * d + k]) {
+                    int64_t pos = (j * d + k) * (int64_t)n_m + i;
+                    packed[pos >> 3] |= (uint8_t)(1u << (pos & 7));
+                }
+            }
+}
+
+/* packed stream -> masks[i][j][k] in {0,1}. */
+void oracle_unpack_masks(const uint8_t *packed, int n_m, int64_t d, int64_t h,
+                         uint8_t *masks)
+{
+    for (int i = 0; i < n_m; ++i)
+        for (int64_t j = 0; j < h; ++j)
+            for (int64_t k = 0; k < d; ++k)
+                masks[((int64_t)i * h + j) * d + k] =
+                    (uint8_t)oracle_bit(packed, n_m, d, j, k, i);
+}
+
+/* The three sums for one (b, j): the dense product D, and for each mask i the
+ * gate part g[i] and the value part v[i], each from its own definition.
+ * Returns |sum_k x W| (the scale the invariant is measured against) in *absw
+ * and the worst |g_i + v_i - D| in *resid. */
+void oracle_gate_value(const double *x, int64_t d, const double *Ws,
+                       const uint8_t *packed, int n_m, int64_t b, int64_t j,
+                       double *D, double *g, double *v, double *absw,
+                       double *resid)
+{
+    const double *xb = x + b * d;
+    const double *wj = Ws + j * d;
+    double dense = 0.0, scale = 0.0;
+    for (int64_t k = 0; k < d; ++k) {
+        dense += xb[k] * wj[k];
+        scale += fabs(xb[k] * wj[k]);
+    }
+    double worst = 0.0;
+    for (int i = 0; i < n_m; ++i) {
+        double gi = 0.0, vi = 0.0;
+        for (int64_t k = 0; k < d; ++k) {
+            int m = oracle_bit(packed, n_m, d, j, k, i);
+            gi += xb[k] * wj[k] * (double)m;
+            vi += xb[k] * wj[k] * (double)(1 - m);
+        }
+        g[i] = gi;
+        v[i] = vi;
+        double r = fabs(gi + vi - dense);
+        if (r > worst)
+            worst = r;
+    }
+    *D = dense;
+    *absw = scale;
+    *resid = worst;
+}
+
+/* out[b,j] for one element; returns the invariant residual relative to the
+ * scale sum_k |x W| (0 when the scale is 0). */
+static double oracle_element(const double *x, int64_t d, const double *Ws,
+                             const uint8_t *packed, int n_m, int act,
+                             int64_t b, int64_t j, double *out)
+{
+    double g[8], v[8], D, absw, resid;
+    oracle_gate_value(x, d, Ws, packed, n_m, b, j, &D, g, v, &absw, &resid);
+    double acc = 0.0;
+    for (int i = 0; i < n_m; ++i)
+        acc += oracle_act(act, g[i]) * v[i];
+    *out = acc;
+    return absw > 0.0 ? resid / absw : resid;
+}
+
+/* Full forward: out[T][h].  Columns are independent, so they are spread over
+ * OpenMP threads; each element is the plain sum above.  Returns the worst
+ * relative invariant residual, or -1 for an unsupported n_m / act. */
+double oracle_forward(const double *x, int64_t T, int64_t d, const double *Ws,
+                      int64_t h, const uint8_t *packed, int n_m, int act,
+                      double *out)
+{
+    if (n_m < 1 || n_m > 8 || act < 0 || act > 2)
+        return -1.0;
+    double worst = 0.0;
+#pragma omp parallel for schedule(dynamic, 4) reduction(max : worst)
+    for (int64_t j = 0; j < h; ++j)
+        for (int64_t b = 0; b < T; ++b) {
+            double r = oracle_element(x, d, Ws, packed, n_m, act, b, j,
+                                      &out[b * h + j]);
+            if (r > worst)
+                worst = r;
+        }
+    return worst;
+}
+
+/* The same for a list of n elements (b_idx[e], j_idx[e]) -> out[e]. */
+double oracle_forward_elems(const double *x, int64_t d, const double *Ws,
+                            const uint8_t *packed, int n_m, int act, int64_t n,
+                            const int64_t *b_idx, const int64_t *j_idx,
+                            double *out)
+{
+    if (n_m < 1 || n_m > 8 || act < 0 || act > 2)
+        return -1.0;
+    double worst = 0.0;
+#pragma omp parallel for schedule(dynamic, 16) reduction(max : worst)
+    for (int64_t e = 0; e < n; ++e) {
+        double r = oracle_element(x, d, Ws, packed, n_m, act, b_idx[e],
+                                  j_idx[e], &out[e]);
+        if (r > worst)
+            worst = r;
+    }
+    return worst;
+}
+
+/* FFN down-projection: y[b,c] = sum_j hid[b,j] * Wd[c,j], Wd stored [d][h]
+ * (nn.Linear(h, d).weight).  MGLU replaces only the two GLU projections
+ * ("Masked Gated Linear Unit", summary line and "Problem"); the third FFN
+ * matrix stays dense. */
+void oracle_down(const double *hid, int64_t T, int64_t h, const double *Wd,
+                 int64_t d, double *y)
+{
+#pragma omp parallel for schedule(static)
+    for (int64_t c = 0; c < d; ++c)
+        for (int64_t b = 0; b < T; ++b) {
+            double acc = 0.0;
+            for (int64_t j = 0; j < h; ++j)
+                acc += hid[b * h + j] * Wd[c * h + j];
+            y[b * d + c] = acc;
+        }
+}
+
+/* y for a list of n elements (b_idx[e], c_idx[e]); hid holds the needed rows
+ * of the hidden activation, hid_row[e] names the row for element e. */
+void oracle_down_elems(const double *hid, int64_t h, const double *Wd,
+                       int64_t n, const int64_t *hid_row, const int64_t *c_idx,
+                       double *y)
+{
+#pragma omp parallel for schedule(static)
+    for (int64_t e = 0; e < n; ++e) {
+        double acc = 0.0;
+        const double *hr = hid + hid_row[e] * h;
+        const double *wc = Wd + c_idx[e] * h;
+        for (int64_t j = 0; j < h; ++j)
+            acc += hr[j] * wc[j];
+        y[e] = acc;
+    }
+}
