@@ -1,0 +1,159 @@
+/*
+ * mglu.h -- C ABI of libmglu.so, a B200 (sm_100a) forward pass of the Masked
+ * Gated Linear Unit (MGLU, "Mixture of Element-wise Gating").
+ *
+ * The method ("Masked Gated Linear Unit", atlas.scime.ai summary of the MGLU
+ * paper, "Approach"): one shared weight matrix W (d x h) and n_m learned
+ * binary masks M_i over it.  Mask i splits W into complementary gate and value
+ * parts; the layer sums the n_m gated products ("Measured effects": summing
+ * all 4 masks is the default the routing ablations are measured against):
+ *
+ *     out[b,j] = sum_{i<n_m} act(g_i[b,j]) * v_i[b,j]
+ *     g_i = x (M_i . W)          v_i = x ((1 - M_i) . W) = x W - g_i
+ *
+ * act is Swish (beta = 1, "SwiMGLU"), exact-erf GELU or ReLU ("Measured
+ * effects" rows on the gating activation).  Which side of a mask is the gate
+ * is not stated on the page; here a set bit marks a gate weight.  No biases.
+ *
+ * Conventions for every call:
+ *  - All tensor pointers are DEVICE pointers owned by the caller.  The library
+ *    allocates no device memory on any call declared here.
+ *  - Calls are asynchronous and ordered on `stream` (a cudaStream_t passed as
+ *    void*; NULL = the legacy default stream).
+ *  - Arguments are checked before anything is launched.  A negative return
+ *    is an mglu_status; nothing was launched when it is INVALID, UNSUPPORTED
+ *    or ALIGN.  MGLU_ERR_CUDA means a launch failed (cudaGetLastError is
+ *    cleared and the text is available from mglu_last_cuda_error()).
+ *  - Layouts (row-major, dense, no padding):
+ *        x       [T][d]            activations
+ *        W       [h][d]            W^T, i.e. nn.Linear(d, h).weight
+ *        masks   [n_m][h][d]       uint8, 0 or 1 (unpacked form)
+ *        packed  mglu_packed_bytes(n_m, d, h) bytes, see mglu_pack_masks
+ *        out     [T][h]
+ *        W_down  [d][h]            nn.Linear(h, d).weight
+ *        y       [T][d]
+ *  - bf16 path (dtype MGLU_BF16): x, W, out, W_down, y are bf16; products are
+ *    exact and accumulate in fp32; the result is rounded to bf16 once.
+ *    Requirements (else MGLU_ERR_ALIGN): every pointer 16-byte aligned,
+ *    d % 8 == 0 and (d * n_m) % 128 == 0, so that a row of W and a row of
+ *    packed mask bytes both start on a 16-byte boundary.
+ *  - fp32 path (dtype MGLU_F32): x, W, out, W_down, y are float; plain fp32
+ *    FMA on CUDA cores (never TF32); any d, h; 4-byte aligned pointers.
+ *  - Supported n_m: 1, 2, 4, 8 (else MGLU_ERR_UNSUPPORTED).  T == 0 is a
+ *    no-op that returns MGLU_OK.  Sizes are limited to d, h < 2^31 and
+ *    T * max(d, h) < 2^62.
+ */
+#ifndef MGLU_H
+#define MGLU_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    MGLU_OK = 0,
+    MGLU_ERR_INVALID = -1,     /* null pointer, negative size, bad act/dtype, small workspace */
+    MGLU_ERR_UNSUPPORTED = -2, /* n_m not in {1,2,4,8} */
+    MGLU_ERR_ALIGN = -3,       /* a pointer or size alignment rule above is broken */
+    MGLU_ERR_CUDA = -4,        /* a CUDA runtime call or a kernel launch failed */
+    MGLU_ERR_TIMEOUT = -5      /* a device-side bounded wait gave up (see mglu_last_device_status) */
+} mglu_status;
+
+typedef enum { MGLU_ACT_SWISH = 0, MGLU_ACT_GELU = 1, MGLU_ACT_RELU = 2 } mglu_act;
+typedef enum { MGLU_BF16 = 0, MGLU_F32 = 1 } mglu_dtype;
+
+/* Kernel families mglu_forward can launch (see mglu_forward_path). */
+typedef enum { MGLU_PATH_DECODE = 0, MGLU_PATH_PREFILL = 1, MGLU_PATH_F32 = 2 } mglu_path;
+
+/* Bytes of the packed mask stream: ceil(h * d * n_m / 8).  0 for bad input. */
+size_t mglu_packed_bytes(int n_m, int64_t d, int64_t h);
+
+/*
+ * Pack n_m binary masks into the bit stream the forward reads ("Approach":
+ * the masks are binary and are unpacked inside the fused kernel; the bit
+ * format is this library's own).  Weight (j, k) owns the n_m consecutive bits
+ * starting at bit (j*d + k)*n_m; bit i of that field is mask i; bits are
+ * numbered from the least significant bit of each byte.  So for n_m = 8 byte
+ * j*d+k holds the eight masks of weight (j, k); for n_m = 4 the low nibble of
+ * a byte is weight k (even) and the high nibble weight k+1.  A row of W
+ * (fixed j) and its mask bits are therefore tiled alike along k.
+ *   masks   in : [n_m][h][d] uint8; any nonzero byte counts as 1.
+ *   packed out : mglu_packed_bytes(n_m, d, h) bytes, every byte written.
+ * Requirements: d % 8 == 0 (so each byte holds whole weights), packed
+ * 16-byte aligned.  Errors: INVALID, UNSUPPORTED, ALIGN, CUDA.
+ */
+int mglu_pack_masks(const uint8_t *masks, int n_m, int64_t d, int64_t h,
+                    uint8_t *packed, void *stream);
+
+/* Exact inverse of mglu_pack_masks: writes [n_m][h][d] bytes, each 0 or 1. */
+int mglu_unpack_masks(const uint8_t *packed, int n_m, int64_t d, int64_t h,
+                      uint8_t *masks, void *stream);
+
+/*
+ * MGLU up-projection with the act-and-sum epilogue fused: out = MGLU(x).
+ * Reads each weight and its mask bits once per pass; for T up to the decode
+ * limit (16 by default) one pass serves all tokens; above it a tensor-core
+ * (tcgen05) kernel tiles tokens and weights.
+ *   x [T][d], W [h][d], packed (from mglu_pack_masks with the same n_m, d, h),
+ *   act in mglu_act, dtype in mglu_dtype, out [T][h].
+ * Errors: INVALID, UNSUPPORTED, ALIGN, CUDA.
+ */
+int mglu_forward(const void *x, int64_t T, int64_t d, const void *W, int64_t h,
+                 const uint8_t *packed, int n_m, int act, int dtype, void *out,
+                 void *stream);
+
+/*
+ * The FFN down-projection alone, a dense product (MGLU replaces only the two
+ * GLU projections; "Masked Gated Linear Unit", summary line):
+ *   y[b,c] = sum_j hid[b,j] * W_down[c,j]
+ *   hid [T][h], W_down [d][h], y [T][d].
+ * bf16 requirements: 16-byte aligned pointers, h % 8 == 0.
+ */
+int mglu_down_proj(const void *hid, int64_t T, int64_t h, const void *W_down,
+                   int64_t d, int dtype, void *y, void *stream);
+
+/* Workspace bytes mglu_forward_down needs: the hidden activation [T][h] in
+ * the path's dtype, rounded up to 256 bytes. */
+size_t mglu_workspace_bytes(int64_t T, int64_t d, int64_t h, int n_m, int dtype);
+
+/*
+ * The FFN block: y = MGLU(x) W_down^T.  The hidden activation is written to
+ * the caller's workspace (dtype of the path; bf16 rounding happens once, as
+ * in mglu_forward) and then multiplied by W_down, both on `stream`.
+ * workspace_bytes must be >= mglu_workspace_bytes(...) (else INVALID).
+ */
+int mglu_forward_down(const void *x, int64_t T, int64_t d, const void *W,
+                      int64_t h, const uint8_t *packed, int n_m, int act,
+                      int dtype, const void *W_down, void *workspace,
+                      size_t workspace_bytes, void *y, void *stream);
+
+/* Which kernel family mglu_forward uses for T tokens of `dtype`. */
+int mglu_forward_path(int64_t T, int dtype);
+
+/* Largest T served by the decode kernel (the rest go to the tensor-core
+ * kernel).  Accepts 0..16 (0 = always the tensor-core kernel); returns the
+ * previous value, or MGLU_ERR_INVALID.  Process-wide setting. */
+int mglu_set_decode_max_tokens(int t);
+
+/*
+ * Synchronizes `stream`, then reads and clears the library's device status
+ * word for the current device.  Kernels whose bounded waits give up record
+ * MGLU_ERR_TIMEOUT there instead of hanging.  Returns MGLU_OK, an error
+ * recorded by a kernel, or MGLU_ERR_CUDA if the synchronization failed.
+ */
+int mglu_last_device_status(void *stream);
+
+/* Text of the last CUDA error seen by the library on this thread ("" if none). */
+const char *mglu_last_cuda_error(void);
+
+/* Static text for an mglu_status value. */
+const char *mglu_status_string(int status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MGLU_H */

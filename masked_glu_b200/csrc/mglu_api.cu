@@ -1,0 +1,479 @@
+// mglu_api.cu -- the C ABI of libmglu.so (declared in include/mglu.h):
+// argument checks, TMA descriptor encoding, kernel choice and launches.
+// Everything is one translation unit so the device status word is shared.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+#include "mglu.h"
+#include "common.cuh"
+#include "decode.cuh"
+#include "pack.cuh"
+#include "prefill.cuh"
+#include "ptx.cuh"
+#include "simt.cuh"
+
+namespace {
+
+thread_local char g_last_cuda_error[256] = "";
+int g_decode_max_tokens = 16;
+constexpr int kMaxDevices = 64;
+
+int cuda_fail(cudaError_t e, const char *what)
+{
+    snprintf(g_last_cuda_error, sizeof(g_last_cuda_error), "%s: %s", what, cudaGetErrorString(e));
+    return MGLU_ERR_CUDA;
+}
+
+int check_launch(const char *what)
+{
+    const cudaError_t e = cudaGetLastError();
+    return e == cudaSuccess ? MGLU_OK : cuda_fail(e, what);
+}
+
+bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+bool nm_supported(int n_m) { return n_m == 1 || n_m == 2 || n_m == 4 || n_m == 8; }
+
+int current_device(int *dev)
+{
+    const cudaError_t e = cudaGetDevice(dev);
+    if (e != cudaSuccess)
+        return cuda_fail(e, "cudaGetDevice");
+    if (*dev < 0 || *dev >= kMaxDevices)
+        return MGLU_ERR_INVALID;
+    return MGLU_OK;
+}
+
+int sm_count(int dev)
+{
+    static int cache[kMaxDevices] = {0};
+    if (cache[dev] == 0) {
+        int n = 0;
+        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+        cache[dev] = n > 0 ? n : 148;
+    }
+    return cache[dev];
+}
+
+// cuTensorMapEncodeTiled through the runtime's driver entry point, so the
+// library does not link libcuda directly.
+using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                   const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn()
+{
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    });
+    return fn;
+}
+
+// 2-D tensor map: `outer` rows of `inner` elements, rows `row_bytes` apart;
+// box of box_outer rows x box_inner elements; out-of-range reads give zeros.
+int make_map(CUtensorMap *m, CUtensorMapDataType dt, const void *base, uint64_t inner, uint64_t outer,
+             uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle sw)
+{
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) {
+        snprintf(g_last_cuda_error, sizeof(g_last_cuda_error), "cuTensorMapEncodeTiled unavailable");
+        return MGLU_ERR_CUDA;
+    }
+    const cuuint64_t dims[2] = {inner, outer};
+    const cuuint64_t strides[1] = {row_bytes};
+    const cuuint32_t box[2] = {box_inner, box_outer};
+    const cuuint32_t es[2] = {1, 1};
+    const CUresult r = fn(m, dt, 2, const_cast<void *>(base), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                          sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) {
+        snprintf(g_last_cuda_error, sizeof(g_last_cuda_error), "cuTensorMapEncodeTiled failed (%d)", (int)r);
+        return MGLU_ERR_CUDA;
+    }
+    return MGLU_OK;
+}
+
+// Raise the kernel's dynamic shared-memory limit once per device (one flag
+// array per kernel instantiation).
+template <auto Kernel>
+int ensure_smem(int bytes, int dev)
+{
+    static bool done[kMaxDevices] = {false};
+    if (!done[dev]) {
+        const cudaError_t e =
+            cudaFuncSetAttribute(reinterpret_cast<const void *>(Kernel), cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+        if (e != cudaSuccess)
+            return cuda_fail(e, "cudaFuncSetAttribute");
+        done[dev] = true;
+    }
+    return MGLU_OK;
+}
+
+// ------------------------------------------------------------------ decode
+int choose_ksplit(int64_t row_blocks, int nst, int sms)
+{
+    const int64_t target = (int64_t)sms * 8;
+    int ks = 1;
+    while (ks < 8 && row_blocks * ks < target && nst >= 4 * ks)
+        ks *= 2;
+    return ks;
+}
+
+template <int NM, int NT>
+int launch_decode(const void *x, int64_t T, int64_t d, const void *W, int64_t rows, const uint8_t *packed, int act,
+                  void *out, cudaStream_t s)
+{
+    using L = mglu::dec::Layout<NM, NT>;
+    int dev = 0, rc = current_device(&dev);
+    if (rc)
+        return rc;
+    CUtensorMap tw, tx, tm;
+    if ((rc = make_map(&tw, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, W, d, rows, d * 2, mglu::dec::SUBK, mglu::dec::ROWS,
+                       CU_TENSOR_MAP_SWIZZLE_128B)))
+        return rc;
+    if ((rc = make_map(&tx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, x, d, T, d * 2, mglu::dec::SUBK, 8 * NT,
+                       CU_TENSOR_MAP_SWIZZLE_128B)))
+        return rc;
+    if (NM > 0) {
+        if ((rc = make_map(&tm, CU_TENSOR_MAP_DATA_TYPE_UINT8, packed, d * NM / 8, rows, d * NM / 8,
+                           mglu::dec::KS * NM / 8, mglu::dec::ROWS, CU_TENSOR_MAP_SWIZZLE_NONE)))
+            return rc;
+    } else {
+        tm = tw;  // not read
+    }
+    auto kernel = mglu::dec::decode_kernel<NM, NT>;
+    if ((rc = ensure_smem<mglu::dec::decode_kernel<NM, NT>>(L::SMEM, dev)))
+        return rc;
+    const int64_t rb = (rows + mglu::dec::ROWS - 1) / mglu::dec::ROWS;
+    const int nst = (int)((d + mglu::dec::KS - 1) / mglu::dec::KS);
+    const int ks = choose_ksplit(rb, nst, sm_count(dev));
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)(rb * ks));
+    cfg.blockDim = dim3(mglu::dec::NTHREADS);
+    cfg.dynamicSmemBytes = L::SMEM;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = (unsigned)ks;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = ks > 1 ? 1 : 0;
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, tw, tx, tm, (int)T, (int)rows, (int)d, ks, act,
+                                             reinterpret_cast<__nv_bfloat16 *>(out));
+    if (e != cudaSuccess)
+        return cuda_fail(e, "decode launch");
+    return check_launch("decode launch");
+}
+
+template <int NM>
+int decode_nt(const void *x, int64_t T, int64_t d, const void *W, int64_t rows, const uint8_t *packed, int act,
+              void *out, cudaStream_t s)
+{
+    return T <= 8 ? launch_decode<NM, 1>(x, T, d, W, rows, packed, act, out, s)
+                  : launch_decode<NM, 2>(x, T, d, W, rows, packed, act, out, s);
+}
+
+// ------------------------------------------------------------------ prefill
+template <int NM>
+int launch_prefill(const void *x, int64_t T, int64_t d, const void *W, int64_t rows, const uint8_t *packed, int act,
+                   void *out, cudaStream_t s)
+{
+    using C = mglu::pf::Cfg<NM>;
+    int dev = 0, rc = current_device(&dev);
+    if (rc)
+        return rc;
+    CUtensorMap tx, tw, tm;
+    if ((rc = make_map(&tx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, x, d, T, d * 2, mglu::pf::BK, mglu::pf::BM,
+                       CU_TENSOR_MAP_SWIZZLE_128B)))
+        return rc;
+    if ((rc = make_map(&tw, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, W, d, rows, d * 2, mglu::pf::BK, C::NJ,
+                       CU_TENSOR_MAP_SWIZZLE_128B)))
+        return rc;
+    if (NM > 0) {
+        if ((rc = make_map(&tm, CU_TENSOR_MAP_DATA_TYPE_UINT8, packed, d * NM / 8, rows, d * NM / 8, C::MB, C::NJ,
+                           CU_TENSOR_MAP_SWIZZLE_NONE)))
+            return rc;
+    } else {
+        tm = tw;  // not read
+    }
+    auto kernel = mglu::pf::prefill_kernel<NM>;
+    if ((rc = ensure_smem<mglu::pf::prefill_kernel<NM>>(C::SMEM, dev)))
+        return rc;
+    const int64_t tiles = ((T + mglu::pf::BM - 1) / mglu::pf::BM) * ((rows + C::NJ - 1) / C::NJ);
+    const int grid = (int)(tiles < sm_count(dev) ? tiles : sm_count(dev));
+    kernel<<<grid, mglu::pf::NTHREADS, C::SMEM, s>>>(tx, tw, tm, (int)T, (int)rows, (int)d, act,
+                                                     reinterpret_cast<__nv_bfloat16 *>(out));
+    return check_launch("prefill launch");
+}
+
+// ------------------------------------------------------------------ fp32
+template <int NM>
+int launch_simt(const void *x, int64_t T, int64_t d, const void *W, int64_t rows, const uint8_t *packed, int act,
+                void *out, cudaStream_t s)
+{
+    const dim3 grid((unsigned)((rows + 7) / 8), (unsigned)((T + mglu::kSimtTokens - 1) / mglu::kSimtTokens));
+    if (grid.y > 65535u)
+        return MGLU_ERR_INVALID;
+    mglu::simt_f32_kernel<NM><<<grid, 256, 0, s>>>(reinterpret_cast<const float *>(x), T, d,
+                                                     reinterpret_cast<const float *>(W), rows, packed, act,
+                                                     reinterpret_cast<float *>(out));
+    return check_launch("fp32 launch");
+}
+
+// Dispatch on n_m at compile time.
+template <template <int> class F, typename... A>
+int by_nm(int n_m, A... a)
+{
+    switch (n_m) {
+    case 0: return F<0>::run(a...);
+    case 1: return F<1>::run(a...);
+    case 2: return F<2>::run(a...);
+    case 4: return F<4>::run(a...);
+    case 8: return F<8>::run(a...);
+    default: return MGLU_ERR_UNSUPPORTED;
+    }
+}
+
+template <int NM>
+struct DecodeF {
+    template <typename... A>
+    static int run(A... a) { return decode_nt<NM>(a...); }
+};
+template <int NM>
+struct PrefillF {
+    template <typename... A>
+    static int run(A... a) { return launch_prefill<NM>(a...); }
+};
+template <int NM>
+struct SimtF {
+    template <typename... A>
+    static int run(A... a) { return launch_simt<NM>(a...); }
+};
+
+int path_for(int64_t T, int dtype)
+{
+    if (dtype == MGLU_F32)
+        return MGLU_PATH_F32;
+    return T <= g_decode_max_tokens ? MGLU_PATH_DECODE : MGLU_PATH_PREFILL;
+}
+
+// One product of the library: out[T][rows] from x[T][d] and W[rows][d] with
+// n_m masks (n_m = 0: dense).  Arguments already validated.
+int run_product(const void *x, int64_t T, int64_t d, const void *W, int64_t rows, const uint8_t *packed, int n_m,
+                int act, int dtype, void *out, cudaStream_t s)
+{
+    if (T == 0)
+        return MGLU_OK;
+    switch (path_for(T, dtype)) {
+    case MGLU_PATH_F32: return by_nm<SimtF>(n_m, x, T, d, W, rows, packed, act, out, s);
+    case MGLU_PATH_DECODE: return by_nm<DecodeF>(n_m, x, T, d, W, rows, packed, act, out, s);
+    default: return by_nm<PrefillF>(n_m, x, T, d, W, rows, packed, act, out, s);
+    }
+}
+
+bool sizes_ok(int64_t T, int64_t d, int64_t h)
+{
+    const int64_t lim = (int64_t)1 << 31;
+    if (T < 0 || d <= 0 || h <= 0 || T >= lim || d >= lim || h >= lim)
+        return false;
+    const int64_t mx = d > h ? d : h;
+    return T == 0 || mx <= ((int64_t)1 << 62) / (T > 0 ? T : 1);
+}
+
+int check_forward(const void *x, int64_t T, int64_t d, const void *W, int64_t h, const uint8_t *packed, int n_m,
+                  int act, int dtype, const void *out)
+{
+    if (!sizes_ok(T, d, h))
+        return MGLU_ERR_INVALID;
+    if (act < 0 || act > 2 || (dtype != MGLU_BF16 && dtype != MGLU_F32))
+        return MGLU_ERR_INVALID;
+    if (!nm_supported(n_m))
+        return MGLU_ERR_UNSUPPORTED;
+    if (!W || !packed || (T > 0 && (!x || !out)))
+        return MGLU_ERR_INVALID;
+    if (dtype == MGLU_BF16) {
+        if (!aligned(W, 16) || !aligned(packed, 16) || (T > 0 && (!aligned(x, 16) || !aligned(out, 16))))
+            return MGLU_ERR_ALIGN;
+        if (d % 8 != 0 || (d * n_m) % 128 != 0)
+            return MGLU_ERR_ALIGN;
+    } else {
+        if (!aligned(W, 4) || (T > 0 && (!aligned(x, 4) || !aligned(out, 4))))
+            return MGLU_ERR_ALIGN;
+    }
+    return MGLU_OK;
+}
+
+int check_down(const void *hid, int64_t T, int64_t h, const void *Wd, int64_t d, int dtype, const void *y)
+{
+    if (!sizes_ok(T, h, d))
+        return MGLU_ERR_INVALID;
+    if (dtype != MGLU_BF16 && dtype != MGLU_F32)
+        return MGLU_ERR_INVALID;
+    if (!Wd || (T > 0 && (!hid || !y)))
+        return MGLU_ERR_INVALID;
+    if (dtype == MGLU_BF16) {
+        if (!aligned(Wd, 16) || (T > 0 && (!aligned(hid, 16) || !aligned(y, 16))))
+            return MGLU_ERR_ALIGN;
+        if (h % 8 != 0)
+            return MGLU_ERR_ALIGN;
+    } else {
+        if (!aligned(Wd, 4) || (T > 0 && (!aligned(hid, 4) || !aligned(y, 4))))
+            return MGLU_ERR_ALIGN;
+    }
+    return MGLU_OK;
+}
+
+template <int NM>
+int pack_dispatch(const uint8_t *in, int64_t d, int64_t h, uint8_t *outp, bool unpack, cudaStream_t s)
+{
+    const int64_t hd = h * d;
+    const int64_t nbytes = hd * NM / 8;
+    const int64_t chunks = (nbytes + 15) / 16;
+    const int vec = (hd % 16 == 0) && aligned(unpack ? outp : in, 16);
+    const int64_t blocks = (chunks + 255) / 256;
+    if (blocks > 0x7FFFFFFF)
+        return MGLU_ERR_INVALID;
+    if (unpack)
+        mglu::unpack_kernel<NM><<<(unsigned)blocks, 256, 0, s>>>(in, hd, nbytes, outp, vec);
+    else
+        mglu::pack_kernel<NM><<<(unsigned)blocks, 256, 0, s>>>(in, hd, nbytes, outp, vec);
+    return check_launch(unpack ? "unpack launch" : "pack launch");
+}
+
+int pack_common(const uint8_t *in, int n_m, int64_t d, int64_t h, uint8_t *outp, bool unpack, void *stream)
+{
+    if (d <= 0 || h <= 0 || !in || !outp)
+        return MGLU_ERR_INVALID;
+    if (!nm_supported(n_m))
+        return MGLU_ERR_UNSUPPORTED;
+    if (d % 8 != 0 || !aligned(unpack ? in : outp, 16))
+        return MGLU_ERR_ALIGN;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    switch (n_m) {
+    case 1: return pack_dispatch<1>(in, d, h, outp, unpack, s);
+    case 2: return pack_dispatch<2>(in, d, h, outp, unpack, s);
+    case 4: return pack_dispatch<4>(in, d, h, outp, unpack, s);
+    default: return pack_dispatch<8>(in, d, h, outp, unpack, s);
+    }
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t mglu_packed_bytes(int n_m, int64_t d, int64_t h)
+{
+    if (!nm_supported(n_m) || d <= 0 || h <= 0)
+        return 0;
+    return (size_t)((h * d * n_m + 7) / 8);
+}
+
+int mglu_pack_masks(const uint8_t *masks, int n_m, int64_t d, int64_t h, uint8_t *packed, void *stream)
+{
+    return pack_common(masks, n_m, d, h, packed, false, stream);
+}
+
+int mglu_unpack_masks(const uint8_t *packed, int n_m, int64_t d, int64_t h, uint8_t *masks, void *stream)
+{
+    return pack_common(packed, n_m, d, h, masks, true, stream);
+}
+
+int mglu_forward(const void *x, int64_t T, int64_t d, const void *W, int64_t h, const uint8_t *packed, int n_m,
+                 int act, int dtype, void *out, void *stream)
+{
+    const int rc = check_forward(x, T, d, W, h, packed, n_m, act, dtype, out);
+    if (rc)
+        return rc;
+    return run_product(x, T, d, W, h, packed, n_m, act, dtype, out, reinterpret_cast<cudaStream_t>(stream));
+}
+
+int mglu_down_proj(const void *hid, int64_t T, int64_t h, const void *W_down, int64_t d, int dtype, void *y,
+                   void *stream)
+{
+    const int rc = check_down(hid, T, h, W_down, d, dtype, y);
+    if (rc)
+        return rc;
+    return run_product(hid, T, h, W_down, d, nullptr, 0, 0, dtype, y, reinterpret_cast<cudaStream_t>(stream));
+}
+
+size_t mglu_workspace_bytes(int64_t T, int64_t d, int64_t h, int n_m, int dtype)
+{
+    (void)d;
+    (void)n_m;
+    if (T < 0 || h <= 0 || (dtype != MGLU_BF16 && dtype != MGLU_F32))
+        return 0;
+    const size_t bytes = (size_t)T * (size_t)h * (dtype == MGLU_BF16 ? 2u : 4u);
+    return (bytes + 255) / 256 * 256;
+}
+
+int mglu_forward_down(const void *x, int64_t T, int64_t d, const void *W, int64_t h, const uint8_t *packed, int n_m,
+                      int act, int dtype, const void *W_down, void *workspace, size_t workspace_bytes, void *y,
+                      void *stream)
+{
+    int rc = check_forward(x, T, d, W, h, packed, n_m, act, dtype, workspace);
+    if (rc)
+        return rc;
+    if ((rc = check_down(workspace, T, h, W_down, d, dtype, y)))
+        return rc;
+    if (T > 0 && (!workspace || workspace_bytes < mglu_workspace_bytes(T, d, h, n_m, dtype)))
+        return MGLU_ERR_INVALID;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if ((rc = run_product(x, T, d, W, h, packed, n_m, act, dtype, workspace, s)))
+        return rc;
+    return run_product(workspace, T, h, W_down, d, nullptr, 0, 0, dtype, y, s);
+}
+
+int mglu_forward_path(int64_t T, int dtype) { return path_for(T, dtype); }
+
+int mglu_set_decode_max_tokens(int t)
+{
+    if (t < 0 || t > 16)
+        return MGLU_ERR_INVALID;
+    const int prev = g_decode_max_tokens;
+    g_decode_max_tokens = t;
+    return prev;
+}
+
+int mglu_last_device_status(void *stream)
+{
+    cudaError_t e = cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess)
+        return cuda_fail(e, "cudaStreamSynchronize");
+    int v = 0;
+    if ((e = cudaMemcpyFromSymbol(&v, mglu::g_status, sizeof(int))) != cudaSuccess)
+        return cuda_fail(e, "read status");
+    if (v != 0) {
+        const int zero = 0;
+        if ((e = cudaMemcpyToSymbol(mglu::g_status, &zero, sizeof(int))) != cudaSuccess)
+            return cuda_fail(e, "clear status");
+    }
+    return v;
+}
+
+const char *mglu_last_cuda_error(void) { return g_last_cuda_error; }
+
+const char *mglu_status_string(int status)
+{
+    switch (status) {
+    case MGLU_OK: return "ok";
+    case MGLU_ERR_INVALID: return "invalid argument";
+    case MGLU_ERR_UNSUPPORTED: return "unsupported n_m";
+    case MGLU_ERR_ALIGN: return "alignment requirement not met";
+    case MGLU_ERR_CUDA: return "CUDA error";
+    case MGLU_ERR_TIMEOUT: return "device wait timed out";
+    default: return "unknown status";
+    }
+}
+
+}  // extern "C"

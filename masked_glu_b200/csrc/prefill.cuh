@@ -1,0 +1,321 @@
+// prefill.cuh -- MGLU up-projection for many tokens on the 5th-generation
+// tensor cores (tcgen05, accumulators in TMEM), and the dense product
+// (NM = 0) used as the prefill down-projection.
+//
+// For many tokens the MGLU forward is a dense contraction: for every token b
+// and column j it needs D = x W and the NM gate products g_i = x (M_i . W).
+// The kernel computes them as ONE matrix product per tile whose B operand is
+// the stack [W; M_1.W; ...; M_NM.W] of NJ weight rows each, so one MMA per
+// k16 step yields every accumulator of the tile and the x tile is read once
+// per step ("Approach" of "Masked Gated Linear Unit": one shared weight
+// matrix, masks split it into gate and value parts; values are D - g_i).
+//
+// Warp roles of the persistent CTA (one per SM):
+//   warp 0      TMA producer: x tile (128 tokens x 64 k), W tile (NJ x 64),
+//               packed-mask tile, into a ring of STAGES shared-memory stages
+//   warp 1      TMEM allocator and the single thread that issues tcgen05.mma
+//   warps 2-5   builders: write the NM masked copies of the W tile next to
+//               it in shared memory (same 128-byte swizzle), then signal
+//   warps 6-9   epilogue: tcgen05.ld the accumulators, out = sum_i
+//               act(g_i)(D - g_i), bf16 stores; overlaps the next tile's
+//               MMAs through a double-buffered accumulator
+#pragma once
+#include <cstdint>
+#include <cuda_bf16.h>
+
+#include "common.cuh"
+#include "ptx.cuh"
+
+namespace mglu {
+namespace pf {
+
+constexpr int BM = 128;  // tokens per tile (UMMA M)
+constexpr int BK = 64;   // k per stage: one 128-byte swizzle atom of bf16
+constexpr int NTHREADS = 320;
+constexpr int TMEM_COLS = 512;
+constexpr int ACC_STRIDE = 256;  // TMEM columns between the two accumulator buffers
+
+template <int NM>
+struct Cfg {
+    // Weight rows per tile: the stacked operand has N = (NM+1)*NJ rows with
+    // N <= 256 and N % 16 == 0 (UMMA shape rule for M = 128); NJ % 8 == 0 so
+    // every variant block starts on an 8-row swizzle boundary.
+    static constexpr int NJ = NM == 0 ? 256 : NM == 1 ? 128 : NM == 2 ? 80 : NM == 4 ? 48 : 16;
+    static constexpr int N = (NM + 1) * NJ;
+    static constexpr int STAGES = NM == 8 ? 5 : 4;
+    static constexpr int A_BYTES = BM * BK * 2;  // 16 KB
+    static constexpr int B_BYTES = N * BK * 2;
+    static constexpr int MB = NM == 0 ? 0 : (BK * NM / 8 < 16 ? 16 : BK * NM / 8);  // mask bytes per row per stage
+    static constexpr int M_BYTES = NJ * MB;
+    static constexpr int STAGE = (A_BYTES + B_BYTES + M_BYTES + 1023) / 1024 * 1024;
+    static constexpr uint32_t TX = A_BYTES + NJ * BK * 2 + M_BYTES;
+    static constexpr int BAR_OFF = STAGES * STAGE;
+    static constexpr int SMEM = BAR_OFF + 256 + 1024;
+    static constexpr int EC = NM >= 8 ? 8 : 16;  // epilogue columns per TMEM load round
+    static_assert(N <= 256 && N % 16 == 0 && NJ % 8 == 0, "bad tile shape");
+    static_assert(NJ % EC == 0, "epilogue chunking");
+    static_assert(SMEM <= 227 * 1024, "shared memory");
+};
+
+template <int NM>
+__device__ __forceinline__ void load_mask_bytes(const uint8_t *p, uint32_t &lo, uint32_t &hi)
+{
+    if constexpr (NM == 8) {
+        const uint2 v = *reinterpret_cast<const uint2 *>(p);
+        lo = v.x;
+        hi = v.y;
+    } else if constexpr (NM == 4) {
+        lo = *reinterpret_cast<const uint32_t *>(p);
+        hi = 0;
+    } else if constexpr (NM == 2) {
+        lo = *reinterpret_cast<const uint16_t *>(p);
+        hi = 0;
+    } else {
+        lo = *p;
+        hi = 0;
+    }
+}
+
+template <int NM, int I>
+__device__ __forceinline__ void build_variants(uint8_t *B, int off, uint4 w, uint32_t lo, uint32_t hi)
+{
+    if constexpr (I < NM) {
+        uint4 m;
+        m.x = w.x & pair_mask<NM, 0, I>(lo, hi);
+        m.y = w.y & pair_mask<NM, 1, I>(lo, hi);
+        m.z = w.z & pair_mask<NM, 2, I>(lo, hi);
+        m.w = w.w & pair_mask<NM, 3, I>(lo, hi);
+        *reinterpret_cast<uint4 *>(B + (1 + I) * Cfg<NM>::NJ * 128 + off) = m;
+        build_variants<NM, I + 1>(B, off, w, lo, hi);
+    }
+}
+
+template <int NM>
+__global__ void __launch_bounds__(NTHREADS, 1) prefill_kernel(const __grid_constant__ CUtensorMap tm_x,
+                                                              const __grid_constant__ CUtensorMap tm_w,
+                                                              const __grid_constant__ CUtensorMap tm_m, int T,
+                                                              int rows, int d, int act,
+                                                              __nv_bfloat16 *__restrict__ out)
+{
+    using C = Cfg<NM>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t *full = reinterpret_cast<uint64_t *>(smem + C::BAR_OFF);
+    uint64_t *built = full + C::STAGES;
+    uint64_t *empty = built + C::STAGES;
+    uint64_t *acc_full = empty + C::STAGES;
+    uint64_t *acc_empty = acc_full + 2;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(acc_empty + 2);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int num_m = (T + BM - 1) / BM;
+    const int num_n = (rows + C::NJ - 1) / C::NJ;
+    const int num_tiles = num_m * num_n;
+    const int nkb = (d + BK - 1) / BK;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < C::STAGES; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&built[s], 4);
+            mbar_init(&empty[s], 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&acc_full[b], 1);
+            mbar_init(&acc_empty[b], 4);
+        }
+        fence_mbar_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_slot, TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+
+    if (warp == 0) {
+        // ---------------------------------------------------------- producer
+        if (lane == 0) {
+            prefetch_tensormap(&tm_x);
+            prefetch_tensormap(&tm_w);
+            if (NM > 0)
+                prefetch_tensormap(&tm_m);
+            int it = 0;
+            bool ok = true;
+            for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+                const int m0 = (tile % num_m) * BM;
+                const int n0 = (tile / num_m) * C::NJ;
+                for (int kb = 0; kb < nkb; ++kb, ++it) {
+                    const int s = it % C::STAGES;
+                    const uint32_t ph = (uint32_t)(it / C::STAGES) & 1u;
+                    if (!mbar_wait(&empty[s], ph ^ 1u)) {
+                        ok = false;
+                        break;
+                    }
+                    uint8_t *st = smem + s * C::STAGE;
+                    mbar_arrive_expect_tx(&full[s], C::TX);
+                    tma_load_2d(st, &tm_x, &full[s], kb * BK, m0);
+                    tma_load_2d(st + C::A_BYTES, &tm_w, &full[s], kb * BK, n0);
+                    if constexpr (NM > 0) {
+                        const int mc = (kb * BK * NM / 8) / C::MB * C::MB;  // 16-byte aligned column
+                        tma_load_2d(st + C::A_BYTES + C::B_BYTES, &tm_m, &full[s], mc, n0);
+                    }
+                }
+            }
+        }
+    } else if (warp == 1) {
+        // ---------------------------------------------------------- MMA issuer
+        if (lane == 0) {
+            constexpr uint32_t idesc = umma_idesc_bf16(BM, C::N);
+            int it = 0, acc_it = 0;
+            bool ok = true;
+            for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x, ++acc_it) {
+                const int b = acc_it & 1;
+                const uint32_t aph = (uint32_t)(acc_it >> 1) & 1u;
+                if (!mbar_wait(&acc_empty[b], aph ^ 1u))
+                    break;
+                tc_fence_after();
+                const uint32_t d_tmem = tmem_base + (uint32_t)(b * ACC_STRIDE);
+                for (int kb = 0; kb < nkb; ++kb, ++it) {
+                    const int s = it % C::STAGES;
+                    const uint32_t ph = (uint32_t)(it / C::STAGES) & 1u;
+                    if (!mbar_wait(NM > 0 ? &built[s] : &full[s], ph)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t a_addr = smem_u32(smem + s * C::STAGE);
+                    const uint32_t b_addr = a_addr + C::A_BYTES;
+#pragma unroll
+                    for (int k16 = 0; k16 < BK / 16; ++k16)
+                        umma_f16_ss(d_tmem, sw128_kmajor_desc(a_addr + k16 * 32), sw128_kmajor_desc(b_addr + k16 * 32),
+                                    idesc, (kb | k16) != 0 ? 1u : 0u);
+                    umma_commit(&empty[s]);
+                }
+                if (ok)
+                    umma_commit(&acc_full[b]);
+            }
+        }
+    } else if (warp < 6) {
+        // ---------------------------------------------------------- builders
+        if constexpr (NM > 0) {
+            const int bt = threadIdx.x - 64;  // 0..127
+            int it = 0;
+            bool ok = true;
+            for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+                for (int kb = 0; kb < nkb; ++kb, ++it) {
+                    const int s = it % C::STAGES;
+                    const uint32_t ph = (uint32_t)(it / C::STAGES) & 1u;
+                    if (!mbar_wait(&full[s], ph)) {
+                        ok = false;
+                        break;
+                    }
+                    uint8_t *B = smem + s * C::STAGE + C::A_BYTES;
+                    const uint8_t *Mt = B + C::B_BYTES;
+                    const int moff = (kb * BK * NM / 8) % C::MB;  // nonzero only when NM = 1
+                    for (int item = bt; item < C::NJ * 8; item += 128) {
+                        const int r = item >> 3, c = item & 7;
+                        const int off = r * 128 + ((c ^ (r & 7)) << 4);
+                        const uint4 w = *reinterpret_cast<const uint4 *>(B + off);
+                        uint32_t lo, hi;
+                        load_mask_bytes<NM>(Mt + r * C::MB + moff + c * NM, lo, hi);
+                        build_variants<NM, 0>(B, off, w, lo, hi);
+                    }
+                    fence_proxy_async_smem();  // generic-proxy writes -> visible to the tensor core
+                    __syncwarp();
+                    if (lane == 0)
+                        mbar_arrive(&built[s]);
+                }
+            }
+        }
+    } else {
+        // ---------------------------------------------------------- epilogue
+        const int q = warp & 3;  // TMEM lane quadrant this warp may access
+        int acc_it = 0;
+        for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++acc_it) {
+            const int b = acc_it & 1;
+            const uint32_t aph = (uint32_t)(acc_it >> 1) & 1u;
+            if (!mbar_wait(&acc_full[b], aph))
+                break;
+            tc_fence_after();
+            const int m0 = (tile % num_m) * BM;
+            const int n0 = (tile / num_m) * C::NJ;
+            const int tok = m0 + 32 * q + lane;
+            const uint32_t tbase = tmem_base + ((uint32_t)(32 * q) << 16) + (uint32_t)(b * ACC_STRIDE);
+            __nv_bfloat16 *orow = out + (int64_t)tok * rows;
+            for (int jc = 0; jc < C::NJ; jc += C::EC) {
+                float o[C::EC];
+                {
+                    uint32_t dv[C::EC];
+#pragma unroll
+                    for (int h8 = 0; h8 < C::EC / 8; ++h8)
+                        tmem_ld_x8(tbase + jc + 8 * h8, *reinterpret_cast<uint32_t(*)[8]>(&dv[8 * h8]));
+                    if constexpr (NM == 0) {
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int e = 0; e < C::EC; ++e)
+                            o[e] = __uint_as_float(dv[e]);
+                    } else {
+                        uint32_t gv[NM][C::EC];
+#pragma unroll
+                        for (int i = 0; i < NM; ++i)
+#pragma unroll
+                            for (int h8 = 0; h8 < C::EC / 8; ++h8)
+                                tmem_ld_x8(tbase + (1 + i) * C::NJ + jc + 8 * h8,
+                                           *reinterpret_cast<uint32_t(*)[8]>(&gv[i][8 * h8]));
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int e = 0; e < C::EC; ++e) {
+                            const float D = __uint_as_float(dv[e]);
+                            float acc = 0.f;
+#pragma unroll
+                            for (int i = 0; i < NM; ++i) {
+                                const float gi = __uint_as_float(gv[i][e]);
+                                acc += act_fn(act, gi) * (D - gi);
+                            }
+                            o[e] = acc;
+                        }
+                    }
+                }
+                if (tok < T) {
+                    const int j = n0 + jc;
+                    if ((rows & 7) == 0 && j + C::EC <= rows) {
+#pragma unroll
+                        for (int e = 0; e < C::EC; e += 8) {
+                            uint4 pk;
+                            __nv_bfloat162 p0 = __floats2bfloat162_rn(o[e + 0], o[e + 1]);
+                            __nv_bfloat162 p1 = __floats2bfloat162_rn(o[e + 2], o[e + 3]);
+                            __nv_bfloat162 p2 = __floats2bfloat162_rn(o[e + 4], o[e + 5]);
+                            __nv_bfloat162 p3 = __floats2bfloat162_rn(o[e + 6], o[e + 7]);
+                            pk.x = *reinterpret_cast<uint32_t *>(&p0);
+                            pk.y = *reinterpret_cast<uint32_t *>(&p1);
+                            pk.z = *reinterpret_cast<uint32_t *>(&p2);
+                            pk.w = *reinterpret_cast<uint32_t *>(&p3);
+                            *reinterpret_cast<uint4 *>(orow + j + e) = pk;
+                        }
+                    } else {
+#pragma unroll
+                        for (int e = 0; e < C::EC; ++e)
+                            if (j + e < rows)
+                                orow[j + e] = __float2bfloat16_rn(o[e]);
+                    }
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0)
+                mbar_arrive(&acc_empty[b]);
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem_base, TMEM_COLS);
+    }
+}
+
+}  // namespace pf
+}  // namespace mglu

@@ -1,0 +1,191 @@
+"""Thin ctypes binding of libmglu.so (see include/mglu.h).
+
+Argument marshalling only: tensors are passed as raw device pointers with the
+current torch stream; every step of the computation runs in the library's
+CUDA kernels.  There is no fallback: if the library is missing, or a call
+fails, an exception is raised.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+from typing import Optional
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libmglu.so")
+HEADER = os.path.join(os.path.dirname(_PKG), "include", "mglu.h")
+
+OK, ERR_INVALID, ERR_UNSUPPORTED, ERR_ALIGN, ERR_CUDA, ERR_TIMEOUT = 0, -1, -2, -3, -4, -5
+ACTS = {"swish": 0, "gelu": 1, "relu": 2}
+DTYPES = {torch.bfloat16: 0, torch.float32: 1}
+PATH_DECODE, PATH_PREFILL, PATH_F32 = 0, 1, 2
+
+_lib = None
+
+
+class MGLUError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        msg = f"{where}: {status_string(status)} ({status})"
+        if status == ERR_CUDA:
+            msg += f": {last_cuda_error()}"
+        super().__init__(msg)
+
+
+def header_functions():
+    """Names of the functions include/mglu.h declares."""
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return re.findall(r"^\s*(?:const\s+)?[a-z_0-9]+\s*\*?\s*(mglu_[a-z_0-9]+)\s*\(", text, flags=re.M)
+
+
+def lib() -> ctypes.CDLL:
+    """Load libmglu.so (built in-tree by ``python -m masked_glu_b200.build``)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: build it with `python -m masked_glu_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        P, I64, I32, SZ = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_size_t
+        sig = {
+            "mglu_packed_bytes": (SZ, [I32, I64, I64]),
+            "mglu_pack_masks": (I32, [P, I32, I64, I64, P, P]),
+            "mglu_unpack_masks": (I32, [P, I32, I64, I64, P, P]),
+            "mglu_forward": (I32, [P, I64, I64, P, I64, P, I32, I32, I32, P, P]),
+            "mglu_down_proj": (I32, [P, I64, I64, P, I64, I32, P, P]),
+            "mglu_workspace_bytes": (SZ, [I64, I64, I64, I32, I32]),
+            "mglu_forward_down": (I32, [P, I64, I64, P, I64, P, I32, I32, I32, P, P, SZ, P, P]),
+            "mglu_forward_path": (I32, [I64, I32]),
+            "mglu_set_decode_max_tokens": (I32, [I32]),
+            "mglu_last_device_status": (I32, [P]),
+            "mglu_last_cuda_error": (ctypes.c_char_p, []),
+            "mglu_status_string": (ctypes.c_char_p, [I32]),
+        }
+        for name, (res, args) in sig.items():
+            f = getattr(L, name)
+            f.restype = res
+            f.argtypes = args
+        _lib = L
+    return _lib
+
+
+def status_string(status: int) -> str:
+    return lib().mglu_status_string(int(status)).decode()
+
+
+def last_cuda_error() -> str:
+    return lib().mglu_last_cuda_error().decode()
+
+
+def _check(rc: int, where: str) -> None:
+    if rc != OK:
+        raise MGLUError(rc, where)
+
+
+def _stream(stream) -> int:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("tensors must be on a CUDA device")
+    if not t.is_contiguous():
+        raise ValueError("tensors must be contiguous")
+    return t.data_ptr()
+
+
+def _dtype(t: torch.Tensor) -> int:
+    if t.dtype not in DTYPES:
+        raise ValueError(f"unsupported dtype {t.dtype}")
+    return DTYPES[t.dtype]
+
+
+def _act(act) -> int:
+    return ACTS[act] if isinstance(act, str) else int(act)
+
+
+def packed_bytes(n_m: int, d: int, h: int) -> int:
+    return int(lib().mglu_packed_bytes(n_m, d, h))
+
+
+def pack_masks(masks: torch.Tensor, stream=None) -> torch.Tensor:
+    """masks [n_m][h][d] uint8 (0/1) on the GPU -> packed uint8 stream."""
+    n_m, h, d = masks.shape
+    out = torch.empty(packed_bytes(n_m, d, h), dtype=torch.uint8, device=masks.device)
+    _check(lib().mglu_pack_masks(_ptr(masks), n_m, d, h, _ptr(out), _stream(stream)), "mglu_pack_masks")
+    return out
+
+
+def unpack_masks(packed: torch.Tensor, n_m: int, d: int, h: int, stream=None) -> torch.Tensor:
+    out = torch.empty((n_m, h, d), dtype=torch.uint8, device=packed.device)
+    _check(lib().mglu_unpack_masks(_ptr(packed), n_m, d, h, _ptr(out), _stream(stream)), "mglu_unpack_masks")
+    return out
+
+
+def forward(x: torch.Tensor, W: torch.Tensor, packed: torch.Tensor, n_m: int, act="swish",
+            out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """out [T][h] = MGLU(x [T][d]) with W [h][d] and packed masks."""
+    T, d = x.shape
+    h = W.shape[0]
+    if W.shape[1] != d or W.dtype != x.dtype:
+        raise ValueError("W must be [h][d] with x's dtype")
+    if out is None:
+        out = torch.empty((T, h), dtype=x.dtype, device=x.device)
+    _check(lib().mglu_forward(_ptr(x), T, d, _ptr(W), h, _ptr(packed), n_m, _act(act), _dtype(x),
+                              _ptr(out), _stream(stream)), "mglu_forward")
+    return out
+
+
+def down_proj(hid: torch.Tensor, W_down: torch.Tensor, out: Optional[torch.Tensor] = None,
+              stream=None) -> torch.Tensor:
+    """y [T][d] = hid [T][h] @ W_down[d][h]^T."""
+    T, h = hid.shape
+    d = W_down.shape[0]
+    if out is None:
+        out = torch.empty((T, d), dtype=hid.dtype, device=hid.device)
+    _check(lib().mglu_down_proj(_ptr(hid), T, h, _ptr(W_down), d, _dtype(hid), _ptr(out), _stream(stream)),
+           "mglu_down_proj")
+    return out
+
+
+def workspace_bytes(T: int, d: int, h: int, n_m: int, dtype=torch.bfloat16) -> int:
+    return int(lib().mglu_workspace_bytes(T, d, h, n_m, DTYPES[dtype]))
+
+
+def forward_down(x: torch.Tensor, W: torch.Tensor, packed: torch.Tensor, n_m: int, W_down: torch.Tensor,
+                 act="swish", workspace: Optional[torch.Tensor] = None, out: Optional[torch.Tensor] = None,
+                 stream=None) -> torch.Tensor:
+    """y = MGLU(x) @ W_down^T through a caller-owned workspace."""
+    T, d = x.shape
+    h = W.shape[0]
+    need = workspace_bytes(T, d, h, n_m, x.dtype)
+    if workspace is None:
+        workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=x.device)
+    if out is None:
+        out = torch.empty((T, d), dtype=x.dtype, device=x.device)
+    _check(lib().mglu_forward_down(_ptr(x), T, d, _ptr(W), h, _ptr(packed), n_m, _act(act), _dtype(x),
+                                   _ptr(W_down), _ptr(workspace), workspace.numel() * workspace.element_size(),
+                                   _ptr(out), _stream(stream)), "mglu_forward_down")
+    return out
+
+
+def forward_path(T: int, dtype=torch.bfloat16) -> int:
+    return int(lib().mglu_forward_path(T, DTYPES[dtype]))
+
+
+def set_decode_max_tokens(t: int) -> int:
+    prev = lib().mglu_set_decode_max_tokens(int(t))
+    if prev < 0:
+        raise MGLUError(prev, "mglu_set_decode_max_tokens")
+    return prev
+
+
+def last_device_status(stream=None) -> int:
+    return int(lib().mglu_last_device_status(_stream(stream)))

@@ -1,0 +1,70 @@
+"""Helpers shared by the GPU parity tests: move seeded cases to the device,
+run the oracle on the same rounded values, compare with the stated bars."""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+import oracle
+from masked_glu_b200 import inputs
+from masked_glu_b200 import mglu
+
+# Parity bars: bf16 inputs with fp32 accumulation, max |err| <= 1e-2 * rms(ref);
+# the fp32 path, max |err| <= 1e-5 * rms(ref).
+TOL = {"bf16": 1e-2, "f32": 1e-5}
+ACT_NAMES = ["swish", "gelu", "relu"]
+GUARD = 64  # guard elements on each side of every output buffer
+
+
+def to_device(t: inputs.Tensor) -> torch.Tensor:
+    if t.dtype == "bf16":
+        return torch.from_numpy(t.storage.view(np.int16)).view(torch.bfloat16).cuda()
+    return torch.from_numpy(t.storage).cuda()
+
+
+def guarded(shape, dtype):
+    """An output buffer with sentinel-filled guard bands on both sides."""
+    n = int(np.prod(shape))
+    big = torch.full((n + 2 * GUARD,), 1234.5, dtype=dtype, device="cuda")
+    return big, big[GUARD:GUARD + n].view(*shape)
+
+
+def check_guards(big):
+    torch.cuda.synchronize()
+    head = big[:GUARD].float().cpu()
+    tail = big[-GUARD:].float().cpu()
+    assert torch.all(head == 1234.5) and torch.all(tail == 1234.5), "write outside the output buffer"
+
+
+def to_f64(t: torch.Tensor) -> np.ndarray:
+    return t.float().cpu().numpy().astype(np.float64)
+
+
+def assert_close(got: np.ndarray, ref: np.ndarray, dtype: str, what: str = ""):
+    rms = float(np.sqrt(np.mean(ref * ref))) if ref.size else 0.0
+    err = float(np.max(np.abs(got - ref))) if ref.size else 0.0
+    bar = TOL[dtype] * rms
+    assert np.all(np.isfinite(got)), f"{what}: non-finite output"
+    assert err <= bar, f"{what}: max|err| {err:.3e} > {TOL[dtype]} * rms {rms:.3e}"
+
+
+def device_case(case: inputs.Case):
+    x = to_device(case.x)
+    W = to_device(case.W)
+    masks = torch.from_numpy(case.masks).cuda()
+    packed = mglu.pack_masks(masks)
+    Wd = to_device(case.W_down) if case.W_down is not None else None
+    return x, W, packed, Wd
+
+
+def oracle_packed(case: inputs.Case) -> np.ndarray:
+    return oracle.pack_masks(case.masks)
+
+
+def run_forward(case: inputs.Case, act: str):
+    x, W, packed, _ = device_case(case)
+    big, out = guarded((case.T, case.h), x.dtype)
+    mglu.forward(x, W, packed, case.n_m, act, out=out)
+    check_guards(big)
+    assert mglu.last_device_status() == 0
+    return to_f64(out)

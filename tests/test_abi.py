@@ -1,0 +1,130 @@
+"""The C ABI without a GPU: the library builds and loads, exports every
+function include/mglu.h declares, and rejects bad arguments with the
+documented status before touching the device."""
+import ctypes
+import os
+import subprocess
+
+import pytest
+
+from masked_glu_b200 import build as mbuild
+from masked_glu_b200 import mglu
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def L():
+    mbuild.build()
+    return mglu.lib()
+
+
+def test_exports_every_declared_symbol(L):
+    names = mglu.header_functions()
+    assert len(names) >= 12
+    for n in names:
+        assert hasattr(L, n), n
+    out = subprocess.run(["nm", "-D", "--defined-only", mglu.LIB_PATH], capture_output=True, text=True).stdout
+    for n in names:
+        assert f" T {n}" in out, n
+
+
+def test_status_strings(L):
+    for s in (0, -1, -2, -3, -4, -5):
+        assert mglu.status_string(s) and mglu.status_string(s) != "unknown status"
+    assert mglu.status_string(7) == "unknown status"
+
+
+def test_sizes(L):
+    assert mglu.packed_bytes(8, 4096, 14336) == 4096 * 14336
+    assert mglu.packed_bytes(4, 2048, 8192) == 2048 * 8192 // 2
+    assert mglu.packed_bytes(1, 8, 3) == 3
+    assert mglu.packed_bytes(3, 8, 3) == 0
+    assert mglu.workspace_bytes(16, 4096, 14336, 8) == 16 * 14336 * 2
+    assert L.mglu_workspace_bytes(3, 64, 100, 8, 1) == (3 * 100 * 4 + 255) // 256 * 256
+
+
+def test_path_choice(L):
+    prev = mglu.set_decode_max_tokens(16)
+    try:
+        assert mglu.forward_path(1) == mglu.PATH_DECODE
+        assert mglu.forward_path(16) == mglu.PATH_DECODE
+        assert mglu.forward_path(17) == mglu.PATH_PREFILL
+        assert L.mglu_forward_path(3, 1) == mglu.PATH_F32
+        assert mglu.set_decode_max_tokens(0) == 16
+        assert mglu.forward_path(1) == mglu.PATH_PREFILL
+        assert L.mglu_set_decode_max_tokens(17) == mglu.ERR_INVALID
+        assert L.mglu_set_decode_max_tokens(-1) == mglu.ERR_INVALID
+    finally:
+        mglu.set_decode_max_tokens(prev)
+
+
+A = 0x10000  # a 16-byte-aligned fake device address: never dereferenced, every call below fails validation
+
+
+def fwd(L, x=A, T=1, d=128, W=A, h=16, pk=A, n_m=8, act=0, dtype=0, out=A):
+    return L.mglu_forward(x, T, d, W, h, pk, n_m, act, dtype, out, None)
+
+
+def test_forward_rejects_bad_arguments(L):
+    assert fwd(L, n_m=3) == mglu.ERR_UNSUPPORTED
+    assert fwd(L, n_m=0) == mglu.ERR_UNSUPPORTED
+    assert fwd(L, n_m=16) == mglu.ERR_UNSUPPORTED
+    assert fwd(L, x=None) == mglu.ERR_INVALID
+    assert fwd(L, W=None) == mglu.ERR_INVALID
+    assert fwd(L, pk=None) == mglu.ERR_INVALID
+    assert fwd(L, out=None) == mglu.ERR_INVALID
+    assert fwd(L, act=3) == mglu.ERR_INVALID
+    assert fwd(L, dtype=2) == mglu.ERR_INVALID
+    assert fwd(L, T=-1) == mglu.ERR_INVALID
+    assert fwd(L, d=0) == mglu.ERR_INVALID
+    assert fwd(L, h=0) == mglu.ERR_INVALID
+    assert fwd(L, d=1 << 31) == mglu.ERR_INVALID
+    # bf16 alignment rules
+    assert fwd(L, x=A + 8) == mglu.ERR_ALIGN
+    assert fwd(L, W=A + 2) == mglu.ERR_ALIGN
+    assert fwd(L, pk=A + 4) == mglu.ERR_ALIGN
+    assert fwd(L, out=A + 8) == mglu.ERR_ALIGN
+    assert fwd(L, d=100) == mglu.ERR_ALIGN             # d % 8
+    assert fwd(L, d=200, n_m=8) == mglu.ERR_ALIGN      # d * n_m % 128
+    assert fwd(L, d=64, n_m=1) == mglu.ERR_ALIGN
+    assert fwd(L, d=80, n_m=4) == mglu.ERR_ALIGN
+    # fp32 path: 4-byte alignment only
+    assert fwd(L, dtype=1, x=A + 2) == mglu.ERR_ALIGN
+
+
+def test_forward_zero_tokens_is_a_noop(L):
+    # T == 0 returns before any device work, even with no x / out
+    assert fwd(L, T=0, x=None, out=None) == mglu.OK
+
+
+def test_down_and_block_reject_bad_arguments(L):
+    assert L.mglu_down_proj(A, 1, 100, A, 64, 0, A, None) == mglu.ERR_ALIGN  # h % 8
+    assert L.mglu_down_proj(None, 1, 128, A, 64, 0, A, None) == mglu.ERR_INVALID
+    assert L.mglu_down_proj(A, 1, 128, A, 64, 5, A, None) == mglu.ERR_INVALID
+    assert L.mglu_down_proj(A, 0, 128, A, 64, 0, None, None) == mglu.OK
+    need = L.mglu_workspace_bytes(4, 128, 64, 8, 0)
+    args = lambda ws, wsb: L.mglu_forward_down(A, 4, 128, A, 64, A, 8, 0, 0, A, ws, wsb, A, None)
+    assert args(A, need - 1) == mglu.ERR_INVALID
+    assert args(None, need) == mglu.ERR_INVALID
+    assert L.mglu_forward_down(A, 4, 128, A, 64, A, 8, 0, 0, None, A, need, A, None) == mglu.ERR_INVALID
+
+
+def test_pack_rejects_bad_arguments(L):
+    assert L.mglu_pack_masks(A, 3, 8, 8, A, None) == mglu.ERR_UNSUPPORTED
+    assert L.mglu_pack_masks(None, 8, 8, 8, A, None) == mglu.ERR_INVALID
+    assert L.mglu_pack_masks(A, 8, 12, 8, A, None) == mglu.ERR_ALIGN
+    assert L.mglu_pack_masks(A, 8, 8, 8, A + 1, None) == mglu.ERR_ALIGN
+    assert L.mglu_unpack_masks(A + 4, 8, 8, 8, A, None) == mglu.ERR_ALIGN
+    assert L.mglu_pack_masks(A, 8, 0, 8, A, None) == mglu.ERR_INVALID
+
+
+def test_mask_expansion_host_check(tmp_path):
+    """The bit -> bf16x2 lane-mask helper the kernels use, compiled for the
+    host (with an emulation of prmt) and checked against the packed-format
+    definition for every n_m, register and mask."""
+    exe = tmp_path / "pair_mask_check"
+    subprocess.run(["g++", "-std=c++17", "-O1", "-I", os.path.join(ROOT, "masked_glu_b200", "csrc"),
+                    "-o", str(exe), os.path.join(ROOT, "tests", "native", "pair_mask_check.cpp")], check=True)
+    r = subprocess.run([str(exe)], capture_output=True, text=True)
+    assert r.returncode == 0 and r.stdout.strip() == "ok", r.stdout

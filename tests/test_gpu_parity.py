@@ -1,0 +1,204 @@
+"""GPU parity: every kernel of libmglu.so against the float64 oracle, through
+the C ABI, on seeded inputs.  Small cases are compared element by element at
+sizes that span several tiles with ragged tails; the full-size workloads are
+compared on exact samples the oracle computes one element at a time."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from masked_glu_b200 import inputs
+from masked_glu_b200 import mglu
+
+from gpu_util import (ACT_NAMES, assert_close, check_guards, device_case, guarded, oracle_packed, run_forward,
+                      to_device, to_f64)
+
+pytestmark = pytest.mark.gpu
+ACT = {"swish": oracle.ACT_SWISH, "gelu": oracle.ACT_GELU, "relu": oracle.ACT_RELU}
+
+
+@pytest.fixture(autouse=True, scope="module")
+def _built():
+    from masked_glu_b200 import build
+    build.build()
+    mglu.set_decode_max_tokens(16)
+
+
+# ------------------------------------------------------------------ packing (bit-exact)
+@pytest.mark.parametrize("n_m,d,h", [(8, 8, 3), (4, 16, 5), (2, 64, 7), (1, 128, 9), (1, 8, 1), (8, 4096, 130),
+                                     (4, 2048, 33), (2, 24, 5), (1, 40, 3)])
+def test_pack_unpack_bit_exact(n_m, d, h):
+    case = inputs.make_case(1, d, h, n_m, seed=7 + d + h + n_m)
+    masks = torch.from_numpy(case.masks).cuda()
+    packed = mglu.pack_masks(masks)
+    want = oracle_packed(case)
+    np.testing.assert_array_equal(packed.cpu().numpy(), want)
+    back = mglu.unpack_masks(packed, n_m, d, h)
+    np.testing.assert_array_equal(back.cpu().numpy(), case.masks)
+
+
+def test_pack_treats_nonzero_as_one():
+    m = torch.tensor([[[0, 7, 255, 1, 0, 0, 2, 0]]], dtype=torch.uint8).cuda()  # n_m=1, h=1, d=8
+    assert mglu.pack_masks(m).cpu().tolist() == [0b01001110]
+
+
+# ------------------------------------------------------------------ fp32 path
+def test_fp32_tiny_full():
+    w = inputs.WORKLOADS["tiny_f32"]
+    case = inputs.make_case(w["T"], w["d"], w["h"], w["n_m"], seed=inputs.WORKLOAD_SEEDS["tiny_f32"], dtype="f32")
+    for act in ACT_NAMES:
+        got = run_forward(case, act)
+        ref, _ = oracle.forward(case.x.values, case.W.values, oracle_packed(case), case.n_m, ACT[act])
+        assert_close(got, ref, "f32", f"fp32 {act}")
+
+
+@pytest.mark.parametrize("n_m,T,d,h", [(8, 9, 100, 37), (1, 3, 13 * 8, 5), (4, 1, 64, 70)])
+def test_fp32_odd_shapes(n_m, T, d, h):
+    case = inputs.make_case(T, d, h, n_m, seed=31 + T + d, dtype="f32")
+    got = run_forward(case, "gelu")
+    ref, _ = oracle.forward(case.x.values, case.W.values, oracle_packed(case), n_m, ACT["gelu"])
+    assert_close(got, ref, "f32", "fp32 odd")
+
+
+def test_fp32_down():
+    rng = np.random.default_rng(5)
+    hid = rng.standard_normal((6, 77)).astype(np.float32)
+    Wd = (rng.standard_normal((45, 77)) * 0.02).astype(np.float32)
+    big, y = guarded((6, 45), torch.float32)
+    mglu.down_proj(torch.from_numpy(hid).cuda(), torch.from_numpy(Wd).cuda(), out=y)
+    check_guards(big)
+    assert_close(to_f64(y), oracle.down(hid.astype(np.float64), Wd.astype(np.float64)), "f32", "fp32 down")
+
+
+# ------------------------------------------------------------------ decode kernel (T <= 16)
+DECODE_CASES = [
+    # n_m, d, h: ragged row block (h % 16 != 0) and ragged k stage (d % 256 != 0)
+    (8, 336, 200),
+    (4, 352, 200),
+    (2, 384, 72),
+    (1, 384, 40),
+    (8, 2048, 256),   # k split over a cluster of 4
+    (8, 4096, 64),    # k split over a cluster of 8
+    (4, 64 * 5, 16),  # one row block, one ragged stage
+]
+
+
+@pytest.mark.parametrize("n_m,d,h", DECODE_CASES)
+@pytest.mark.parametrize("T", [1, 3, 8, 9, 16])
+def test_decode_parity(n_m, d, h, T):
+    case = inputs.make_case(T, d, h, n_m, seed=100 + n_m * 7 + d + h + T)
+    assert mglu.forward_path(T) == mglu.PATH_DECODE
+    got = run_forward(case, "swish")
+    ref, _ = oracle.forward(case.x.values, case.W.values, oracle_packed(case), n_m, ACT["swish"])
+    assert_close(got, ref, "bf16", f"decode n_m={n_m} d={d} h={h} T={T}")
+
+
+@pytest.mark.parametrize("act", ACT_NAMES)
+@pytest.mark.parametrize("n_m", [1, 2, 4, 8])
+def test_decode_acts(act, n_m):
+    case = inputs.make_case(5, 512, 48, n_m, seed=200 + n_m)
+    got = run_forward(case, act)
+    ref, _ = oracle.forward(case.x.values, case.W.values, oracle_packed(case), n_m, ACT[act])
+    assert_close(got, ref, "bf16", f"decode {act}")
+
+
+# ------------------------------------------------------------------ prefill kernel (tcgen05)
+PREFILL_CASES = [
+    # n_m, T, d, h: ragged token tile, ragged weight tile, ragged k stage
+    (4, 17, 320, 200),
+    (4, 129, 320, 200),
+    (4, 300, 256, 100),
+    (8, 129, 336, 40),
+    (8, 200, 512, 72),
+    (2, 150, 384, 170),
+    (1, 130, 384, 300),
+    (1, 40, 256, 128),
+]
+
+
+@pytest.mark.parametrize("n_m,T,d,h", PREFILL_CASES)
+def test_prefill_parity(n_m, T, d, h):
+    case = inputs.make_case(T, d, h, n_m, seed=300 + n_m + T + d + h)
+    assert mglu.forward_path(T) == mglu.PATH_PREFILL
+    got = run_forward(case, "swish")
+    ref, _ = oracle.forward(case.x.values, case.W.values, oracle_packed(case), n_m, ACT["swish"])
+    assert_close(got, ref, "bf16", f"prefill n_m={n_m} T={T} d={d} h={h}")
+
+
+@pytest.mark.parametrize("act", ACT_NAMES)
+def test_prefill_acts(act):
+    case = inputs.make_case(160, 256, 96, 4, seed=401)
+    got = run_forward(case, act)
+    ref, _ = oracle.forward(case.x.values, case.W.values, oracle_packed(case), 4, ACT[act])
+    assert_close(got, ref, "bf16", f"prefill {act}")
+
+
+def test_prefill_many_tiles_per_cta():
+    """More tiles than SMs: each persistent CTA runs several tiles through both
+    accumulator buffers.  Checked on an exact sample of elements."""
+    T, d, h, n_m = 1024, 256, 2048, 4
+    case = inputs.make_case(T, d, h, n_m, seed=402)
+    got = run_forward(case, "swish")
+    rng = np.random.default_rng(3)
+    b = np.concatenate([rng.integers(0, T, 3000), np.repeat([0, T - 1], h)])
+    j = np.concatenate([rng.integers(0, h, 3000), np.tile(np.arange(h), 2)])
+    ref, _ = oracle.forward_elems(case.x.values, case.W.values, oracle_packed(case), n_m, ACT["swish"], b, j)
+    assert_close(got[b, j], ref, "bf16", "prefill many tiles")
+
+
+def test_decode_limit_zero_routes_small_T_to_prefill():
+    case = inputs.make_case(3, 256, 64, 8, seed=403)
+    prev = mglu.set_decode_max_tokens(0)
+    try:
+        assert mglu.forward_path(3) == mglu.PATH_PREFILL
+        got = run_forward(case, "swish")
+    finally:
+        mglu.set_decode_max_tokens(prev)
+    ref, _ = oracle.forward(case.x.values, case.W.values, oracle_packed(case), 8, ACT["swish"])
+    assert_close(got, ref, "bf16", "prefill at T=3")
+
+
+# ------------------------------------------------------------------ exact special cases
+@pytest.mark.parametrize("T", [2, 40])
+def test_single_full_mask_gives_exact_zero(T):
+    """n_m = 1 with every weight in the gate: the value is empty, out == 0."""
+    case = inputs.make_case(T, 256, 48, 1, seed=500 + T)
+    case.masks[:] = 1
+    got = run_forward(case, "swish")
+    assert np.all(got == 0.0)
+
+
+@pytest.mark.parametrize("T", [2, 40])
+@pytest.mark.parametrize("n_m", [2, 8])
+def test_empty_masks_give_exact_zero(T, n_m):
+    case = inputs.make_case(T, 256, 48, n_m, seed=510 + T + n_m)
+    case.masks[:] = 0
+    for act in ACT_NAMES:
+        got = run_forward(case, act)
+        assert np.all(got == 0.0), act
+
+
+# ------------------------------------------------------------------ down-projection and FFN block
+@pytest.mark.parametrize("T,h,d", [(1, 1000, 200), (5, 1000, 200), (16, 14336, 64), (200, 512, 300),
+                                   (17, 136, 40)])
+def test_down_proj(T, h, d):
+    rng = np.random.default_rng(T + h + d)
+    hid = inputs.normal(rng, (T, h), 1.0, "bf16")
+    Wd = inputs.normal(rng, (d, h), 0.02, "bf16")
+    big, y = guarded((T, d), torch.bfloat16)
+    mglu.down_proj(to_device(hid), to_device(Wd), out=y)
+    check_guards(big)
+    assert_close(to_f64(y), oracle.down(hid.values, Wd.values), "bf16", f"down T={T}")
+
+
+@pytest.mark.parametrize("T", [1, 16, 64])
+def test_forward_down_block(T):
+    case = inputs.make_case(T, 256, 1024, 8, seed=600 + T, with_down=True)
+    x, W, packed, Wd = device_case(case)
+    big, y = guarded((T, 256), torch.bfloat16)
+    mglu.forward_down(x, W, packed, 8, Wd, "swish", out=y)
+    check_guards(big)
+    assert mglu.last_device_status() == 0
+    hid, _ = oracle.forward(case.x.values, case.W.values, oracle_packed(case), 8, ACT["swish"])
+    ref = oracle.down(hid, case.W_down.values)
+    assert_close(to_f64(y), ref, "bf16", f"block T={T}")
