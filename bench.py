@@ -1,0 +1,497 @@
+#!/usr/bin/env python
+"""Benchmark of the MGLU forward on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--tokens T]
+    python bench.py --impl reference ...     # the float64 CPU oracle, same workload
+
+A step is one pass of the hot path over one batch: for the decode and prefill
+workloads one ``mglu_forward`` call (mask-bit unpacking, the n_m + 1 products
+and the fused act-sum epilogue); for the FFN-block workload the up-projection
+plus the down-projection.  Mask packing happens once at weight-load time and
+is outside the timed region.  One JSON line is printed by rank 0.
+
+Inputs are seeded synthetic tensors with the workload's shapes.  To keep every
+timed launch reading HBM, each step uses the next of R device copies of
+(W, packed masks[, W_down]) with R * working set > 4 x L2.  Multi-GPU runs are
+independent replicas (each rank its own batch, no collective on the data
+path); timing is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import csv
+import hashlib
+import io
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "MGLU fwd HBM GB/s & tok/s (decode), TFLOP/s (prefill) vs B200 roofline"
+DEFAULT_WORKLOAD = "decode_d2048_h8192_nm4"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+# ---------------------------------------------------------------------- setup
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["mglu", "reference"], default="mglu")
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    ap.add_argument("--tokens", type=int, default=None, help="token count for the sweep workloads")
+    ap.add_argument("--act", default="swish", choices=["swish", "gelu", "relu"])
+    ap.add_argument("--p", type=float, default=0.5, help="mask density (FFN-block workload)")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--probe-seconds", type=float, default=1.0,
+                    help="untimed run of the same step before timing, to settle and sample clocks")
+    return ap.parse_args()
+
+
+def workload_shape(args):
+    from masked_glu_b200 import inputs
+    if args.workload not in inputs.WORKLOADS:
+        raise SystemExit(f"unknown workload {args.workload}; choose from {list(inputs.WORKLOADS)}")
+    w = dict(inputs.WORKLOADS[args.workload])
+    if args.tokens is not None:
+        w["T"] = args.tokens
+    w["kind"] = ("ffn" if args.workload.startswith("ffn") else
+                 "prefill" if args.workload.startswith("prefill") else
+                 "tiny" if args.workload.startswith("tiny") else "decode")
+    w["seed"] = inputs.WORKLOAD_SEEDS[args.workload] + (w["T"] if args.tokens is not None else 0)
+    return w
+
+
+def algorithmic(w):
+    """Roofline work of one step (and of its dominant kernel, the up-projection)."""
+    T, d, h, nm = w["T"], w["d"], w["h"], w["n_m"]
+    esz = 4 if w["dtype"] == "f32" else 2
+    up_bytes = esz * d * h + nm * d * h // 8 + esz * T * d + esz * T * h
+    up_flops = 2 * T * d * h * (nm + 1)
+    down_bytes = esz * h * d + esz * T * h + esz * T * d
+    down_flops = 2 * T * h * d
+    return up_bytes, up_flops, down_bytes, down_flops
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            return json.load(f), "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def kernel_source_hash():
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "masked_glu_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        if name.endswith((".cu", ".cuh")):
+            with open(os.path.join(csrc, name), "rb") as f:
+                h.update(name.encode() + f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(workload, T):
+    """DRAM bytes per launch of the dominant kernel from a committed ncu
+    capture, if the kernel sources have not changed since it was taken."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        rec = json.load(f)
+    e = rec.get(f"{workload}:T{T}")
+    if not e or e.get("source_hash") != kernel_source_hash():
+        return None
+    return e.get("dram_bytes_per_launch")
+
+
+# ---------------------------------------------------------------------- distributed
+class Dist:
+    def __init__(self):
+        self.world = int(os.environ.get("WORLD_SIZE", "1"))
+        self.rank = int(os.environ.get("RANK", "0"))
+        self.local = int(os.environ.get("LOCAL_RANK", "0"))
+        self.pg = False
+
+    def init(self, backend):
+        if self.world > 1:
+            import datetime
+            import torch.distributed as dist
+            os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
+            dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+            self.pg = True
+
+    def barrier(self):
+        if self.pg:
+            import torch.distributed as dist
+            dist.barrier()
+
+    def max(self, v: float, device=None) -> float:
+        if not self.pg:
+            return v
+        import torch
+        import torch.distributed as dist
+        t = torch.tensor([v], dtype=torch.float64, device=device)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    def close(self):
+        if self.pg:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+# ---------------------------------------------------------------------- clocks
+class ClockSampler:
+    """nvidia-smi samples every 100 ms while running (read-only queries)."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,utilization.gpu,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.proc = None
+        self.text = ""
+        self.sel = self._selector(device_index)
+
+    @staticmethod
+    def _selector(i):
+        try:
+            import torch
+            p = torch.cuda.get_device_properties(i)
+            return f"{p.pci_domain_id:08X}:{p.pci_bus_id:02X}:{p.pci_device_id:02X}.0"
+        except Exception:
+            return None
+
+    def start(self):
+        cmd = ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "100"]
+        if self.sel:
+            cmd[1:1] = ["-i", self.sel]
+        try:
+            self.proc = subprocess.Popen(cmd, stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+        self.buf = []
+        if self.proc:
+            self.thread = threading.Thread(target=lambda: self.buf.extend(self.proc.stdout), daemon=True)
+            self.thread.start()
+
+    def stop(self):
+        if not self.proc:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"], "samples": 0}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.thread.join(timeout=5)
+        rows = [r for r in csv.reader(io.StringIO("".join(self.buf))) if len(r) >= 10]
+        load = [r for r in rows if _num(r[4]) and _num(r[4]) > 0] or rows
+        sm = [_num(r[1]) for r in load if _num(r[1])]
+        mx = [_num(r[2]) for r in rows if _num(r[2])]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[k] for r in load for k in range(4) if r[6 + k].strip().lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(load),
+                "power_w_max": max((_num(r[3]) or 0) for r in load) if load else None}
+
+
+def _num(s):
+    try:
+        return float(s)
+    except Exception:
+        return None
+
+
+# ---------------------------------------------------------------------- oracle timing
+def time_oracle(w, budget_s=10.0, max_tokens=None):
+    """Time the float64 oracle on a bounded sample of the workload: whole
+    tokens (every output column of a token), as many as fit in ~budget_s."""
+    import numpy as np
+    import oracle
+    from masked_glu_b200 import inputs
+
+    T = w["T"]
+    rng = np.random.Generator(np.random.PCG64(w["seed"]))
+    d, h, nm = w["d"], w["h"], w["n_m"]
+    W = inputs.normal(rng, (h, d), 0.02, w["dtype"]).values
+    masks = inputs.bernoulli_masks(rng, nm, h, d, w.get("p", 0.5))
+    x = inputs.normal(rng, (1, d), 1.0, w["dtype"]).values
+    pk = oracle.pack_masks(masks)
+    Wd = inputs.normal(rng, (d, h), 0.02, w["dtype"]).values if w["kind"] == "ffn" else None
+    act = {"swish": 0, "gelu": 1, "relu": 2}[w.get("act", "swish")]
+
+    def one_token():
+        out, _ = oracle.forward(x, W, pk, nm, act)
+        if Wd is not None:
+            oracle.down(out, Wd)
+
+    t0 = time.perf_counter()
+    one_token()
+    t1 = time.perf_counter() - t0
+    n = max(1, min(int(budget_s / max(t1, 1e-6)), max_tokens or T))
+    t0 = time.perf_counter()
+    for _ in range(n):
+        one_token()
+    dt = time.perf_counter() - t0
+    cores = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
+    return {"value": n / dt, "unit": "tok/s", "cores": cores, "kind": "oracle",
+            "sample": f"{n} token(s) x all {h} output columns of {w['name']} (d={d}, n_m={nm}), "
+                      f"float64, OpenMP over columns"}, one_token
+
+
+def run_reference(args, dist):
+    """The float64 oracle as it stands, on the host cores (rank 0 only)."""
+    w = workload_shape(args)
+    w["name"], w["act"], w["p"] = args.workload, args.act, args.p
+    if dist.rank != 0:
+        return
+    _, one = time_oracle(w, budget_s=0.5, max_tokens=1)
+    for _ in range(args.warmup):
+        one()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        one()
+    dt = time.perf_counter() - t0
+    tok_s = args.steps / dt
+    cores = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
+    line = {
+        "impl": "reference", "metric": METRIC, "value": tok_s, "unit": "tok/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000 * dt / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": args.workload, "T_per_step": 1, "d": w["d"], "h": w["h"], "n_m": w["n_m"],
+                   "act": args.act},
+        "cpu_baseline": {"value": tok_s, "unit": "tok/s", "cores": cores, "kind": "oracle",
+                         "sample": f"one token (all {w['h']} columns) of {args.workload} per step"},
+        "e2e": {"value": tok_s, "unit": "tok/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------------- GPU run
+def run_mglu(args, dist):
+    import numpy as np
+    import torch
+
+    from masked_glu_b200 import build as mbuild
+    from masked_glu_b200 import inputs, mglu
+
+    if args.warmup < 3:
+        raise SystemExit("--warmup must be >= 3")
+    w = workload_shape(args)
+    w["name"], w["act"], w["p"] = args.workload, args.act, args.p
+    torch.cuda.set_device(dist.local)
+    dev = torch.device("cuda", dist.local)
+    dist.init("nccl")
+    mbuild.build()
+    mglu.lib()
+    mglu.set_decode_max_tokens(16)
+
+    T, d, h, nm = w["T"], w["d"], w["h"], w["n_m"]
+    kind = w["kind"]
+    case = inputs.make_case(T, d, h, nm, seed=w["seed"] + 7919 * dist.rank, p=args.p, dtype=w["dtype"],
+                            with_down=(kind == "ffn"))
+    tdt = torch.float32 if w["dtype"] == "f32" else torch.bfloat16
+
+    def up(t):
+        if t.dtype == "bf16":
+            return torch.from_numpy(t.storage.view(np.int16)).view(torch.bfloat16).to(dev)
+        return torch.from_numpy(t.storage).to(dev)
+
+    x = up(case.x)
+    W0 = up(case.W)
+    pk0 = mglu.pack_masks(torch.from_numpy(case.masks).to(dev))
+    Wd0 = up(case.W_down) if kind == "ffn" else None
+    del case
+    up_bytes, up_flops, down_bytes, down_flops = algorithmic(w)
+    working = up_bytes + (down_bytes if kind == "ffn" else 0)
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    R = max(1, min(16, math.ceil(4 * l2 / max(1, working - 2 * T * (d + h)))))
+    free = torch.cuda.mem_get_info(dev)[0]
+    while R > 1 and R * working > 0.5 * free:
+        R -= 1
+    Ws = [W0] + [W0.clone() for _ in range(R - 1)]
+    pks = [pk0] + [pk0.clone() for _ in range(R - 1)]
+    Wds = ([Wd0] + [Wd0.clone() for _ in range(R - 1)]) if kind == "ffn" else None
+    out = torch.empty((T, h), dtype=tdt, device=dev)
+    y = torch.empty((T, d), dtype=tdt, device=dev) if kind == "ffn" else None
+    ws = (torch.zeros(max(256, mglu.workspace_bytes(T, d, h, nm, tdt)), dtype=torch.uint8, device=dev)
+          if kind == "ffn" else None)
+    scratch = torch.zeros(mglu.scratch_bytes(max(d, h)), dtype=torch.uint8, device=dev)
+    def step(i, ev=None):
+        """One step on the current stream; ev = events bracketing its kernels."""
+        r = i % R
+        if ev is not None:
+            ev[0].record()
+        mglu.forward(x, Ws[r], pks[r], nm, args.act, out=out, scratch=scratch)
+        if ev is not None:
+            ev[1].record()
+        if kind == "ffn":
+            mglu.down_proj(out, Wds[r], out=y, scratch=scratch)
+            if ev is not None:
+                ev[2].record()
+
+    # warm-up (untimed, eager)
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize(dev)
+    if mglu.last_device_status() != 0:
+        raise SystemExit("device status error during warm-up")
+
+    # the K timed steps are captured once as a CUDA graph (launch overhead
+    # out of the way), with event nodes around every kernel for its duration
+    K = args.steps
+    nev = 3 if kind == "ffn" else 2
+    evs = [[torch.cuda.Event(enable_timing=True, external=True) for _ in range(nev)] for _ in range(K)]
+    graph = torch.cuda.CUDAGraph()
+    cap = torch.cuda.Stream(dev)
+    cap.wait_stream(torch.cuda.current_stream(dev))
+    with torch.cuda.graph(graph, stream=cap):
+        for i in range(K):
+            step(i, evs[i])
+    torch.cuda.current_stream(dev).wait_stream(cap)
+    graph.replay()  # one untimed replay
+    torch.cuda.synchronize(dev)
+
+    # an untimed run of the same graph to settle and sample clocks
+    sampler = ClockSampler(dist.local)
+    sampler.start()
+    t_end = time.perf_counter() + args.probe_seconds
+    while time.perf_counter() < t_end:
+        graph.replay()
+        torch.cuda.synchronize(dev)
+
+    # timed region: exactly K steps (one replay of the captured graph)
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    dist.barrier()
+    torch.cuda.synchronize(dev)
+    t0.record()
+    graph.replay()
+    t1.record()
+    torch.cuda.synchronize(dev)
+    dist.barrier()
+    clocks = sampler.stop()
+    status = mglu.last_device_status()
+    total_ms = t0.elapsed_time(t1)
+    up_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
+    down_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in evs) if kind == "ffn" else None
+    total_ms = dist.max(total_ms, dev)
+    up_ms = dist.max(up_ms, dev)
+    ms_per_step = total_ms / K
+    value = dist.world * T * K / (total_ms / 1000.0)
+    del graph
+
+    # end to end: pinned host x in, result out, every step
+    x_h = torch.empty((T, d), dtype=tdt, pin_memory=True)
+    x_h.copy_(x.cpu())
+    res = y if kind == "ffn" else out
+    res_h = torch.empty(res.shape, dtype=tdt, pin_memory=True)
+    x_dev = torch.empty_like(x)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    stream = torch.cuda.current_stream(dev)
+
+    def e2e_step(i):
+        r = i % R
+        x_dev.copy_(x_h, non_blocking=True)
+        if kind == "ffn":
+            mglu.forward_down(x_dev, Ws[r], pks[r], nm, Wds[r], args.act, workspace=ws, out=y)
+        else:
+            mglu.forward(x_dev, Ws[r], pks[r], nm, args.act, out=out, scratch=scratch)
+        res_h.copy_(res, non_blocking=True)
+
+    for i in range(args.warmup):
+        e2e_step(i)
+    torch.cuda.synchronize(dev)
+    # host cost of one public call (no device sync inside the loop)
+    n_host = 50
+    h0 = time.perf_counter()
+    for i in range(n_host):
+        mglu.forward(x, Ws[i % R], pks[i % R], nm, args.act, out=out, scratch=scratch)
+    host_us = (time.perf_counter() - h0) / n_host * 1e6
+    torch.cuda.synchronize(dev)
+    dist.barrier()
+    torch.cuda.synchronize(dev)
+    e0.record(stream)
+    for i in range(K):
+        e2e_step(i)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    dist.barrier()
+    e2e_ms = dist.max(e0.elapsed_time(e1), dev)
+    e2e_value = dist.world * T * K / (e2e_ms / 1000.0)
+
+    peaks, peak_src = load_peaks()
+    if kind in ("decode", "ffn", "tiny") and T <= 16:
+        achieved = up_bytes / (up_ms / 1000.0) / 1e9
+        roof = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": achieved / peaks["hbm_gbs"], "peak_source": f"{peak_src} hbm_gbs (copy)"}
+    else:
+        achieved = up_flops / (up_ms / 1000.0) / 1e12
+        pk = peaks["bf16_tflops"]
+        roof = {"bound": "tensor", "achieved": achieved, "peak": pk, "unit": "TFLOP/s",
+                "frac": achieved / pk, "peak_source": f"{peak_src} bf16_tflops (burst, kernel timed alone)"}
+    roof["traffic"] = recorded_traffic(args.workload, T)
+    roof["kernel"] = "mglu up-projection (decode)" if (T <= 16 and w["dtype"] != "f32") else \
+        "mglu up-projection (tcgen05)" if w["dtype"] != "f32" else "mglu fp32"
+    roof["kernel_us"] = up_ms * 1000.0
+    roof["algorithmic_bytes"] = up_bytes
+    roof["algorithmic_flops"] = up_flops
+
+    line = {
+        "metric": METRIC, "value": value, "unit": "tok/s", "n_gpus": dist.world, "steps": K,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": w["dtype"],
+        "data": "synthetic: x ~ N(0,1), W ~ N(0,0.02^2), Bernoulli(p) masks, seeded PCG64",
+        "config": {"workload": args.workload, "T": T, "d": d, "h": h, "n_m": nm, "act": args.act,
+                   "p": args.p if kind == "ffn" else 0.5,
+                   "l2": f"inputs larger than L2: {R} rotating device copies of W and packed masks"
+                         f"{' and W_down' if kind == 'ffn' else ''} ({R * working / 1e6:.0f} MB vs "
+                         f"{l2 / 1e6:.0f} MB L2)",
+                   "parallelism": "replicas" if dist.world > 1 else "single"},
+        "roofline": roof,
+        "e2e": {"value": e2e_value, "unit": "tok/s", "h2d_bytes_per_step": x_h.numel() * x_h.element_size(),
+                "d2h_bytes_per_step": res_h.numel() * res_h.element_size()},
+        "gpu_launches": K * (2 if kind == "ffn" else 1),
+        "timing": "device-side: one CUDA-graph replay of the K steps, event nodes around each kernel; "
+                  "e2e: eager calls through the Python binding with pinned host copies",
+        "clocks": clocks,
+        "host_us_per_forward_call": host_us,
+        "device_status": status,
+    }
+    if kind == "ffn":
+        line["down_kernel_us"] = down_ms * 1000.0
+        line["down_gbs"] = down_bytes / (down_ms / 1000.0) / 1e9
+    if kind == "prefill" or T > 16:
+        line["tflops"] = up_flops / (up_ms / 1000.0) / 1e12
+    else:
+        line["hbm_gbs"] = up_bytes / (up_ms / 1000.0) / 1e9
+
+    # the CPU oracle on a bounded sample: rank 0, one GPU only
+    if dist.world == 1 and dist.rank == 0 and not args.no_cpu_baseline:
+        cb, _ = time_oracle(w)
+        line["cpu_baseline"] = cb
+    dist.barrier()
+    if dist.rank == 0:
+        print(json.dumps(line), flush=True)
+    dist.close()
+
+
+def main():
+    args = parse_args()
+    dist = Dist()
+    if args.impl == "reference":
+        run_reference(args, dist)
+        return
+    run_mglu(args, dist)
+
+
+if __name__ == "__main__":
+    main()

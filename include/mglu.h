@@ -17,7 +17,9 @@
  *
  * Conventions for every call:
  *  - All tensor pointers are DEVICE pointers owned by the caller.  The library
- *    allocates no device memory on any call declared here.
+ *    allocates no device memory on any call declared here; the little global
+ *    scratch the decode kernel needs is a caller-provided buffer (see
+ *    mglu_scratch_bytes).
  *  - Calls are asynchronous and ordered on `stream` (a cudaStream_t passed as
  *    void*; NULL = the legacy default stream).
  *  - Arguments are checked before anything is launched.  A negative return
@@ -81,9 +83,11 @@ size_t mglu_packed_bytes(int n_m, int64_t d, int64_t h);
  * a byte is weight k (even) and the high nibble weight k+1.  A row of W
  * (fixed j) and its mask bits are therefore tiled alike along k.
  *   masks   in : [n_m][h][d] uint8; any nonzero byte counts as 1.
- *   packed out : mglu_packed_bytes(n_m, d, h) bytes, every byte written.
- * Requirements: d % 8 == 0 (so each byte holds whole weights), packed
- * 16-byte aligned.  Errors: INVALID, UNSUPPORTED, ALIGN, CUDA.
+ *   packed out : mglu_packed_bytes(n_m, d, h) bytes, every byte written
+ *                (unused high bits of a partial last byte are 0).
+ * Requirements: packed 16-byte aligned.  Any d and h are accepted; the bf16
+ * forward additionally needs (d * n_m) % 128 == 0.
+ * Errors: INVALID, UNSUPPORTED, ALIGN, CUDA.
  */
 int mglu_pack_masks(const uint8_t *masks, int n_m, int64_t d, int64_t h,
                     uint8_t *packed, void *stream);
@@ -93,37 +97,54 @@ int mglu_unpack_masks(const uint8_t *packed, int n_m, int64_t d, int64_t h,
                       uint8_t *masks, void *stream);
 
 /*
+ * Bytes of scratch the decode kernel needs for a product with `rows` output
+ * rows (h for mglu_forward, d for mglu_down_proj): partial sums of the row
+ * blocks that two CTAs share, plus one arrival counter per 16 rows (about
+ * 6 MB).  The scratch must be 16-byte aligned and ZERO-FILLED before its
+ * first use (e.g. one cudaMemset); every call that returns leaves it zeroed
+ * again.  Calls that may run concurrently (other streams) need separate
+ * scratch buffers.  Only the decode path touches it: when
+ * mglu_forward_path(T, dtype) is not MGLU_PATH_DECODE it may be NULL.
+ */
+size_t mglu_scratch_bytes(int64_t rows);
+
+/*
  * MGLU up-projection with the act-and-sum epilogue fused: out = MGLU(x).
  * Reads each weight and its mask bits once per pass; for T up to the decode
  * limit (16 by default) one pass serves all tokens; above it a tensor-core
  * (tcgen05) kernel tiles tokens and weights.
  *   x [T][d], W [h][d], packed (from mglu_pack_masks with the same n_m, d, h),
- *   act in mglu_act, dtype in mglu_dtype, out [T][h].
- * Errors: INVALID, UNSUPPORTED, ALIGN, CUDA.
+ *   act in mglu_act, dtype in mglu_dtype, out [T][h],
+ *   scratch / scratch_bytes: see mglu_scratch_bytes(h).
+ * Errors: INVALID (also: scratch missing or too small on the decode path),
+ * UNSUPPORTED, ALIGN, CUDA.
  */
 int mglu_forward(const void *x, int64_t T, int64_t d, const void *W, int64_t h,
                  const uint8_t *packed, int n_m, int act, int dtype, void *out,
-                 void *stream);
+                 void *scratch, size_t scratch_bytes, void *stream);
 
 /*
  * The FFN down-projection alone, a dense product (MGLU replaces only the two
  * GLU projections; "Masked Gated Linear Unit", summary line):
  *   y[b,c] = sum_j hid[b,j] * W_down[c,j]
- *   hid [T][h], W_down [d][h], y [T][d].
+ *   hid [T][h], W_down [d][h], y [T][d], scratch: mglu_scratch_bytes(d).
  * bf16 requirements: 16-byte aligned pointers, h % 8 == 0.
  */
 int mglu_down_proj(const void *hid, int64_t T, int64_t h, const void *W_down,
-                   int64_t d, int dtype, void *y, void *stream);
+                   int64_t d, int dtype, void *y, void *scratch,
+                   size_t scratch_bytes, void *stream);
 
 /* Workspace bytes mglu_forward_down needs: the hidden activation [T][h] in
- * the path's dtype, rounded up to 256 bytes. */
+ * the path's dtype (rounded up to 256 bytes) followed by the decode scratch
+ * for max(d, h) rows.  Zero-fill it before its first use, as for scratch. */
 size_t mglu_workspace_bytes(int64_t T, int64_t d, int64_t h, int n_m, int dtype);
 
 /*
  * The FFN block: y = MGLU(x) W_down^T.  The hidden activation is written to
- * the caller's workspace (dtype of the path; bf16 rounding happens once, as
- * in mglu_forward) and then multiplied by W_down, both on `stream`.
- * workspace_bytes must be >= mglu_workspace_bytes(...) (else INVALID).
+ * the start of the caller's workspace (dtype of the path; bf16 rounding
+ * happens once, as in mglu_forward) and then multiplied by W_down, both on
+ * `stream`.  workspace_bytes must be >= mglu_workspace_bytes(...) (else
+ * INVALID).
  */
 int mglu_forward_down(const void *x, int64_t T, int64_t d, const void *W,
                       int64_t h, const uint8_t *packed, int n_m, int act,

@@ -80,11 +80,38 @@ EncodeTiledFn encode_fn()
     return fn;
 }
 
+// Encoded maps are cached per thread, keyed by every encoding input, so a
+// repeated call (same weights, same activation buffers) skips the encoding.
+struct MapKey {
+    const void *base;
+    uint64_t inner, outer, row_bytes;
+    uint32_t box_inner, box_outer;
+    int dt, sw;
+    bool operator==(const MapKey &o) const
+    {
+        return base == o.base && inner == o.inner && outer == o.outer && row_bytes == o.row_bytes &&
+               box_inner == o.box_inner && box_outer == o.box_outer && dt == o.dt && sw == o.sw;
+    }
+};
+constexpr int kMapCache = 64;
+struct MapCache {
+    MapKey key[kMapCache];
+    CUtensorMap map[kMapCache];
+    int used = 0, next = 0;
+};
+thread_local MapCache g_maps;
+
 // 2-D tensor map: `outer` rows of `inner` elements, rows `row_bytes` apart;
 // box of box_outer rows x box_inner elements; out-of-range reads give zeros.
 int make_map(CUtensorMap *m, CUtensorMapDataType dt, const void *base, uint64_t inner, uint64_t outer,
              uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle sw)
 {
+    const MapKey key{base, inner, outer, row_bytes, box_inner, box_outer, (int)dt, (int)sw};
+    for (int i = 0; i < g_maps.used; ++i)
+        if (g_maps.key[i] == key) {
+            *m = g_maps.map[i];
+            return MGLU_OK;
+        }
     EncodeTiledFn fn = encode_fn();
     if (!fn) {
         snprintf(g_last_cuda_error, sizeof(g_last_cuda_error), "cuTensorMapEncodeTiled unavailable");
@@ -100,6 +127,9 @@ int make_map(CUtensorMap *m, CUtensorMapDataType dt, const void *base, uint64_t 
         snprintf(g_last_cuda_error, sizeof(g_last_cuda_error), "cuTensorMapEncodeTiled failed (%d)", (int)r);
         return MGLU_ERR_CUDA;
     }
+    const int slot = g_maps.used < kMapCache ? g_maps.used++ : (g_maps.next++ % kMapCache);
+    g_maps.key[slot] = key;
+    g_maps.map[slot] = *m;
     return MGLU_OK;
 }
 
@@ -120,18 +150,9 @@ int ensure_smem(int bytes, int dev)
 }
 
 // ------------------------------------------------------------------ decode
-int choose_ksplit(int64_t row_blocks, int nst, int sms)
-{
-    const int64_t target = (int64_t)sms * 8;
-    int ks = 1;
-    while (ks < 8 && row_blocks * ks < target && nst >= 4 * ks)
-        ks *= 2;
-    return ks;
-}
-
 template <int NM, int NT>
 int launch_decode(const void *x, int64_t T, int64_t d, const void *W, int64_t rows, const uint8_t *packed, int act,
-                  void *out, cudaStream_t s)
+                  void *out, void *ws, cudaStream_t s)
 {
     using L = mglu::dec::Layout<NM, NT>;
     int dev = 0, rc = current_device(&dev);
@@ -145,49 +166,40 @@ int launch_decode(const void *x, int64_t T, int64_t d, const void *W, int64_t ro
                        CU_TENSOR_MAP_SWIZZLE_128B)))
         return rc;
     if (NM > 0) {
-        if ((rc = make_map(&tm, CU_TENSOR_MAP_DATA_TYPE_UINT8, packed, d * NM / 8, rows, d * NM / 8,
-                           mglu::dec::KS * NM / 8, mglu::dec::ROWS, CU_TENSOR_MAP_SWIZZLE_NONE)))
+        if ((rc = make_map(&tm, CU_TENSOR_MAP_DATA_TYPE_UINT8, packed, d * NM / 8, rows, d * NM / 8, L::M_BOX,
+                           mglu::dec::ROWS, mglu::dec::mask_swizzle_mode<L::M_BOX>())))
             return rc;
     } else {
         tm = tw;  // not read
     }
-    auto kernel = mglu::dec::decode_kernel<NM, NT>;
     if ((rc = ensure_smem<mglu::dec::decode_kernel<NM, NT>>(L::SMEM, dev)))
         return rc;
     const int64_t rb = (rows + mglu::dec::ROWS - 1) / mglu::dec::ROWS;
-    const int nst = (int)((d + mglu::dec::KS - 1) / mglu::dec::KS);
-    const int ks = choose_ksplit(rb, nst, sm_count(dev));
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)(rb * ks));
-    cfg.blockDim = dim3(mglu::dec::NTHREADS);
-    cfg.dynamicSmemBytes = L::SMEM;
-    cfg.stream = s;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = (unsigned)ks;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = ks > 1 ? 1 : 0;
-    const cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, tw, tx, tm, (int)T, (int)rows, (int)d, ks, act,
-                                             reinterpret_cast<__nv_bfloat16 *>(out));
-    if (e != cudaSuccess)
-        return cuda_fail(e, "decode launch");
+    const int64_t units = rb * ((d + mglu::dec::KS - 1) / mglu::dec::KS);
+    int64_t grid = (int64_t)sm_count(dev) * L::CPS;
+    if (grid > mglu::dec::MAX_CTAS)
+        grid = mglu::dec::MAX_CTAS;
+    if (grid > units)
+        grid = units;
+    float *ws_part = reinterpret_cast<float *>(ws);
+    int *ws_count = reinterpret_cast<int *>(reinterpret_cast<uint8_t *>(ws) + mglu::dec::part_bytes());
+    mglu::dec::decode_kernel<NM, NT><<<(unsigned)grid, mglu::dec::NTHREADS, L::SMEM, s>>>(
+        tw, tx, tm, (int)T, (int)rows, (int)d, act, ws_part, ws_count, reinterpret_cast<__nv_bfloat16 *>(out));
     return check_launch("decode launch");
 }
 
 template <int NM>
 int decode_nt(const void *x, int64_t T, int64_t d, const void *W, int64_t rows, const uint8_t *packed, int act,
-              void *out, cudaStream_t s)
+              void *out, void *ws, cudaStream_t s)
 {
-    return T <= 8 ? launch_decode<NM, 1>(x, T, d, W, rows, packed, act, out, s)
-                  : launch_decode<NM, 2>(x, T, d, W, rows, packed, act, out, s);
+    return T <= 8 ? launch_decode<NM, 1>(x, T, d, W, rows, packed, act, out, ws, s)
+                  : launch_decode<NM, 2>(x, T, d, W, rows, packed, act, out, ws, s);
 }
 
 // ------------------------------------------------------------------ prefill
 template <int NM>
 int launch_prefill(const void *x, int64_t T, int64_t d, const void *W, int64_t rows, const uint8_t *packed, int act,
-                   void *out, cudaStream_t s)
+                   void *out, void *, cudaStream_t s)
 {
     using C = mglu::pf::Cfg<NM>;
     int dev = 0, rc = current_device(&dev);
@@ -220,7 +232,7 @@ int launch_prefill(const void *x, int64_t T, int64_t d, const void *W, int64_t r
 // ------------------------------------------------------------------ fp32
 template <int NM>
 int launch_simt(const void *x, int64_t T, int64_t d, const void *W, int64_t rows, const uint8_t *packed, int act,
-                void *out, cudaStream_t s)
+                void *out, void *, cudaStream_t s)
 {
     const dim3 grid((unsigned)((rows + 7) / 8), (unsigned)((T + mglu::kSimtTokens - 1) / mglu::kSimtTokens));
     if (grid.y > 65535u)
@@ -271,15 +283,29 @@ int path_for(int64_t T, int dtype)
 // One product of the library: out[T][rows] from x[T][d] and W[rows][d] with
 // n_m masks (n_m = 0: dense).  Arguments already validated.
 int run_product(const void *x, int64_t T, int64_t d, const void *W, int64_t rows, const uint8_t *packed, int n_m,
-                int act, int dtype, void *out, cudaStream_t s)
+                int act, int dtype, void *out, void *ws, cudaStream_t s)
 {
     if (T == 0)
         return MGLU_OK;
     switch (path_for(T, dtype)) {
-    case MGLU_PATH_F32: return by_nm<SimtF>(n_m, x, T, d, W, rows, packed, act, out, s);
-    case MGLU_PATH_DECODE: return by_nm<DecodeF>(n_m, x, T, d, W, rows, packed, act, out, s);
-    default: return by_nm<PrefillF>(n_m, x, T, d, W, rows, packed, act, out, s);
+    case MGLU_PATH_F32: return by_nm<SimtF>(n_m, x, T, d, W, rows, packed, act, out, ws, s);
+    case MGLU_PATH_DECODE: return by_nm<DecodeF>(n_m, x, T, d, W, rows, packed, act, out, ws, s);
+    default: return by_nm<PrefillF>(n_m, x, T, d, W, rows, packed, act, out, ws, s);
     }
+}
+
+size_t scratch_bytes(int64_t rows) { return rows > 0 ? (size_t)mglu::dec::workspace_bytes(rows) : 0; }
+
+// The decode kernel needs its scratch; other paths ignore it.
+int check_scratch(int64_t T, int dtype, int64_t rows, const void *ws, size_t ws_bytes)
+{
+    if (T == 0 || path_for(T, dtype) != MGLU_PATH_DECODE)
+        return MGLU_OK;
+    if (!ws || ws_bytes < scratch_bytes(rows))
+        return MGLU_ERR_INVALID;
+    if (!aligned(ws, 16))
+        return MGLU_ERR_ALIGN;
+    return MGLU_OK;
 }
 
 bool sizes_ok(int64_t T, int64_t d, int64_t h)
@@ -338,7 +364,7 @@ template <int NM>
 int pack_dispatch(const uint8_t *in, int64_t d, int64_t h, uint8_t *outp, bool unpack, cudaStream_t s)
 {
     const int64_t hd = h * d;
-    const int64_t nbytes = hd * NM / 8;
+    const int64_t nbytes = (hd * NM + 7) / 8;
     const int64_t chunks = (nbytes + 15) / 16;
     const int vec = (hd % 16 == 0) && aligned(unpack ? outp : in, 16);
     const int64_t blocks = (chunks + 255) / 256;
@@ -357,8 +383,10 @@ int pack_common(const uint8_t *in, int n_m, int64_t d, int64_t h, uint8_t *outp,
         return MGLU_ERR_INVALID;
     if (!nm_supported(n_m))
         return MGLU_ERR_UNSUPPORTED;
-    if (d % 8 != 0 || !aligned(unpack ? in : outp, 16))
+    if (!aligned(unpack ? in : outp, 16))
         return MGLU_ERR_ALIGN;
+    if (h > ((int64_t)1 << 62) / d)
+        return MGLU_ERR_INVALID;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     switch (n_m) {
     case 1: return pack_dispatch<1>(in, d, h, outp, unpack, s);
@@ -389,32 +417,37 @@ int mglu_unpack_masks(const uint8_t *packed, int n_m, int64_t d, int64_t h, uint
     return pack_common(packed, n_m, d, h, masks, true, stream);
 }
 
+size_t mglu_scratch_bytes(int64_t rows) { return scratch_bytes(rows); }
+
 int mglu_forward(const void *x, int64_t T, int64_t d, const void *W, int64_t h, const uint8_t *packed, int n_m,
-                 int act, int dtype, void *out, void *stream)
+                 int act, int dtype, void *out, void *scratch, size_t scratch_bytes_, void *stream)
 {
-    const int rc = check_forward(x, T, d, W, h, packed, n_m, act, dtype, out);
+    int rc = check_forward(x, T, d, W, h, packed, n_m, act, dtype, out);
     if (rc)
         return rc;
-    return run_product(x, T, d, W, h, packed, n_m, act, dtype, out, reinterpret_cast<cudaStream_t>(stream));
+    if ((rc = check_scratch(T, dtype, h, scratch, scratch_bytes_)))
+        return rc;
+    return run_product(x, T, d, W, h, packed, n_m, act, dtype, out, scratch, reinterpret_cast<cudaStream_t>(stream));
 }
 
 int mglu_down_proj(const void *hid, int64_t T, int64_t h, const void *W_down, int64_t d, int dtype, void *y,
-                   void *stream)
+                   void *scratch, size_t scratch_bytes_, void *stream)
 {
-    const int rc = check_down(hid, T, h, W_down, d, dtype, y);
+    int rc = check_down(hid, T, h, W_down, d, dtype, y);
     if (rc)
         return rc;
-    return run_product(hid, T, h, W_down, d, nullptr, 0, 0, dtype, y, reinterpret_cast<cudaStream_t>(stream));
+    if ((rc = check_scratch(T, dtype, d, scratch, scratch_bytes_)))
+        return rc;
+    return run_product(hid, T, h, W_down, d, nullptr, 0, 0, dtype, y, scratch, reinterpret_cast<cudaStream_t>(stream));
 }
 
 size_t mglu_workspace_bytes(int64_t T, int64_t d, int64_t h, int n_m, int dtype)
 {
-    (void)d;
     (void)n_m;
-    if (T < 0 || h <= 0 || (dtype != MGLU_BF16 && dtype != MGLU_F32))
+    if (T < 0 || d <= 0 || h <= 0 || (dtype != MGLU_BF16 && dtype != MGLU_F32))
         return 0;
-    const size_t bytes = (size_t)T * (size_t)h * (dtype == MGLU_BF16 ? 2u : 4u);
-    return (bytes + 255) / 256 * 256;
+    const size_t hid = ((size_t)T * (size_t)h * (dtype == MGLU_BF16 ? 2u : 4u) + 255) / 256 * 256;
+    return hid + scratch_bytes(d > h ? d : h);
 }
 
 int mglu_forward_down(const void *x, int64_t T, int64_t d, const void *W, int64_t h, const uint8_t *packed, int n_m,
@@ -428,10 +461,14 @@ int mglu_forward_down(const void *x, int64_t T, int64_t d, const void *W, int64_
         return rc;
     if (T > 0 && (!workspace || workspace_bytes < mglu_workspace_bytes(T, d, h, n_m, dtype)))
         return MGLU_ERR_INVALID;
+    if (T == 0)
+        return MGLU_OK;
+    const size_t hid = ((size_t)T * (size_t)h * (dtype == MGLU_BF16 ? 2u : 4u) + 255) / 256 * 256;
+    void *scratch = reinterpret_cast<uint8_t *>(workspace) + hid;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    if ((rc = run_product(x, T, d, W, h, packed, n_m, act, dtype, workspace, s)))
+    if ((rc = run_product(x, T, d, W, h, packed, n_m, act, dtype, workspace, scratch, s)))
         return rc;
-    return run_product(workspace, T, h, W_down, d, nullptr, 0, 0, dtype, y, s);
+    return run_product(workspace, T, h, W_down, d, nullptr, 0, 0, dtype, y, scratch, s);
 }
 
 int mglu_forward_path(int64_t T, int dtype) { return path_for(T, dtype); }

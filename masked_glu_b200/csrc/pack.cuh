@@ -13,7 +13,9 @@ namespace mglu {
 
 // One thread writes one 16-byte chunk of the packed stream (128 / NM
 // weights, every mask plane read once).  `vec` selects 16-byte loads of the
-// mask planes (needs (h*d) % 16 == 0 and a 16-byte aligned `masks`).
+// mask planes (needs (h*d) % 16 == 0 and a 16-byte aligned `masks`).  The
+// last byte may be partial when h*d*NM is not a multiple of 8; its unused
+// high bits are written as 0.
 template <int NM>
 __global__ void __launch_bounds__(256) pack_kernel(const uint8_t *__restrict__ masks, int64_t hd, int64_t nbytes,
                                                    uint8_t *__restrict__ packed, int vec)
@@ -25,7 +27,7 @@ __global__ void __launch_bounds__(256) pack_kernel(const uint8_t *__restrict__ m
         return;
     const int nb = (int)(nbytes - b0 < 16 ? nbytes - b0 : 16);
     const int64_t w0 = b0 * WPB;
-    const int nw = nb * WPB;
+    const int nw = (int)(hd - w0 < (int64_t)nb * WPB ? hd - w0 : (int64_t)nb * WPB);
     uint32_t word[4] = {0u, 0u, 0u, 0u};
     if (vec && nb == 16) {
 #pragma unroll
@@ -73,7 +75,7 @@ __global__ void __launch_bounds__(256) unpack_kernel(const uint8_t *__restrict__
         return;
     const int nb = (int)(nbytes - b0 < 16 ? nbytes - b0 : 16);
     const int64_t w0 = b0 * WPB;
-    const int nw = nb * WPB;
+    const int nw = (int)(hd - w0 < (int64_t)nb * WPB ? hd - w0 : (int64_t)nb * WPB);
     uint32_t word[4] = {0u, 0u, 0u, 0u};
     if (nb == 16) {
         const uint4 v = *reinterpret_cast<const uint4 *>(packed + b0);

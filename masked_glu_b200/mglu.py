@@ -54,8 +54,9 @@ def lib() -> ctypes.CDLL:
             "mglu_packed_bytes": (SZ, [I32, I64, I64]),
             "mglu_pack_masks": (I32, [P, I32, I64, I64, P, P]),
             "mglu_unpack_masks": (I32, [P, I32, I64, I64, P, P]),
-            "mglu_forward": (I32, [P, I64, I64, P, I64, P, I32, I32, I32, P, P]),
-            "mglu_down_proj": (I32, [P, I64, I64, P, I64, I32, P, P]),
+            "mglu_scratch_bytes": (SZ, [I64]),
+            "mglu_forward": (I32, [P, I64, I64, P, I64, P, I32, I32, I32, P, P, SZ, P]),
+            "mglu_down_proj": (I32, [P, I64, I64, P, I64, I32, P, P, SZ, P]),
             "mglu_workspace_bytes": (SZ, [I64, I64, I64, I32, I32]),
             "mglu_forward_down": (I32, [P, I64, I64, P, I64, P, I32, I32, I32, P, P, SZ, P, P]),
             "mglu_forward_path": (I32, [I64, I32]),
@@ -94,10 +95,8 @@ def _stream(stream) -> int:
 def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:
     if t is None:
         return None
-    if not t.is_cuda:
-        raise ValueError("tensors must be on a CUDA device")
-    if not t.is_contiguous():
-        raise ValueError("tensors must be contiguous")
+    if not (t.is_cuda and t.is_contiguous()):
+        raise ValueError("tensors must be contiguous and on a CUDA device")
     return t.data_ptr()
 
 
@@ -129,8 +128,34 @@ def unpack_masks(packed: torch.Tensor, n_m: int, d: int, h: int, stream=None) ->
     return out
 
 
+def scratch_bytes(rows: int) -> int:
+    return int(lib().mglu_scratch_bytes(rows))
+
+
+_scratch = {}
+
+
+def default_scratch(rows: int, device) -> torch.Tensor:
+    """A zero-filled scratch buffer per device, grown on demand and shared by
+    calls that pass none.  Calls on several streams at once must pass their
+    own buffers (the decode kernel's counters are not safe to share)."""
+    dev = torch.device(device)
+    key = dev.index if dev.index is not None else torch.cuda.current_device()
+    need = scratch_bytes(rows)
+    buf = _scratch.get(key)
+    if buf is None or buf.numel() < need:
+        buf = torch.zeros(need, dtype=torch.uint8, device=dev)
+        _scratch[key] = buf
+    return buf
+
+
+def _nbytes(t: Optional[torch.Tensor]) -> int:
+    return 0 if t is None else t.numel() * t.element_size()
+
+
 def forward(x: torch.Tensor, W: torch.Tensor, packed: torch.Tensor, n_m: int, act="swish",
-            out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+            out: Optional[torch.Tensor] = None, scratch: Optional[torch.Tensor] = None,
+            stream=None) -> torch.Tensor:
     """out [T][h] = MGLU(x [T][d]) with W [h][d] and packed masks."""
     T, d = x.shape
     h = W.shape[0]
@@ -138,20 +163,24 @@ def forward(x: torch.Tensor, W: torch.Tensor, packed: torch.Tensor, n_m: int, ac
         raise ValueError("W must be [h][d] with x's dtype")
     if out is None:
         out = torch.empty((T, h), dtype=x.dtype, device=x.device)
+    if scratch is None:
+        scratch = default_scratch(h, x.device)
     _check(lib().mglu_forward(_ptr(x), T, d, _ptr(W), h, _ptr(packed), n_m, _act(act), _dtype(x),
-                              _ptr(out), _stream(stream)), "mglu_forward")
+                              _ptr(out), _ptr(scratch), _nbytes(scratch), _stream(stream)), "mglu_forward")
     return out
 
 
 def down_proj(hid: torch.Tensor, W_down: torch.Tensor, out: Optional[torch.Tensor] = None,
-              stream=None) -> torch.Tensor:
+              scratch: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
     """y [T][d] = hid [T][h] @ W_down[d][h]^T."""
     T, h = hid.shape
     d = W_down.shape[0]
     if out is None:
         out = torch.empty((T, d), dtype=hid.dtype, device=hid.device)
-    _check(lib().mglu_down_proj(_ptr(hid), T, h, _ptr(W_down), d, _dtype(hid), _ptr(out), _stream(stream)),
-           "mglu_down_proj")
+    if scratch is None:
+        scratch = default_scratch(d, hid.device)
+    _check(lib().mglu_down_proj(_ptr(hid), T, h, _ptr(W_down), d, _dtype(hid), _ptr(out), _ptr(scratch),
+                                _nbytes(scratch), _stream(stream)), "mglu_down_proj")
     return out
 
 
@@ -167,7 +196,7 @@ def forward_down(x: torch.Tensor, W: torch.Tensor, packed: torch.Tensor, n_m: in
     h = W.shape[0]
     need = workspace_bytes(T, d, h, n_m, x.dtype)
     if workspace is None:
-        workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=x.device)
+        workspace = torch.zeros(max(need, 256), dtype=torch.uint8, device=x.device)
     if out is None:
         out = torch.empty((T, d), dtype=x.dtype, device=x.device)
     _check(lib().mglu_forward_down(_ptr(x), T, d, _ptr(W), h, _ptr(packed), n_m, _act(act), _dtype(x),

@@ -40,8 +40,8 @@ def test_sizes(L):
     assert mglu.packed_bytes(4, 2048, 8192) == 2048 * 8192 // 2
     assert mglu.packed_bytes(1, 8, 3) == 3
     assert mglu.packed_bytes(3, 8, 3) == 0
-    assert mglu.workspace_bytes(16, 4096, 14336, 8) == 16 * 14336 * 2
-    assert L.mglu_workspace_bytes(3, 64, 100, 8, 1) == (3 * 100 * 4 + 255) // 256 * 256
+    assert mglu.workspace_bytes(16, 4096, 14336, 8) == 16 * 14336 * 2 + L.mglu_scratch_bytes(14336)
+    assert L.mglu_workspace_bytes(3, 64, 100, 8, 1) == (3 * 100 * 4 + 255) // 256 * 256 + L.mglu_scratch_bytes(100)
 
 
 def test_path_choice(L):
@@ -62,8 +62,8 @@ def test_path_choice(L):
 A = 0x10000  # a 16-byte-aligned fake device address: never dereferenced, every call below fails validation
 
 
-def fwd(L, x=A, T=1, d=128, W=A, h=16, pk=A, n_m=8, act=0, dtype=0, out=A):
-    return L.mglu_forward(x, T, d, W, h, pk, n_m, act, dtype, out, None)
+def fwd(L, x=A, T=1, d=128, W=A, h=16, pk=A, n_m=8, act=0, dtype=0, out=A, ws=A, wsb=1 << 30):
+    return L.mglu_forward(x, T, d, W, h, pk, n_m, act, dtype, out, ws, wsb, None)
 
 
 def test_forward_rejects_bad_arguments(L):
@@ -91,6 +91,13 @@ def test_forward_rejects_bad_arguments(L):
     assert fwd(L, d=80, n_m=4) == mglu.ERR_ALIGN
     # fp32 path: 4-byte alignment only
     assert fwd(L, dtype=1, x=A + 2) == mglu.ERR_ALIGN
+    # decode scratch: required (and sized for h) on the decode path only
+    need = L.mglu_scratch_bytes(16)
+    assert need > 0
+    assert fwd(L, ws=None) == mglu.ERR_INVALID
+    assert fwd(L, wsb=need - 1) == mglu.ERR_INVALID
+    assert fwd(L, ws=A + 8, wsb=need) == mglu.ERR_ALIGN
+    assert L.mglu_scratch_bytes(14336) > L.mglu_scratch_bytes(16)
 
 
 def test_forward_zero_tokens_is_a_noop(L):
@@ -99,10 +106,12 @@ def test_forward_zero_tokens_is_a_noop(L):
 
 
 def test_down_and_block_reject_bad_arguments(L):
-    assert L.mglu_down_proj(A, 1, 100, A, 64, 0, A, None) == mglu.ERR_ALIGN  # h % 8
-    assert L.mglu_down_proj(None, 1, 128, A, 64, 0, A, None) == mglu.ERR_INVALID
-    assert L.mglu_down_proj(A, 1, 128, A, 64, 5, A, None) == mglu.ERR_INVALID
-    assert L.mglu_down_proj(A, 0, 128, A, 64, 0, None, None) == mglu.OK
+    big = 1 << 30
+    assert L.mglu_down_proj(A, 1, 100, A, 64, 0, A, A, big, None) == mglu.ERR_ALIGN  # h % 8
+    assert L.mglu_down_proj(None, 1, 128, A, 64, 0, A, A, big, None) == mglu.ERR_INVALID
+    assert L.mglu_down_proj(A, 1, 128, A, 64, 5, A, A, big, None) == mglu.ERR_INVALID
+    assert L.mglu_down_proj(A, 1, 128, A, 64, 0, A, None, 0, None) == mglu.ERR_INVALID  # decode needs scratch
+    assert L.mglu_down_proj(A, 0, 128, A, 64, 0, None, None, 0, None) == mglu.OK
     need = L.mglu_workspace_bytes(4, 128, 64, 8, 0)
     args = lambda ws, wsb: L.mglu_forward_down(A, 4, 128, A, 64, A, 8, 0, 0, A, ws, wsb, A, None)
     assert args(A, need - 1) == mglu.ERR_INVALID
@@ -113,7 +122,6 @@ def test_down_and_block_reject_bad_arguments(L):
 def test_pack_rejects_bad_arguments(L):
     assert L.mglu_pack_masks(A, 3, 8, 8, A, None) == mglu.ERR_UNSUPPORTED
     assert L.mglu_pack_masks(None, 8, 8, 8, A, None) == mglu.ERR_INVALID
-    assert L.mglu_pack_masks(A, 8, 12, 8, A, None) == mglu.ERR_ALIGN
     assert L.mglu_pack_masks(A, 8, 8, 8, A + 1, None) == mglu.ERR_ALIGN
     assert L.mglu_unpack_masks(A + 4, 8, 8, 8, A, None) == mglu.ERR_ALIGN
     assert L.mglu_pack_masks(A, 8, 0, 8, A, None) == mglu.ERR_INVALID

@@ -26,7 +26,8 @@ def _built():
 
 # ------------------------------------------------------------------ packing (bit-exact)
 @pytest.mark.parametrize("n_m,d,h", [(8, 8, 3), (4, 16, 5), (2, 64, 7), (1, 128, 9), (1, 8, 1), (8, 4096, 130),
-                                     (4, 2048, 33), (2, 24, 5), (1, 40, 3)])
+                                     (4, 2048, 33), (2, 24, 5), (1, 40, 3), (1, 13, 3), (2, 5, 7), (4, 100, 37),
+                                     (8, 100, 37)])
 def test_pack_unpack_bit_exact(n_m, d, h):
     case = inputs.make_case(1, d, h, n_m, seed=7 + d + h + n_m)
     masks = torch.from_numpy(case.masks).cuda()
@@ -201,4 +202,22 @@ def test_forward_down_block(T):
     assert mglu.last_device_status() == 0
     hid, _ = oracle.forward(case.x.values, case.W.values, oracle_packed(case), 8, ACT["swish"])
     ref = oracle.down(hid, case.W_down.values)
-    assert_close(to_f64(y), ref, "bf16", f"block T={T}")
+    # the hidden activation is rounded to bf16 before the down-projection, so
+    # y is not the oracle's y rounded once: value bar only
+    assert_close(to_f64(y), ref, "bf16", f"block T={T}", exact_check=False)
+
+
+@pytest.mark.parametrize("T", [1, 9])
+def test_decode_scratch_is_left_zeroed(T):
+    """Row blocks split between CTAs go through the scratch counters; every
+    call must leave them at zero for the next one."""
+    case = inputs.make_case(T, 2048, 256, 8, seed=700 + T)
+    x, W, packed, _ = device_case(case)
+    scratch = torch.zeros(mglu.scratch_bytes(256), dtype=torch.uint8, device="cuda")
+    outs = []
+    for _ in range(3):
+        outs.append(to_f64(mglu.forward(x, W, packed, 8, "swish", scratch=scratch)))
+        torch.cuda.synchronize()
+        counters = scratch[mglu.scratch_bytes(256) - 256:].cpu().numpy()
+        assert not counters.any(), "scratch counters not reset"
+    assert np.array_equal(outs[0], outs[1]) and np.array_equal(outs[1], outs[2]), "run-to-run difference"
