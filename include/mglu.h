@@ -36,9 +36,9 @@
  *        y       [T][d]
  *  - bf16 path (dtype MGLU_BF16): x, W, out, W_down, y are bf16; products are
  *    exact and accumulate in fp32; the result is rounded to bf16 once.
- *    Requirements (else MGLU_ERR_ALIGN): every pointer 16-byte aligned,
- *    d % 8 == 0 and (d * n_m) % 128 == 0, so that a row of W and a row of
- *    packed mask bytes both start on a 16-byte boundary.
+ *    Requirements (else MGLU_ERR_ALIGN): every pointer 16-byte aligned and
+ *    d % 128 == 0 (rows of W and of packed mask bits are then moved in whole
+ *    128-element pieces; Llama-style FFN widths satisfy it).
  *  - fp32 path (dtype MGLU_F32): x, W, out, W_down, y are float; plain fp32
  *    FMA on CUDA cores (never TF32); any d, h; 4-byte aligned pointers.
  *  - Supported n_m: 1, 2, 4, 8 (else MGLU_ERR_UNSUPPORTED).  T == 0 is a
@@ -86,7 +86,7 @@ size_t mglu_packed_bytes(int n_m, int64_t d, int64_t h);
  *   packed out : mglu_packed_bytes(n_m, d, h) bytes, every byte written
  *                (unused high bits of a partial last byte are 0).
  * Requirements: packed 16-byte aligned.  Any d and h are accepted; the bf16
- * forward additionally needs (d * n_m) % 128 == 0.
+ * forward additionally needs d % 128 == 0.
  * Errors: INVALID, UNSUPPORTED, ALIGN, CUDA.
  */
 int mglu_pack_masks(const uint8_t *masks, int n_m, int64_t d, int64_t h,
@@ -128,7 +128,7 @@ int mglu_forward(const void *x, int64_t T, int64_t d, const void *W, int64_t h,
  * GLU projections; "Masked Gated Linear Unit", summary line):
  *   y[b,c] = sum_j hid[b,j] * W_down[c,j]
  *   hid [T][h], W_down [d][h], y [T][d], scratch: mglu_scratch_bytes(d).
- * bf16 requirements: 16-byte aligned pointers, h % 8 == 0.
+ * bf16 requirements: 16-byte aligned pointers, h % 64 == 0.
  */
 int mglu_down_proj(const void *hid, int64_t T, int64_t h, const void *W_down,
                    int64_t d, int dtype, void *y, void *scratch,

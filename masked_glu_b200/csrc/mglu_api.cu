@@ -84,14 +84,10 @@ EncodeTiledFn encode_fn()
 // repeated call (same weights, same activation buffers) skips the encoding.
 struct MapKey {
     const void *base;
-    uint64_t inner, outer, row_bytes;
-    uint32_t box_inner, box_outer;
-    int dt, sw;
-    bool operator==(const MapKey &o) const
-    {
-        return base == o.base && inner == o.inner && outer == o.outer && row_bytes == o.row_bytes &&
-               box_inner == o.box_inner && box_outer == o.box_outer && dt == o.dt && sw == o.sw;
-    }
+    uint64_t dims[3], strides[2];
+    uint32_t box[3];
+    int rank, dt, sw;
+    bool operator==(const MapKey &o) const { return memcmp(this, &o, sizeof(MapKey)) == 0; }
 };
 constexpr int kMapCache = 64;
 struct MapCache {
@@ -101,12 +97,23 @@ struct MapCache {
 };
 thread_local MapCache g_maps;
 
-// 2-D tensor map: `outer` rows of `inner` elements, rows `row_bytes` apart;
-// box of box_outer rows x box_inner elements; out-of-range reads give zeros.
-int make_map(CUtensorMap *m, CUtensorMapDataType dt, const void *base, uint64_t inner, uint64_t outer,
-             uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle sw)
+// Tensor map of rank 2 or 3 (dims innermost first, strides in bytes for
+// dims 1..rank-1, box in elements); out-of-range reads give zeros.
+int make_map_n(CUtensorMap *m, CUtensorMapDataType dt, const void *base, int rank, const uint64_t *dims,
+               const uint64_t *strides, const uint32_t *box, CUtensorMapSwizzle sw)
 {
-    const MapKey key{base, inner, outer, row_bytes, box_inner, box_outer, (int)dt, (int)sw};
+    MapKey key;
+    memset(&key, 0, sizeof(key));
+    key.base = base;
+    key.rank = rank;
+    key.dt = (int)dt;
+    key.sw = (int)sw;
+    for (int i = 0; i < rank; ++i) {
+        key.dims[i] = dims[i];
+        key.box[i] = box[i];
+        if (i + 1 < rank)
+            key.strides[i] = strides[i];
+    }
     for (int i = 0; i < g_maps.used; ++i)
         if (g_maps.key[i] == key) {
             *m = g_maps.map[i];
@@ -117,12 +124,17 @@ int make_map(CUtensorMap *m, CUtensorMapDataType dt, const void *base, uint64_t 
         snprintf(g_last_cuda_error, sizeof(g_last_cuda_error), "cuTensorMapEncodeTiled unavailable");
         return MGLU_ERR_CUDA;
     }
-    const cuuint64_t dims[2] = {inner, outer};
-    const cuuint64_t strides[1] = {row_bytes};
-    const cuuint32_t box[2] = {box_inner, box_outer};
-    const cuuint32_t es[2] = {1, 1};
-    const CUresult r = fn(m, dt, 2, const_cast<void *>(base), dims, strides, box, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                          sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    cuuint64_t d[3], st[2];
+    cuuint32_t bx[3], es[3] = {1, 1, 1};
+    for (int i = 0; i < rank; ++i) {
+        d[i] = dims[i];
+        bx[i] = box[i];
+        if (i + 1 < rank)
+            st[i] = strides[i];
+    }
+    const CUresult r = fn(m, dt, (cuuint32_t)rank, const_cast<void *>(base), d, st, bx, es,
+                          CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS) {
         snprintf(g_last_cuda_error, sizeof(g_last_cuda_error), "cuTensorMapEncodeTiled failed (%d)", (int)r);
         return MGLU_ERR_CUDA;
@@ -131,6 +143,29 @@ int make_map(CUtensorMap *m, CUtensorMapDataType dt, const void *base, uint64_t 
     g_maps.key[slot] = key;
     g_maps.map[slot] = *m;
     return MGLU_OK;
+}
+
+// 2-D tensor map: `outer` rows of `inner` elements, rows `row_bytes` apart.
+int make_map(CUtensorMap *m, CUtensorMapDataType dt, const void *base, uint64_t inner, uint64_t outer,
+             uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle sw)
+{
+    const uint64_t dims[2] = {inner, outer};
+    const uint64_t strides[1] = {row_bytes};
+    const uint32_t box[2] = {box_inner, box_outer};
+    return make_map_n(m, dt, base, 2, dims, strides, box, sw);
+}
+
+// 3-D view of a row-major [outer][inner] matrix as (chunk of `cw` elements,
+// row, chunk index): a box {cw, box_rows, box_chunks} lands in shared memory
+// as box_chunks consecutive [box_rows][cw] tiles.  inner % cw == 0.
+int make_chunked_map(CUtensorMap *m, CUtensorMapDataType dt, const void *base, uint64_t inner, uint64_t outer,
+                     uint64_t row_bytes, uint32_t cw, uint32_t esize, uint32_t box_rows, uint32_t box_chunks,
+                     CUtensorMapSwizzle sw)
+{
+    const uint64_t dims[3] = {cw, outer, inner / cw};
+    const uint64_t strides[2] = {row_bytes, (uint64_t)cw * esize};
+    const uint32_t box[3] = {cw, box_rows, box_chunks};
+    return make_map_n(m, dt, base, 3, dims, strides, box, sw);
 }
 
 // Raise the kernel's dynamic shared-memory limit once per device (one flag
@@ -149,25 +184,52 @@ int ensure_smem(int bytes, int dev)
     return MGLU_OK;
 }
 
+// Launch with programmatic stream serialization, so a kernel's launch and
+// prologue overlap the tail of the previous kernel on the stream; the kernels
+// wait (griddepcontrol.wait) before they touch global memory.
+template <typename... KArgs, typename... Args>
+int launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, int smem, cudaStream_t s, const char *what,
+               Args... args)
+{
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = (size_t)smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+    if (e != cudaSuccess)
+        return cuda_fail(e, what);
+    return check_launch(what);
+}
+
 // ------------------------------------------------------------------ decode
 template <int NM, int NT>
 int launch_decode(const void *x, int64_t T, int64_t d, const void *W, int64_t rows, const uint8_t *packed, int act,
                   void *out, void *ws, cudaStream_t s)
 {
     using L = mglu::dec::Layout<NM, NT>;
+    if (d >= ((int64_t)1 << 22) || rows >= ((int64_t)1 << 27))
+        return MGLU_ERR_INVALID;  // the kernel's 32-bit schedule arithmetic
     int dev = 0, rc = current_device(&dev);
     if (rc)
         return rc;
     CUtensorMap tw, tx, tm;
-    if ((rc = make_map(&tw, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, W, d, rows, d * 2, mglu::dec::SUBK, mglu::dec::ROWS,
-                       CU_TENSOR_MAP_SWIZZLE_128B)))
+    if ((rc = make_chunked_map(&tw, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, W, d, rows, d * 2, 64, 2, mglu::dec::ROWS,
+                               L::NKC, CU_TENSOR_MAP_SWIZZLE_128B)))
         return rc;
-    if ((rc = make_map(&tx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, x, d, T, d * 2, mglu::dec::SUBK, 8 * NT,
-                       CU_TENSOR_MAP_SWIZZLE_128B)))
+    const int xr = (int)(T < L::XR ? T : L::XR);  // token rows the x box loads
+    if ((rc = make_chunked_map(&tx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, x, d, T, d * 2, 64, 2, (uint32_t)xr, L::NKC,
+                               CU_TENSOR_MAP_SWIZZLE_128B)))
         return rc;
     if (NM > 0) {
-        if ((rc = make_map(&tm, CU_TENSOR_MAP_DATA_TYPE_UINT8, packed, d * NM / 8, rows, d * NM / 8, L::M_BOX,
-                           mglu::dec::ROWS, mglu::dec::mask_swizzle_mode<L::M_BOX>())))
+        if ((rc = make_chunked_map(&tm, CU_TENSOR_MAP_DATA_TYPE_UINT8, packed, d * NM / 8, rows, d * NM / 8,
+                                   L::M_BOX > 0 ? L::M_BOX : 16, 1, mglu::dec::ROWS, L::M_CHUNKS,
+                                   mglu::dec::mask_swizzle_mode<L::M_BOX>())))
             return rc;
     } else {
         tm = tw;  // not read
@@ -175,17 +237,17 @@ int launch_decode(const void *x, int64_t T, int64_t d, const void *W, int64_t ro
     if ((rc = ensure_smem<mglu::dec::decode_kernel<NM, NT>>(L::SMEM, dev)))
         return rc;
     const int64_t rb = (rows + mglu::dec::ROWS - 1) / mglu::dec::ROWS;
-    const int64_t units = rb * ((d + mglu::dec::KS - 1) / mglu::dec::KS);
-    int64_t grid = (int64_t)sm_count(dev) * L::CPS;
+    const int64_t units = rb * ((d + L::KS - 1) / L::KS);
+    int64_t grid = (int64_t)sm_count(dev);
     if (grid > mglu::dec::MAX_CTAS)
         grid = mglu::dec::MAX_CTAS;
     if (grid > units)
         grid = units;
     float *ws_part = reinterpret_cast<float *>(ws);
     int *ws_count = reinterpret_cast<int *>(reinterpret_cast<uint8_t *>(ws) + mglu::dec::part_bytes());
-    mglu::dec::decode_kernel<NM, NT><<<(unsigned)grid, mglu::dec::NTHREADS, L::SMEM, s>>>(
-        tw, tx, tm, (int)T, (int)rows, (int)d, act, ws_part, ws_count, reinterpret_cast<__nv_bfloat16 *>(out));
-    return check_launch("decode launch");
+    return launch_pdl(mglu::dec::decode_kernel<NM, NT>, dim3((unsigned)grid), dim3(L::NTHREADS), L::SMEM, s,
+                      "decode launch", tw, tx, tm, (int)T, xr, (int)rows, (int)d, act, ws_part, ws_count,
+                      reinterpret_cast<__nv_bfloat16 *>(out));
 }
 
 template <int NM>
@@ -224,9 +286,10 @@ int launch_prefill(const void *x, int64_t T, int64_t d, const void *W, int64_t r
         return rc;
     const int64_t tiles = ((T + mglu::pf::BM - 1) / mglu::pf::BM) * ((rows + C::NJ - 1) / C::NJ);
     const int grid = (int)(tiles < sm_count(dev) ? tiles : sm_count(dev));
-    kernel<<<grid, mglu::pf::NTHREADS, C::SMEM, s>>>(tx, tw, tm, (int)T, (int)rows, (int)d, act,
-                                                     reinterpret_cast<__nv_bfloat16 *>(out));
-    return check_launch("prefill launch");
+    (void)kernel;
+    return launch_pdl(mglu::pf::prefill_kernel<NM>, dim3((unsigned)grid), dim3(mglu::pf::NTHREADS), C::SMEM, s,
+                      "prefill launch", tx, tw, tm, (int)T, (int)rows, (int)d, act,
+                      reinterpret_cast<__nv_bfloat16 *>(out));
 }
 
 // ------------------------------------------------------------------ fp32
@@ -331,7 +394,7 @@ int check_forward(const void *x, int64_t T, int64_t d, const void *W, int64_t h,
     if (dtype == MGLU_BF16) {
         if (!aligned(W, 16) || !aligned(packed, 16) || (T > 0 && (!aligned(x, 16) || !aligned(out, 16))))
             return MGLU_ERR_ALIGN;
-        if (d % 8 != 0 || (d * n_m) % 128 != 0)
+        if (d % 128 != 0)
             return MGLU_ERR_ALIGN;
     } else {
         if (!aligned(W, 4) || (T > 0 && (!aligned(x, 4) || !aligned(out, 4))))
@@ -351,7 +414,7 @@ int check_down(const void *hid, int64_t T, int64_t h, const void *Wd, int64_t d,
     if (dtype == MGLU_BF16) {
         if (!aligned(Wd, 16) || (T > 0 && (!aligned(hid, 16) || !aligned(y, 16))))
             return MGLU_ERR_ALIGN;
-        if (h % 8 != 0)
+        if (h % 64 != 0)
             return MGLU_ERR_ALIGN;
     } else {
         if (!aligned(Wd, 4) || (T > 0 && (!aligned(hid, 4) || !aligned(y, 4))))

@@ -107,6 +107,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) prefill_kernel(const __grid_const
     uint64_t *acc_empty = acc_full + 2;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(acc_empty + 2);
 
+    pdl_launch_dependents();
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int num_m = (T + BM - 1) / BM;
     const int num_n = (rows + C::NJ - 1) / C::NJ;
@@ -133,6 +134,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) prefill_kernel(const __grid_const
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
+    pdl_wait();  // the previous kernel's outputs (x) are complete from here on
 
     if (warp == 0) {
         // ---------------------------------------------------------- producer

@@ -85,7 +85,8 @@ def test_forward_rejects_bad_arguments(L):
     assert fwd(L, W=A + 2) == mglu.ERR_ALIGN
     assert fwd(L, pk=A + 4) == mglu.ERR_ALIGN
     assert fwd(L, out=A + 8) == mglu.ERR_ALIGN
-    assert fwd(L, d=100) == mglu.ERR_ALIGN             # d % 8
+    assert fwd(L, d=100) == mglu.ERR_ALIGN             # d % 128
+    assert fwd(L, d=192) == mglu.ERR_ALIGN
     assert fwd(L, d=200, n_m=8) == mglu.ERR_ALIGN      # d * n_m % 128
     assert fwd(L, d=64, n_m=1) == mglu.ERR_ALIGN
     assert fwd(L, d=80, n_m=4) == mglu.ERR_ALIGN
@@ -107,7 +108,8 @@ def test_forward_zero_tokens_is_a_noop(L):
 
 def test_down_and_block_reject_bad_arguments(L):
     big = 1 << 30
-    assert L.mglu_down_proj(A, 1, 100, A, 64, 0, A, A, big, None) == mglu.ERR_ALIGN  # h % 8
+    assert L.mglu_down_proj(A, 1, 100, A, 64, 0, A, A, big, None) == mglu.ERR_ALIGN  # h % 64
+    assert L.mglu_down_proj(A, 1, 96, A, 64, 0, A, A, big, None) == mglu.ERR_ALIGN
     assert L.mglu_down_proj(None, 1, 128, A, 64, 0, A, A, big, None) == mglu.ERR_INVALID
     assert L.mglu_down_proj(A, 1, 128, A, 64, 5, A, A, big, None) == mglu.ERR_INVALID
     assert L.mglu_down_proj(A, 1, 128, A, 64, 0, A, None, 0, None) == mglu.ERR_INVALID  # decode needs scratch

@@ -73,14 +73,16 @@ def test_fp32_down():
 
 # ------------------------------------------------------------------ decode kernel (T <= 16)
 DECODE_CASES = [
-    # n_m, d, h: ragged row block (h % 16 != 0) and ragged k stage (d % 256 != 0)
-    (8, 336, 200),
-    (4, 352, 200),
+    # n_m, d, h: ragged row block (h % 16 != 0) and ragged k stage (d % 512 != 0);
+    # with few units per CTA most row blocks are split between CTAs
+    (8, 640, 200),
+    (4, 896, 200),
     (2, 384, 72),
-    (1, 384, 40),
-    (8, 2048, 256),   # k split over a cluster of 4
-    (8, 4096, 64),    # k split over a cluster of 8
-    (4, 64 * 5, 16),  # one row block, one ragged stage
+    (1, 1152, 40),
+    (8, 2048, 256),   # each row block shared by several CTAs
+    (8, 4096, 64),
+    (4, 128 * 5, 16),  # one row block
+    (4, 2048, 8192),   # many units per CTA: whole row blocks inside one CTA
 ]
 
 
@@ -105,11 +107,11 @@ def test_decode_acts(act, n_m):
 
 # ------------------------------------------------------------------ prefill kernel (tcgen05)
 PREFILL_CASES = [
-    # n_m, T, d, h: ragged token tile, ragged weight tile, ragged k stage
-    (4, 17, 320, 200),
-    (4, 129, 320, 200),
+    # n_m, T, d, h: ragged token tile, ragged weight tile
+    (4, 17, 384, 200),
+    (4, 129, 640, 200),
     (4, 300, 256, 100),
-    (8, 129, 336, 40),
+    (8, 129, 384, 40),
     (8, 200, 512, 72),
     (2, 150, 384, 170),
     (1, 130, 384, 300),
@@ -180,8 +182,8 @@ def test_empty_masks_give_exact_zero(T, n_m):
 
 
 # ------------------------------------------------------------------ down-projection and FFN block
-@pytest.mark.parametrize("T,h,d", [(1, 1000, 200), (5, 1000, 200), (16, 14336, 64), (200, 512, 300),
-                                   (17, 136, 40)])
+@pytest.mark.parametrize("T,h,d", [(1, 1088, 200), (5, 1088, 200), (16, 14336, 64), (200, 512, 300),
+                                   (17, 192, 40)])
 def test_down_proj(T, h, d):
     rng = np.random.default_rng(T + h + d)
     hid = inputs.normal(rng, (T, h), 1.0, "bf16")
