@@ -41,49 +41,62 @@
 
 #include "common.cuh"
 #include "ptx.cuh"
+#include "sched.cuh"
 
 namespace mglu {
 namespace dec {
 
-constexpr int ROWS = 16;
 constexpr int MAX_CTAS = 320;         // grid cap; sizes the split-row-block scratch
 constexpr int BAR_SLOTS_FULL = 1;     // consumers arrive, finisher waits
 constexpr int BAR_SLOTS_FREE = 2;     // finisher arrives, consumers wait
 constexpr int MASK_K = 128;           // k covered by one row of a mask box
 
+// Default consumer warps / 32-k units per warp and stage: as many warps as
+// the register file allows (a quadrant holds 16K registers: 4 warps of 128
+// or 5 of 96 registers), two units per warp so a stage is 512..1024 k.
 template <int NM, int NT>
-struct Layout {
-    // consumer warps: as many as the register file allows (a quadrant holds
-    // 16K registers, so 4 warps of 128 or 5 of 96 registers)
+struct DefaultShape {
     static constexpr int NCW = NT == 2 ? 8 : NM == 8 ? 12 : 16;
-    static constexpr int PRODUCER_WARP = NCW;
-    static constexpr int FINISHER_WARP = NCW + 1;
-    static constexpr int NTHREADS = (NCW + 2) * 32;
+    static constexpr int UPW = 2;
+};
+
+constexpr int MAX_STAGES = 12;
+
+template <int NM, int NT, int NCW_ = DefaultShape<NM, NT>::NCW, int UPW_ = DefaultShape<NM, NT>::UPW>
+struct Layout {
+    static constexpr int NCW = NCW_;
+    static constexpr int UPW = UPW_;                   // 32-k units per consumer warp per stage
+    static constexpr int NPW = NM > 0 ? 3 : 2;         // producer warps: W, x, masks
+    static constexpr int W_WARP = NCW;
+    static constexpr int FINISHER_WARP = NCW + NPW;
+    static constexpr int NTHREADS = (NCW + NPW + 1) * 32;
     static constexpr int BAR_COUNT = (NCW + 1) * 32;   // consumers + finisher
-    static constexpr int KS = NCW * 32;                // k per stage: 32 per consumer warp
+    static constexpr int KS = NCW * 32 * UPW;          // k per stage
     static constexpr int NKC = KS / 64;                // 64-k chunks per stage
-    static constexpr int XR = 8 * NT;                  // token rows of the x tile
+    static constexpr int XR = 8 * NT;                  // most token rows of the x tile
     static constexpr int W_CHUNK = ROWS * 128;         // bytes of one 16 x 64 bf16 chunk
-    static constexpr int X_CHUNK = XR * 128;
+    static constexpr int W_BYTES = NKC * W_CHUNK;
     static constexpr int M_BOX = 16 * NM;              // bytes of one row of a mask box (128 k)
     static constexpr int M_CHUNKS = KS / MASK_K;
-    static constexpr int W_OFF = 0;
-    static constexpr int X_OFF = NKC * W_CHUNK;
-    static constexpr int M_OFF = X_OFF + NKC * X_CHUNK;
     static constexpr int M_BYTES = NM == 0 ? 0 : M_CHUNKS * ROWS * M_BOX;
-    static constexpr int STAGE = (M_OFF + M_BYTES + 1023) / 1024 * 1024;
-    // bytes one stage receives when the x box has xr token rows
-    static __device__ __forceinline__ uint32_t tx(int xr) { return (uint32_t)(NKC * W_CHUNK + NKC * xr * 128 + M_BYTES); }
+    static constexpr int M_OFF = W_BYTES;
+    static constexpr int X_OFF = M_OFF + (M_BYTES + 1023) / 1024 * 1024;
     static constexpr int ACC = (NM + 1) * NT * 128;    // floats of one warp's accumulators
     static constexpr int SLOTS = NCW * ACC * 4;
-    static constexpr int BUDGET = 220 * 1024;
-    static constexpr int STAGES_FIT = (BUDGET - SLOTS - 1024 - 256) / STAGE;
-    static constexpr int STAGES = STAGES_FIT > 12 ? 12 : STAGES_FIT;
-    static constexpr int SLOT_OFF = STAGES * STAGE;
-    static constexpr int BAR_OFF = SLOT_OFF + SLOTS;
-    static constexpr int SMEM = BAR_OFF + 2 * STAGES * 8 + 1024;
-    static_assert(STAGES >= 3, "ring too shallow");
-    static_assert(SMEM <= 227 * 1024, "shared memory");
+    // shared memory: barriers, consumer slots, then the ring of stages
+    static constexpr int BAR_OFF = 0;                  // full[MAX_STAGES], empty[MAX_STAGES]
+    static constexpr int SLOT_OFF = 1024;
+    static constexpr int RING_OFF = (SLOT_OFF + SLOTS + 1023) / 1024 * 1024;
+    static constexpr int SMEM = 227 * 1024;            // includes 1 KB of alignment slack
+    static constexpr int RING_BYTES = SMEM - 1024 - RING_OFF;
+    // a stage with xr token rows of x (x boxes hold only the T rows loaded)
+    static __host__ __device__ constexpr int x_bytes(int xr) { return (NKC * xr * 128 + 1023) / 1024 * 1024; }
+    static __host__ __device__ constexpr int stage_bytes(int xr) { return X_OFF + x_bytes(xr); }
+    static __host__ __device__ constexpr int stages(int xr)
+    {
+        return RING_BYTES / stage_bytes(xr) > MAX_STAGES ? MAX_STAGES : RING_BYTES / stage_bytes(xr);
+    }
+    static_assert(RING_BYTES / (X_OFF + (NKC * XR * 128 + 1023) / 1024 * 1024) >= 3, "ring too shallow");
 };
 
 // Byte offset of (row, o) inside one mask box (rows of M_BOX bytes) under the
@@ -157,13 +170,19 @@ __device__ __forceinline__ uint32_t hmul2_bf16(uint32_t a, uint32_t b)
     return d;
 }
 
+// v << S (S >= 0) or v >> -S, written as an integer multiply so it can run on
+// the FMA pipe instead of the busier ALU pipe.
 template <int S>
 __device__ __forceinline__ uint32_t shift_signed(uint32_t v)
 {
-    if constexpr (S >= 0)
-        return v << S;
+    uint32_t r;
+    if constexpr (S == 0)
+        r = v;
+    else if constexpr (S > 0)
+        asm("mul.lo.u32 %0, %1, %2;" : "=r"(r) : "r"(v), "n"(1u << S));
     else
-        return v >> (-S);
+        asm("mul.hi.u32 %0, %1, %2;" : "=r"(r) : "r"(v), "n"(1u << (32 + S)));
+    return r;
 }
 
 // n_m = 8 path.  The ALU pipe is the scarce one here, so masks are applied
@@ -275,97 +294,36 @@ __device__ __forceinline__ void add_slot(float (&acc)[NM + 1][NT][4], const floa
         }
 }
 
-// The work of one CTA: first its stream-K share (units of the last RB_sk row
-// blocks, split evenly over the grid), then its whole row blocks.  Every
-// role of the CTA walks the same sequence with the same counters; no
-// division happens per unit.
-struct Sched {
-    // 32-bit arithmetic throughout (the host keeps d < 2^22 and rows < 2^27,
-    // so every product below fits): the integer divisions run once per CTA.
-    int nst;          // k-stages per row block
-    int G, cta;       // grid size, this CTA
-    int RB;           // row blocks
-    int q;            // whole row blocks per CTA
-    int rb_sk0;       // first stream-K row block
-    uint32_t U_sk;    // stream-K units
-    uint32_t sk_b;    // first stream-K unit of this CTA
-    int n_sk, n;      // units of this CTA: stream-K, all
-
-    __device__ __forceinline__ void init(int rows, int d, int ks_width)
-    {
-        nst = (d + ks_width - 1) / ks_width;
-        G = gridDim.x;
-        cta = blockIdx.x;
-        RB = (rows + ROWS - 1) / ROWS;
-        q = RB / G;
-        rb_sk0 = q * G;
-        U_sk = (uint32_t)(RB - rb_sk0) * (uint32_t)nst;
-        sk_b = sk_begin(cta);
-        n_sk = (int)(sk_begin(cta + 1) - sk_b);
-        n = n_sk + q * nst;
-    }
-    // (row block, stage) of the first unit of this CTA
-    __device__ __forceinline__ void start(int &rb, int &ks) const
-    {
-        if (n_sk > 0) {
-            rb = rb_sk0 + (int)(sk_b / (uint32_t)nst);
-            ks = (int)(sk_b % (uint32_t)nst);
-        } else {
-            rb = cta * q;
-            ks = 0;
-        }
-    }
-    // advance after unit i (0-based) of this CTA
-    __device__ __forceinline__ void next(int i, int &rb, int &ks) const
-    {
-        if (i + 1 == n_sk) {
-            rb = cta * q;
-            ks = 0;
-        } else if (++ks == nst) {
-            ks = 0;
-            ++rb;
-        }
-    }
-    // does unit i end this CTA's part of its row block?
-    __device__ __forceinline__ bool flush_at(int i, int ks) const
-    {
-        return ks == nst - 1 || i == n_sk - 1 || i == n - 1;
-    }
-    // CTA whose stream-K share holds stream-K unit v
-    __device__ __forceinline__ int sk_owner(uint32_t v) const
-    {
-        return (int)(((v + 1) * (uint32_t)G + U_sk - 1) / U_sk) - 1;
-    }
-    __device__ __forceinline__ uint32_t sk_begin(int c) const { return (uint32_t)c * U_sk / (uint32_t)G; }
-};
-
 // Scratch (global, caller-provided): partial sums of split row blocks, two
 // slots per CTA (first and last row block of its stream-K share), then one
 // arrival counter per row block.  Counters must be zero on entry and are
 // zero again when the kernel completes.
-template <int NM, int NT>
-__global__ void __launch_bounds__(Layout<NM, NT>::NTHREADS, 1)
+template <int NM, int NT, int NCW_ = DefaultShape<NM, NT>::NCW, int UPW_ = DefaultShape<NM, NT>::UPW>
+__global__ void __launch_bounds__(Layout<NM, NT, NCW_, UPW_>::NTHREADS, 1)
     decode_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_x,
                   const __grid_constant__ CUtensorMap tm_m, int T, int xr, int rows, int d, int act,
                   float *__restrict__ ws_part, int *__restrict__ ws_count, __nv_bfloat16 *__restrict__ out)
 {
-    using L = Layout<NM, NT>;
+    using L = Layout<NM, NT, NCW_, UPW_>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t *full = reinterpret_cast<uint64_t *>(smem + L::BAR_OFF);
-    uint64_t *empty = full + L::STAGES;
+    uint64_t *empty = full + MAX_STAGES;
     float *slots = reinterpret_cast<float *>(smem + L::SLOT_OFF);
+    uint8_t *ring = smem + L::RING_OFF;
+    const int STAGE = L::stage_bytes(xr);
+    const int NSTAGES = L::stages(xr);
 
     // The next kernel in the stream may start its prologue now; every access
     // to global memory below waits for the previous kernel to finish.
     pdl_launch_dependents();
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     Sched sc;
-    sc.init(rows, d, L::KS);
+    sc.init(rows, d, L::KS, gridDim.x, blockIdx.x);
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < L::STAGES; ++s) {
-            mbar_init(&full[s], 1);
+        for (int s = 0; s < NSTAGES; ++s) {
+            mbar_init(&full[s], L::NPW);
             mbar_init(&empty[s], L::NCW);
         }
         fence_mbar_init();
@@ -375,34 +333,30 @@ __global__ void __launch_bounds__(Layout<NM, NT>::NTHREADS, 1)
         return;
     pdl_wait();
 
-    if (warp == L::PRODUCER_WARP) {
-        // ------------------------------------------------------------- producer
-        constexpr int NTMA = NM > 0 ? 3 : 2;
-        const CUtensorMap *map = lane == 0 ? &tm_w : lane == 1 ? &tm_x : &tm_m;
-        if (lane < NTMA)
+    if (warp >= L::W_WARP && warp < L::FINISHER_WARP) {
+        // ------------------------------------------------------------- producers
+        // one warp per tensor, so the three loads of a stage are issued in
+        // parallel: warp W_WARP loads W (0, row0, k0/64), the next x
+        // (0, 0, k0/64), the last the packed masks (0, row0, k0/128)
+        const int pw = warp - L::W_WARP;
+        if (lane == 0) {
+            const CUtensorMap *map = pw == 0 ? &tm_w : pw == 1 ? &tm_x : &tm_m;
+            const uint32_t bytes = pw == 0 ? (uint32_t)L::W_BYTES : pw == 1 ? (uint32_t)(L::NKC * xr * 128)
+                                                                            : (uint32_t)L::M_BYTES;
+            const int dst_off = pw == 0 ? 0 : pw == 1 ? L::X_OFF : L::M_OFF;
             prefetch_tensormap(map);
-        const int dst_off = lane == 0 ? L::W_OFF : lane == 1 ? L::X_OFF : L::M_OFF;
-        int rb, ks;
-        sc.start(rb, ks);
-        for (int i = 0; i < sc.n; ++i) {
-            const int s = i % L::STAGES;
-            const uint32_t ph = (uint32_t)(i / L::STAGES) & 1u;
-            int ok = 1;
-            if (lane == 0) {
-                ok = mbar_wait(&empty[s], ph ^ 1u);
-                if (ok)
-                    mbar_arrive_expect_tx(&full[s], L::tx(xr));
+            int rb, ks;
+            sc.start(rb, ks);
+            for (int i = 0; i < sc.n; sc.next(i, rb, ks), ++i) {
+                const int s = i % NSTAGES;
+                const uint32_t ph = (uint32_t)(i / NSTAGES) & 1u;
+                if (!mbar_wait(&empty[s], ph ^ 1u))
+                    break;
+                mbar_arrive_expect_tx(&full[s], bytes);
+                const int k0 = ks * L::KS;
+                tma_load_3d(ring + s * STAGE + dst_off, map, &full[s], 0, pw == 1 ? 0 : rb * ROWS,
+                            pw == 2 ? k0 / MASK_K : k0 / 64);
             }
-            if (!__shfl_sync(0xffffffffu, ok, 0))
-                break;
-            __syncwarp();
-            const int row0 = rb * ROWS;
-            const int k0 = ks * L::KS;
-            // lane 0: W (0, row0, k0/64); lane 1: x (0, 0, k0/64); lane 2: masks (0, row0, k0/128)
-            if (lane < NTMA)
-                tma_load_3d(smem + s * L::STAGE + dst_off, map, &full[s], 0, lane == 1 ? 0 : row0,
-                            lane == 2 ? k0 / MASK_K : k0 / 64);
-            sc.next(i, rb, ks);
         }
         return;
     }
@@ -425,13 +379,11 @@ __global__ void __launch_bounds__(Layout<NM, NT>::NTHREADS, 1)
 
             bool finish = true;
             if (i < sc.n_sk) {
-                const uint32_t v0 = (uint32_t)(rb - sc.rb_sk0) * (uint32_t)sc.nst;  // its first stream-K unit
-                const int c_first = sc.sk_owner(v0);
-                const int c_last = sc.sk_owner(v0 + (uint32_t)sc.nst - 1);
+                int c_first, c_last;
+                const int nparts = sc.contributors(rb, c_first, c_last);
                 if (c_first != c_last) {
-                    // split row block: publish this CTA's partial, the last arriver finishes
-                    const int my_slot = 2 * sc.cta + (v0 <= sc.sk_b ? 0 : 1);
-                    float *mine = ws_part + (int64_t)my_slot * L::ACC;
+                    // publish this CTA's partial; the last arriver finishes
+                    float *mine = ws_part + (int64_t)sc.slot(sc.cta, rb) * L::ACC;
 #pragma unroll
                     for (int v = 0; v <= NM; ++v)
 #pragma unroll
@@ -444,15 +396,14 @@ __global__ void __launch_bounds__(Layout<NM, NT>::NTHREADS, 1)
                     if (lane == 0)
                         prev = atomicAdd(ws_count + rb, 1);
                     prev = __shfl_sync(0xffffffffu, prev, 0);
-                    finish = prev == c_last - c_first;
+                    finish = prev == nparts - 1;
                     if (finish) {
                         // every partial, this CTA's included, read back in CTA order
                         __threadfence();
                         zero_acc<NM, NT>(acc);
-                        for (int cc = c_first; cc <= c_last; ++cc) {
-                            const int sl = 2 * cc + (v0 <= sc.sk_begin(cc) ? 0 : 1);
-                            add_slot<NM, NT>(acc, ws_part + (int64_t)sl * L::ACC, lane, true);
-                        }
+                        for (int cc = c_first; cc <= c_last; ++cc)
+                            if (sc.contributes(cc))
+                                add_slot<NM, NT>(acc, ws_part + (int64_t)sc.slot(cc, rb) * L::ACC, lane, true);
                         if (lane == 0)
                             ws_count[rb] = 0;  // leave the scratch zeroed for the next call
                     }
@@ -477,20 +428,25 @@ __global__ void __launch_bounds__(Layout<NM, NT>::NTHREADS, 1)
 
     // ----------------------------------------------------------------- consumers
     const int g = lane >> 2, c = lane & 3;
-    const int kc = warp >> 1, uu = warp & 1;     // this warp's 32 k: chunk kc, half uu
-    const int ch = ((4 * uu + c) ^ g) << 4;      // 128-byte swizzle: 16-byte chunk ^ (row & 7)
-    const int mc = warp >> 2;                    // mask box holding this warp's k
-    const int mo = ((warp & 3) * 32 + 8 * c) * NM / 8;
-    const int moff_a = L::M_OFF + mc * ROWS * L::M_BOX + mask_swz<L::M_BOX>(g, mo);
-    const int moff_b = L::M_OFF + mc * ROWS * L::M_BOX + mask_swz<L::M_BOX>(g + 8, mo);
-    const int woff = L::W_OFF + kc * L::W_CHUNK + g * 128 + ch;
-    // the x box holds xr token rows per 64-k chunk (rows past xr read other
-    // data; they only feed the MMA columns of tokens >= T, never stored)
-    int xoff[NT];
+    // shared-memory offsets of this warp's operands inside a stage, per unit
+    int woff[L::UPW], moff_a[L::UPW], moff_b[L::UPW], xoff[L::UPW][NT];
 #pragma unroll
-    for (int t = 0; t < NT; ++t) {
-        const int xrow = kc * xr + 8 * t + g;
-        xoff[t] = L::X_OFF + xrow * 128 + (((4 * uu + c) ^ (xrow & 7)) << 4);
+    for (int uw = 0; uw < L::UPW; ++uw) {
+        const int un = warp * L::UPW + uw;   // 32-k unit of the stage
+        const int kc = un >> 1, uu = un & 1; // 64-k chunk, half of it
+        const int ch = ((4 * uu + c) ^ g) << 4;  // 128-byte swizzle: 16-byte chunk ^ (row & 7)
+        woff[uw] = kc * L::W_CHUNK + g * 128 + ch;
+        // the x box holds xr token rows per 64-k chunk (rows past xr read other
+        // data; they only feed the MMA columns of tokens >= T, never stored)
+#pragma unroll
+        for (int t = 0; t < NT; ++t) {
+            const int xrow = kc * xr + 8 * t + g;
+            xoff[uw][t] = L::X_OFF + xrow * 128 + (((4 * uu + c) ^ (xrow & 7)) << 4);
+        }
+        const int mc = un >> 2;  // mask box holding this unit
+        const int mo = ((un & 3) * 32 + 8 * c) * NM / 8;
+        moff_a[uw] = L::M_OFF + mc * ROWS * L::M_BOX + mask_swz<L::M_BOX>(g, mo);
+        moff_b[uw] = L::M_OFF + mc * ROWS * L::M_BOX + mask_swz<L::M_BOX>(g + 8, mo);
     }
     float acc[NM + 1][NT][4];
     zero_acc<NM, NT>(acc);
@@ -503,32 +459,39 @@ __global__ void __launch_bounds__(Layout<NM, NT>::NTHREADS, 1)
     int rb, ks;
     sc.start(rb, ks);
     for (int i = 0; i < sc.n; sc.next(i, rb, ks), ++i) {
-        const int s = i % L::STAGES;
-        const uint32_t ph = (uint32_t)(i / L::STAGES) & 1u;
+        const int s = i % NSTAGES;
+        const uint32_t ph = (uint32_t)(i / NSTAGES) & 1u;
         if (ok && !mbar_wait(&full[s], ph))
             ok = false;
         if (ok) {
-            const uint8_t *st = smem + s * L::STAGE;
-            uint32_t wa[4], wb[4], xb[NT][4];
-            const uint4 va = *reinterpret_cast<const uint4 *>(st + woff);
-            const uint4 vb = *reinterpret_cast<const uint4 *>(st + woff + 8 * 128);
-            wa[0] = va.x, wa[1] = va.y, wa[2] = va.z, wa[3] = va.w;
-            wb[0] = vb.x, wb[1] = vb.y, wb[2] = vb.z, wb[3] = vb.w;
+            const uint8_t *st = ring + s * STAGE;
+            uint32_t wa[L::UPW][4], wb[L::UPW][4], xb[L::UPW][NT][4];
+            uint32_t alo[L::UPW], ahi[L::UPW], blo[L::UPW], bhi[L::UPW];
 #pragma unroll
-            for (int t = 0; t < NT; ++t) {
-                const uint4 vx = *reinterpret_cast<const uint4 *>(st + xoff[t]);
-                xb[t][0] = vx.x, xb[t][1] = vx.y, xb[t][2] = vx.z, xb[t][3] = vx.w;
-            }
-            uint32_t alo = 0, ahi = 0, blo = 0, bhi = 0;
-            if constexpr (NM > 0) {
-                load_mask_chunk<NM>(st + moff_a, alo, ahi);
-                load_mask_chunk<NM>(st + moff_b, blo, bhi);
+            for (int uw = 0; uw < L::UPW; ++uw) {
+                const uint4 va = *reinterpret_cast<const uint4 *>(st + woff[uw]);
+                const uint4 vb = *reinterpret_cast<const uint4 *>(st + woff[uw] + 8 * 128);
+                wa[uw][0] = va.x, wa[uw][1] = va.y, wa[uw][2] = va.z, wa[uw][3] = va.w;
+                wb[uw][0] = vb.x, wb[uw][1] = vb.y, wb[uw][2] = vb.z, wb[uw][3] = vb.w;
+#pragma unroll
+                for (int t = 0; t < NT; ++t) {
+                    const uint4 vx = *reinterpret_cast<const uint4 *>(st + xoff[uw][t]);
+                    xb[uw][t][0] = vx.x, xb[uw][t][1] = vx.y, xb[uw][t][2] = vx.z, xb[uw][t][3] = vx.w;
+                }
+                alo[uw] = ahi[uw] = blo[uw] = bhi[uw] = 0;
+                if constexpr (NM > 0) {
+                    load_mask_chunk<NM>(st + moff_a[uw], alo[uw], ahi[uw]);
+                    load_mask_chunk<NM>(st + moff_b[uw], blo[uw], bhi[uw]);
+                }
             }
             __syncwarp();
             if (lane == 0)
                 mbar_arrive(&empty[s]);  // operands are in registers: the stage can be refilled
-            unit_step<NM, NT, 0>(acc, wa, wb, xb, alo, ahi, blo, bhi);
-            unit_step<NM, NT, 1>(acc, wa, wb, xb, alo, ahi, blo, bhi);
+#pragma unroll
+            for (int uw = 0; uw < L::UPW; ++uw) {
+                unit_step<NM, NT, 0>(acc, wa[uw], wb[uw], xb[uw], alo[uw], ahi[uw], blo[uw], bhi[uw]);
+                unit_step<NM, NT, 1>(acc, wa[uw], wb[uw], xb[uw], alo[uw], ahi[uw], blo[uw], bhi[uw]);
+            }
         }
         if (!sc.flush_at(i, ks))
             continue;

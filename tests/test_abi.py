@@ -138,3 +138,14 @@ def test_mask_expansion_host_check(tmp_path):
                     "-o", str(exe), os.path.join(ROOT, "tests", "native", "pair_mask_check.cpp")], check=True)
     r = subprocess.run([str(exe)], capture_output=True, text=True)
     assert r.returncode == 0 and r.stdout.strip() == "ok", r.stdout
+
+
+def test_decode_schedule_host_check(tmp_path):
+    """The decode kernel's work split (csrc/sched.cuh), compiled for the host:
+    every (row block, k-stage) unit done once, split row blocks' contributor
+    counts and scratch slots consistent, over many shapes and grid sizes."""
+    exe = tmp_path / "sched_check"
+    subprocess.run(["g++", "-std=c++17", "-O1", "-I", os.path.join(ROOT, "masked_glu_b200", "csrc"),
+                    "-o", str(exe), os.path.join(ROOT, "tests", "native", "sched_check.cpp")], check=True)
+    r = subprocess.run([str(exe)], capture_output=True, text=True)
+    assert r.returncode == 0 and r.stdout.strip() == "ok", r.stdout
