@@ -66,17 +66,15 @@ template <int NM, int NT, int NCW_ = DefaultShape<NM, NT>::NCW, int UPW_ = Defau
 struct Layout {
     static constexpr int NCW = NCW_;
     static constexpr int UPW = UPW_;                   // 32-k units per consumer warp per stage
-    static constexpr int NPW = NM > 0 ? 3 : 2;         // producer warps: W, x, masks
-    static constexpr int W_WARP = NCW;
-    static constexpr int FINISHER_WARP = NCW + NPW;
-    static constexpr int NTHREADS = (NCW + NPW + 1) * 32;
+    static constexpr int W_WARP = NCW;                 // producer warp (one thread issues every load)
+    static constexpr int FINISHER_WARP = NCW + 1;
+    static constexpr int NTHREADS = (NCW + 2) * 32;
     static constexpr int BAR_COUNT = (NCW + 1) * 32;   // consumers + finisher
     static constexpr int KS = NCW * 32 * UPW;          // k per stage
     static constexpr int NKC = KS / 64;                // 64-k chunks per stage
     static constexpr int XR = 8 * NT;                  // most token rows of the x tile
-    static constexpr int W_CHUNK = ROWS * 128;         // bytes of one 16 x 64 bf16 chunk
-    static constexpr int W_BYTES = NKC * W_CHUNK;
-    static constexpr int M_BOX = 16 * NM;              // bytes of one row of a mask box (128 k)
+    static constexpr int W_BYTES = ROWS * NKC * 128;   // W tile [16 rows][NKC chunks of 64 k]
+    static constexpr int M_BOX = 16 * NM;              // mask bytes of one row per 128 k
     static constexpr int M_CHUNKS = KS / MASK_K;
     static constexpr int M_BYTES = NM == 0 ? 0 : M_CHUNKS * ROWS * M_BOX;
     static constexpr int M_OFF = W_BYTES;
@@ -99,19 +97,18 @@ struct Layout {
     static_assert(RING_BYTES / (X_OFF + (NKC * XR * 128 + 1023) / 1024 * 1024) >= 3, "ring too shallow");
 };
 
-// Byte offset of (row, o) inside one mask box (rows of M_BOX bytes) under the
-// swizzle the tensor map uses for that width.
-template <int M_BOX>
-__device__ __forceinline__ int mask_swz(int row, int o)
+// Byte offset of a linear position inside a staged tile under the tensor
+// map's swizzle: the 16-byte unit index (address bits 4 and up) is XORed with
+// the 128-byte line index (address bits 7 and up) over 3, 2 or 1 bits for the
+// 128-, 64- and 32-byte swizzles; narrower tiles are not swizzled.  Every
+// tile starts on a 1024-byte boundary, so tile offsets and addresses agree.
+template <int SPAN>
+__host__ __device__ constexpr int swz(int lin)
 {
-    if constexpr (M_BOX == 128)
-        return row * 128 + ((((o >> 4) ^ (row & 7)) << 4) | (o & 15));
-    else if constexpr (M_BOX == 64)
-        return row * 64 + ((((o >> 4) ^ ((row >> 1) & 3)) << 4) | (o & 15));
-    else if constexpr (M_BOX == 32)
-        return row * 32 + ((((o >> 4) ^ ((row >> 2) & 1)) << 4) | (o & 15));
-    else
-        return row * M_BOX + o;
+    return SPAN == 128 ? lin ^ (((lin >> 7) & 7) << 4)
+         : SPAN == 64  ? lin ^ (((lin >> 7) & 3) << 4)
+         : SPAN == 32  ? lin ^ (((lin >> 7) & 1) << 4)
+                       : lin;
 }
 
 template <int M_BOX>
@@ -323,7 +320,7 @@ __global__ void __launch_bounds__(Layout<NM, NT, NCW_, UPW_>::NTHREADS, 1)
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < NSTAGES; ++s) {
-            mbar_init(&full[s], L::NPW);
+            mbar_init(&full[s], 1);
             mbar_init(&empty[s], L::NCW);
         }
         fence_mbar_init();
@@ -333,18 +330,17 @@ __global__ void __launch_bounds__(Layout<NM, NT, NCW_, UPW_>::NTHREADS, 1)
         return;
     pdl_wait();
 
-    if (warp >= L::W_WARP && warp < L::FINISHER_WARP) {
-        // ------------------------------------------------------------- producers
-        // one warp per tensor, so the three loads of a stage are issued in
-        // parallel: warp W_WARP loads W (0, row0, k0/64), the next x
-        // (0, 0, k0/64), the last the packed masks (0, row0, k0/128)
-        const int pw = warp - L::W_WARP;
+    if (warp == L::W_WARP) {
+        // ------------------------------------------------------------- producer
+        // One thread issues the W, x and mask boxes of a stage against one
+        // expected byte count.  (Separate producer warps arriving on the same
+        // barrier gave occasional wrong operands on B200; one did not.)
         if (lane == 0) {
-            const CUtensorMap *map = pw == 0 ? &tm_w : pw == 1 ? &tm_x : &tm_m;
-            const uint32_t bytes = pw == 0 ? (uint32_t)L::W_BYTES : pw == 1 ? (uint32_t)(L::NKC * xr * 128)
-                                                                            : (uint32_t)L::M_BYTES;
-            const int dst_off = pw == 0 ? 0 : pw == 1 ? L::X_OFF : L::M_OFF;
-            prefetch_tensormap(map);
+            const uint32_t bytes = (uint32_t)(L::W_BYTES + L::NKC * xr * 128 + (NM > 0 ? L::M_BYTES : 0));
+            prefetch_tensormap(&tm_w);
+            prefetch_tensormap(&tm_x);
+            if (NM > 0)
+                prefetch_tensormap(&tm_m);
             int rb, ks;
             sc.start(rb, ks);
             for (int i = 0; i < sc.n; sc.next(i, rb, ks), ++i) {
@@ -353,9 +349,13 @@ __global__ void __launch_bounds__(Layout<NM, NT, NCW_, UPW_>::NTHREADS, 1)
                 if (!mbar_wait(&empty[s], ph ^ 1u))
                     break;
                 mbar_arrive_expect_tx(&full[s], bytes);
+                uint8_t *st = ring + s * STAGE;
                 const int k0 = ks * L::KS;
-                tma_load_3d(ring + s * STAGE + dst_off, map, &full[s], 0, pw == 1 ? 0 : rb * ROWS,
-                            pw == 2 ? k0 / MASK_K : k0 / 64);
+                // boxes: W (0, k0/64, row0), x (0, k0/64, 0), masks (0, k0/128, row0)
+                tma_load_3d(st, &tm_w, &full[s], 0, k0 / 64, rb * ROWS);
+                tma_load_3d(st + L::X_OFF, &tm_x, &full[s], 0, k0 / 64, 0);
+                if constexpr (NM > 0)
+                    tma_load_3d(st + L::M_OFF, &tm_m, &full[s], 0, k0 / MASK_K, rb * ROWS);
             }
         }
         return;
@@ -374,8 +374,10 @@ __global__ void __launch_bounds__(Layout<NM, NT, NCW_, UPW_>::NTHREADS, 1)
             zero_acc<NM, NT>(acc);
             for (int w = 0; w < L::NCW; ++w)
                 add_slot<NM, NT>(acc, slots + w * L::ACC, lane, false);
-            if (i != sc.n - 1)
+            if (i != sc.n - 1) {
+                __threadfence_block();  // the slot reads above are done before the consumers may overwrite
                 named_bar_arrive(BAR_SLOTS_FREE, L::BAR_COUNT);
+            }
 
             bool finish = true;
             if (i < sc.n_sk) {
@@ -434,19 +436,21 @@ __global__ void __launch_bounds__(Layout<NM, NT, NCW_, UPW_>::NTHREADS, 1)
     for (int uw = 0; uw < L::UPW; ++uw) {
         const int un = warp * L::UPW + uw;   // 32-k unit of the stage
         const int kc = un >> 1, uu = un & 1; // 64-k chunk, half of it
-        const int ch = ((4 * uu + c) ^ g) << 4;  // 128-byte swizzle: 16-byte chunk ^ (row & 7)
-        woff[uw] = kc * L::W_CHUNK + g * 128 + ch;
-        // the x box holds xr token rows per 64-k chunk (rows past xr read other
-        // data; they only feed the MMA columns of tokens >= T, never stored)
+        // W tile [row][chunk][64 k]: lane (g, c) reads 16 bytes of row g; row
+        // g + 8 is 8 * NKC lines on, the same swizzle phase
+        woff[uw] = swz<128>((g * L::NKC + kc) * 128 + (4 * uu + c) * 16);
+        // x tile [token][chunk][64 k] holds xr tokens; lanes of tokens >= xr
+        // read token xr - 1 (their MMA columns are never stored)
 #pragma unroll
         for (int t = 0; t < NT; ++t) {
-            const int xrow = kc * xr + 8 * t + g;
-            xoff[uw][t] = L::X_OFF + xrow * 128 + (((4 * uu + c) ^ (xrow & 7)) << 4);
+            const int tr = 8 * t + g < xr ? 8 * t + g : xr - 1;
+            xoff[uw][t] = L::X_OFF + swz<128>((tr * L::NKC + kc) * 128 + (4 * uu + c) * 16);
         }
-        const int mc = un >> 2;  // mask box holding this unit
+        // mask tile [row][128-k chunk][M_BOX bytes]
+        const int mc = un >> 2;
         const int mo = ((un & 3) * 32 + 8 * c) * NM / 8;
-        moff_a[uw] = L::M_OFF + mc * ROWS * L::M_BOX + mask_swz<L::M_BOX>(g, mo);
-        moff_b[uw] = L::M_OFF + mc * ROWS * L::M_BOX + mask_swz<L::M_BOX>(g + 8, mo);
+        moff_a[uw] = L::M_OFF + swz<L::M_BOX>((g * L::M_CHUNKS + mc) * L::M_BOX + mo);
+        moff_b[uw] = L::M_OFF + swz<L::M_BOX>(((g + 8) * L::M_CHUNKS + mc) * L::M_BOX + mo);
     }
     float acc[NM + 1][NT][4];
     zero_acc<NM, NT>(acc);
@@ -461,7 +465,7 @@ __global__ void __launch_bounds__(Layout<NM, NT, NCW_, UPW_>::NTHREADS, 1)
     for (int i = 0; i < sc.n; sc.next(i, rb, ks), ++i) {
         const int s = i % NSTAGES;
         const uint32_t ph = (uint32_t)(i / NSTAGES) & 1u;
-        if (ok && !mbar_wait(&full[s], ph))
+        if (ok && !mbar_wait_warp(&full[s], ph))
             ok = false;
         if (ok) {
             const uint8_t *st = ring + s * STAGE;
@@ -470,7 +474,7 @@ __global__ void __launch_bounds__(Layout<NM, NT, NCW_, UPW_>::NTHREADS, 1)
 #pragma unroll
             for (int uw = 0; uw < L::UPW; ++uw) {
                 const uint4 va = *reinterpret_cast<const uint4 *>(st + woff[uw]);
-                const uint4 vb = *reinterpret_cast<const uint4 *>(st + woff[uw] + 8 * 128);
+                const uint4 vb = *reinterpret_cast<const uint4 *>(st + woff[uw] + 8 * L::NKC * 128);
                 wa[uw][0] = va.x, wa[uw][1] = va.y, wa[uw][2] = va.z, wa[uw][3] = va.w;
                 wb[uw][0] = vb.x, wb[uw][1] = vb.y, wb[uw][2] = vb.z, wb[uw][3] = vb.w;
 #pragma unroll
@@ -484,9 +488,24 @@ __global__ void __launch_bounds__(Layout<NM, NT, NCW_, UPW_>::NTHREADS, 1)
                     load_mask_chunk<NM>(st + moff_b[uw], blo[uw], bhi[uw]);
                 }
             }
+            // Release the stage only once every lane's loads have returned:
+            // folding all loaded words into one value makes each lane wait for
+            // its own loads before the warp synchronizes and lane 0 arrives.
+            // (Releasing right after issuing the loads let a refill overwrite
+            // operands still being read, now and then, on B200.)
+            uint32_t dep = 0;
+#pragma unroll
+            for (int uw = 0; uw < L::UPW; ++uw) {
+                dep ^= wa[uw][0] ^ wa[uw][1] ^ wa[uw][2] ^ wa[uw][3] ^ wb[uw][0] ^ wb[uw][1] ^ wb[uw][2] ^ wb[uw][3];
+#pragma unroll
+                for (int t = 0; t < NT; ++t)
+                    dep ^= xb[uw][t][0] ^ xb[uw][t][1] ^ xb[uw][t][2] ^ xb[uw][t][3];
+                dep ^= alo[uw] ^ ahi[uw] ^ blo[uw] ^ bhi[uw];
+            }
+            consume(dep);
             __syncwarp();
             if (lane == 0)
-                mbar_arrive(&empty[s]);  // operands are in registers: the stage can be refilled
+                mbar_arrive(&empty[s]);
 #pragma unroll
             for (int uw = 0; uw < L::UPW; ++uw) {
                 unit_step<NM, NT, 0>(acc, wa[uw], wb[uw], xb[uw], alo[uw], ahi[uw], blo[uw], bhi[uw]);
@@ -505,6 +524,7 @@ __global__ void __launch_bounds__(Layout<NM, NT, NCW_, UPW_>::NTHREADS, 1)
             for (int t = 0; t < NT; ++t)
                 *reinterpret_cast<float4 *>(slot + ((v * NT + t) * 32 + lane) * 4) =
                     make_float4(acc[v][t][0], acc[v][t][1], acc[v][t][2], acc[v][t][3]);
+        __threadfence_block();  // the slot writes are visible before the finisher reads them
         named_bar_arrive(BAR_SLOTS_FULL, L::BAR_COUNT);
         ++nflush;
         zero_acc<NM, NT>(acc);

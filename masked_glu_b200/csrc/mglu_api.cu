@@ -155,16 +155,17 @@ int make_map(CUtensorMap *m, CUtensorMapDataType dt, const void *base, uint64_t 
     return make_map_n(m, dt, base, 2, dims, strides, box, sw);
 }
 
-// 3-D view of a row-major [outer][inner] matrix as (chunk of `cw` elements,
-// row, chunk index): a box {cw, box_rows, box_chunks} lands in shared memory
-// as box_chunks consecutive [box_rows][cw] tiles.  inner % cw == 0.
+// 3-D view of a row-major [outer][inner] matrix as (element of a chunk of
+// `cw` elements, chunk, row): a box {cw, box_chunks, box_rows} lands in shared
+// memory as box_rows consecutive rows of box_chunks chunks.  Strides grow with
+// the dimension, as in a plain 2-D view.  inner % cw == 0.
 int make_chunked_map(CUtensorMap *m, CUtensorMapDataType dt, const void *base, uint64_t inner, uint64_t outer,
-                     uint64_t row_bytes, uint32_t cw, uint32_t esize, uint32_t box_rows, uint32_t box_chunks,
+                     uint64_t row_bytes, uint32_t cw, uint32_t esize, uint32_t box_chunks, uint32_t box_rows,
                      CUtensorMapSwizzle sw)
 {
-    const uint64_t dims[3] = {cw, outer, inner / cw};
-    const uint64_t strides[2] = {row_bytes, (uint64_t)cw * esize};
-    const uint32_t box[3] = {cw, box_rows, box_chunks};
+    const uint64_t dims[3] = {cw, inner / cw, outer};
+    const uint64_t strides[2] = {(uint64_t)cw * esize, row_bytes};
+    const uint32_t box[3] = {cw, box_chunks, box_rows};
     return make_map_n(m, dt, base, 3, dims, strides, box, sw);
 }
 
@@ -219,16 +220,16 @@ int launch_decode(const void *x, int64_t T, int64_t d, const void *W, int64_t ro
     if (rc)
         return rc;
     CUtensorMap tw, tx, tm;
-    if ((rc = make_chunked_map(&tw, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, W, d, rows, d * 2, 64, 2, mglu::dec::ROWS,
-                               L::NKC, CU_TENSOR_MAP_SWIZZLE_128B)))
+    if ((rc = make_chunked_map(&tw, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, W, d, rows, d * 2, 64, 2, L::NKC,
+                               mglu::dec::ROWS, CU_TENSOR_MAP_SWIZZLE_128B)))
         return rc;
     const int xr = (int)(T < L::XR ? T : L::XR);  // token rows the x box loads
-    if ((rc = make_chunked_map(&tx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, x, d, T, d * 2, 64, 2, (uint32_t)xr, L::NKC,
+    if ((rc = make_chunked_map(&tx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, x, d, T, d * 2, 64, 2, L::NKC, (uint32_t)xr,
                                CU_TENSOR_MAP_SWIZZLE_128B)))
         return rc;
     if (NM > 0) {
         if ((rc = make_chunked_map(&tm, CU_TENSOR_MAP_DATA_TYPE_UINT8, packed, d * NM / 8, rows, d * NM / 8,
-                                   L::M_BOX > 0 ? L::M_BOX : 16, 1, mglu::dec::ROWS, L::M_CHUNKS,
+                                   L::M_BOX > 0 ? L::M_BOX : 16, 1, L::M_CHUNKS, mglu::dec::ROWS,
                                    mglu::dec::mask_swizzle_mode<L::M_BOX>())))
             return rc;
     } else {

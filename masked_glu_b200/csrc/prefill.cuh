@@ -209,7 +209,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) prefill_kernel(const __grid_const
                 for (int kb = 0; kb < nkb; ++kb, ++it) {
                     const int s = it % C::STAGES;
                     const uint32_t ph = (uint32_t)(it / C::STAGES) & 1u;
-                    if (!mbar_wait(&full[s], ph)) {
+                    if (!mbar_wait_warp(&full[s], ph)) {
                         ok = false;
                         break;
                     }
@@ -238,7 +238,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) prefill_kernel(const __grid_const
         for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++acc_it) {
             const int b = acc_it & 1;
             const uint32_t aph = (uint32_t)(acc_it >> 1) & 1u;
-            if (!mbar_wait(&acc_full[b], aph))
+            if (!mbar_wait_warp(&acc_full[b], aph))
                 break;
             tc_fence_after();
             const int m0 = (tile % num_m) * BM;

@@ -84,6 +84,27 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity)
     }
 }
 
+// Wait for a phase as a whole warp (all 32 lanes call it together): lane 0
+// polls the barrier, then the warp synchronizes and every lane takes lane 0's
+// answer, so the lanes' later shared-memory reads are ordered after lane 0's
+// acquire.  On B200, warps whose 32 lanes each polled a TMA barrier
+// themselves occasionally read stale operands afterwards (about one read in
+// ten thousand, only when the warp had to wait); with one polling lane per
+// warp every read was correct.
+__device__ __forceinline__ bool mbar_wait_warp(uint64_t *bar, uint32_t parity)
+{
+    int ok = 1;
+    if ((threadIdx.x & 31) == 0)
+        ok = mbar_wait(bar, parity) ? 1 : 0;
+    ok = __shfl_sync(0xffffffffu, ok, 0);
+    __syncwarp();
+    return ok != 0;
+}
+
+// Make the calling thread hold `v` in a register here: every instruction that
+// produced it has completed (used to wait for outstanding loads).
+__device__ __forceinline__ void consume(uint32_t v) { asm volatile("" ::"r"(v) : "memory"); }
+
 // ---------------------------------------------------------------- dependent launch
 // Kernels are launched with programmatic stream serialization: the next
 // kernel on the stream may be scheduled once every CTA of this one has
