@@ -151,6 +151,45 @@ int mglu_forward_down(const void *x, int64_t T, int64_t d, const void *W,
                       int dtype, const void *W_down, void *workspace,
                       size_t workspace_bytes, void *y, void *stream);
 
+/* Most output rows mglu_forward_decode_static accepts (its built-in scratch
+ * holds one counter per 16 of them). */
+#define MGLU_STATIC_SCRATCH_MAX_ROWS 262144
+
+/*
+ * mglu_forward on the decode kernel, with the kernel's cross-CTA scratch
+ * taken from a buffer built into the library (a static device array of
+ * mglu_scratch_bytes(MGLU_STATIC_SCRATCH_MAX_ROWS) bytes, about 6 MB, which
+ * the CUDA runtime places when it loads the library's device code) instead
+ * of a caller buffer.  The paper has no counterpart: it is an interface
+ * convenience of this library, not part of the method.
+ *
+ * It is meant for callers that cannot hand the library a scratch buffer: a
+ * plain-C host that has no device allocator of its own, or a serving loop
+ * with a fixed device-memory budget that must not allocate once it has
+ * started.  No call allocates device memory: there is no cudaMalloc,
+ * cudaFree or other allocating call on this path.
+ *
+ *   Arguments and layouts as mglu_forward with dtype MGLU_BF16 (same
+ *   alignment and d % 128 rules).  T must be in 0..16 (T == 0 is a no-op),
+ *   else MGLU_ERR_UNSUPPORTED.  h must be <= MGLU_STATIC_SCRATCH_MAX_ROWS,
+ *   else MGLU_ERR_INVALID, with the limit stated in mglu_last_cuda_error().
+ *   The decode kernel runs for every T in 1..16, whatever
+ *   mglu_set_decode_max_tokens says.
+ *
+ * The first call on each device does the set-up: it looks up the array's
+ * device address (cudaGetSymbolAddress, return code checked) and clears the
+ * scratch on `stream`.  Make that first call before any stream capture.
+ * Every call also clears the arrival counters of its row blocks on `stream`
+ * before the kernel starts, since those must start at zero.
+ *
+ * There is one such scratch per device, so calls that may overlap in time
+ * (other streams, other host threads) race on it and give wrong results.
+ * Order them on one stream.
+ */
+int mglu_forward_decode_static(const void *x, int64_t T, int64_t d,
+                               const void *W, int64_t h, const uint8_t *packed,
+                               int n_m, int act, void *out, void *stream);
+
 /* Which kernel family mglu_forward uses for T tokens of `dtype`. */
 int mglu_forward_path(int64_t T, int dtype);
 

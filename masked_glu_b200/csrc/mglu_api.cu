@@ -460,6 +460,41 @@ int pack_common(const uint8_t *in, int n_m, int64_t d, int64_t h, uint8_t *outp,
     }
 }
 
+// ------------------------------------------------------------------ built-in scratch
+// Decode scratch for mglu_forward_decode_static: the same layout as a caller
+// buffer of mglu_scratch_bytes(MGLU_STATIC_SCRATCH_MAX_ROWS) bytes.  It lives
+// in the library's device image, so no call has to allocate it: that entry
+// point serves callers with no device allocator of their own (a plain-C host)
+// or with a fixed memory budget that forbids allocating after start-up.
+constexpr size_t kStaticScratchBytes = (size_t)mglu::dec::workspace_bytes(MGLU_STATIC_SCRATCH_MAX_ROWS);
+
+std::mutex g_static_mu;
+void *g_static_scratch_ptr[kMaxDevices] = {nullptr};
+
+}  // namespace
+
+static __device__ __align__(256) unsigned char g_static_scratch[kStaticScratchBytes];
+
+namespace {
+
+// Device address of the built-in scratch on `dev`, looked up (and the whole
+// scratch cleared on `s`) the first time each device is used.
+int static_scratch(int dev, cudaStream_t s, void **ptr)
+{
+    std::lock_guard<std::mutex> lock(g_static_mu);
+    if (!g_static_scratch_ptr[dev]) {
+        void *p = nullptr;
+        cudaError_t e = cudaGetSymbolAddress(&p, g_static_scratch);
+        if (e != cudaSuccess)
+            return cuda_fail(e, "cudaGetSymbolAddress(built-in decode scratch)");
+        if ((e = cudaMemsetAsync(p, 0, kStaticScratchBytes, s)) != cudaSuccess)
+            return cuda_fail(e, "clear built-in decode scratch");
+        g_static_scratch_ptr[dev] = p;
+    }
+    *ptr = g_static_scratch_ptr[dev];
+    return MGLU_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -533,6 +568,38 @@ int mglu_forward_down(const void *x, int64_t T, int64_t d, const void *W, int64_
     if ((rc = run_product(x, T, d, W, h, packed, n_m, act, dtype, workspace, scratch, s)))
         return rc;
     return run_product(workspace, T, h, W_down, d, nullptr, 0, 0, dtype, y, scratch, s);
+}
+
+int mglu_forward_decode_static(const void *x, int64_t T, int64_t d, const void *W, int64_t h,
+                               const uint8_t *packed, int n_m, int act, void *out, void *stream)
+{
+    int rc = check_forward(x, T, d, W, h, packed, n_m, act, MGLU_BF16, out);
+    if (rc)
+        return rc;
+    if (T > 16)
+        return MGLU_ERR_UNSUPPORTED;
+    if (h > MGLU_STATIC_SCRATCH_MAX_ROWS) {
+        snprintf(g_last_cuda_error, sizeof(g_last_cuda_error),
+                 "mglu_forward_decode_static: h = %lld exceeds the built-in scratch limit of %d rows", (long long)h,
+                 MGLU_STATIC_SCRATCH_MAX_ROWS);
+        return MGLU_ERR_INVALID;
+    }
+    if (T == 0)
+        return MGLU_OK;
+    int dev = 0;
+    if ((rc = current_device(&dev)))
+        return rc;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    void *ws = nullptr;
+    if ((rc = static_scratch(dev, s, &ws)))
+        return rc;
+    // the arrival counters of this call's row blocks must start at zero
+    const size_t counters = (size_t)((h + mglu::dec::ROWS - 1) / mglu::dec::ROWS) * sizeof(int);
+    const cudaError_t e =
+        cudaMemsetAsync(reinterpret_cast<uint8_t *>(ws) + mglu::dec::part_bytes(), 0, counters, s);
+    if (e != cudaSuccess)
+        return cuda_fail(e, "clear built-in decode scratch counters");
+    return by_nm<DecodeF>(n_m, x, T, d, W, h, packed, act, out, ws, s);
 }
 
 int mglu_forward_path(int64_t T, int dtype) { return path_for(T, dtype); }

@@ -59,6 +59,7 @@ def lib() -> ctypes.CDLL:
             "mglu_down_proj": (I32, [P, I64, I64, P, I64, I32, P, P, SZ, P]),
             "mglu_workspace_bytes": (SZ, [I64, I64, I64, I32, I32]),
             "mglu_forward_down": (I32, [P, I64, I64, P, I64, P, I32, I32, I32, P, P, SZ, P, P]),
+            "mglu_forward_decode_static": (I32, [P, I64, I64, P, I64, P, I32, I32, P, P]),
             "mglu_forward_path": (I32, [I64, I32]),
             "mglu_set_decode_max_tokens": (I32, [I32]),
             "mglu_last_device_status": (I32, [P]),
@@ -167,6 +168,21 @@ def forward(x: torch.Tensor, W: torch.Tensor, packed: torch.Tensor, n_m: int, ac
         scratch = default_scratch(h, x.device)
     _check(lib().mglu_forward(_ptr(x), T, d, _ptr(W), h, _ptr(packed), n_m, _act(act), _dtype(x),
                               _ptr(out), _ptr(scratch), _nbytes(scratch), _stream(stream)), "mglu_forward")
+    return out
+
+
+def forward_decode_static(x: torch.Tensor, W: torch.Tensor, packed: torch.Tensor, n_m: int, act="swish",
+                          out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """mglu_forward on the decode kernel (bf16, T <= 16) using the library's
+    built-in scratch instead of a caller buffer."""
+    T, d = x.shape
+    h = W.shape[0]
+    if W.shape[1] != d or W.dtype != x.dtype:
+        raise ValueError("W must be [h][d] with x's dtype")
+    if out is None:
+        out = torch.empty((T, h), dtype=x.dtype, device=x.device)
+    _check(lib().mglu_forward_decode_static(_ptr(x), T, d, _ptr(W), h, _ptr(packed), n_m, _act(act), _ptr(out),
+                                            _stream(stream)), "mglu_forward_decode_static")
     return out
 
 
