@@ -51,13 +51,17 @@ constexpr int BAR_SLOTS_FULL = 1;     // consumers arrive, finisher waits
 constexpr int BAR_SLOTS_FREE = 2;     // finisher arrives, consumers wait
 constexpr int MASK_K = 128;           // k covered by one row of a mask box
 
-// Default consumer warps / 32-k units per warp and stage: as many warps as
-// the register file allows (a quadrant holds 16K registers: 4 warps of 128
-// or 5 of 96 registers), two units per warp so a stage is 512..1024 k.
+// Default consumer warps / 32-k units per warp and stage, chosen by timing on
+// B200.  The math of a unit is bound by instruction issue, so more warps do
+// not make it faster; fewer warps that each take more units per stage mean
+// fewer accumulator slots to reduce and leave shared memory for a deeper
+// ring: one warp per SM quadrant with eight units (1024 k per stage) for
+// n_m <= 4, eight warps with two units (512 k) for n_m = 8 and for two token
+// blocks.
 template <int NM, int NT>
 struct DefaultShape {
-    static constexpr int NCW = NT == 2 ? 8 : NM == 8 ? 12 : 16;
-    static constexpr int UPW = 2;
+    static constexpr int NCW = NT == 2 ? 8 : NM == 8 ? 8 : 4;
+    static constexpr int UPW = NT == 2 ? 2 : NM == 8 ? 2 : 8;
 };
 
 constexpr int MAX_STAGES = 12;
@@ -82,7 +86,7 @@ struct Layout {
     static constexpr int ACC = (NM + 1) * NT * 128;    // floats of one warp's accumulators
     static constexpr int SLOTS = NCW * ACC * 4;
     // shared memory: barriers, consumer slots, then the ring of stages
-    static constexpr int BAR_OFF = 0;                  // full[MAX_STAGES], empty[MAX_STAGES]
+    static constexpr int BAR_OFF = 0;                  // full, xfull, mfull, empty: MAX_STAGES each
     static constexpr int SLOT_OFF = 1024;
     static constexpr int RING_OFF = (SLOT_OFF + SLOTS + 1023) / 1024 * 1024;
     static constexpr int SMEM = 227 * 1024;            // includes 1 KB of alignment slack
@@ -305,7 +309,9 @@ __global__ void __launch_bounds__(Layout<NM, NT, NCW_, UPW_>::NTHREADS, 1)
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t *full = reinterpret_cast<uint64_t *>(smem + L::BAR_OFF);
-    uint64_t *empty = full + MAX_STAGES;
+    uint64_t *xfull = full + MAX_STAGES;
+    uint64_t *mfull = xfull + MAX_STAGES;
+    uint64_t *empty = mfull + MAX_STAGES;
     float *slots = reinterpret_cast<float *>(smem + L::SLOT_OFF);
     uint8_t *ring = smem + L::RING_OFF;
     const int STAGE = L::stage_bytes(xr);
@@ -321,6 +327,8 @@ __global__ void __launch_bounds__(Layout<NM, NT, NCW_, UPW_>::NTHREADS, 1)
     if (threadIdx.x == 0) {
         for (int s = 0; s < NSTAGES; ++s) {
             mbar_init(&full[s], 1);
+            mbar_init(&xfull[s], 1);
+            mbar_init(&mfull[s], 1);
             mbar_init(&empty[s], L::NCW);
         }
         fence_mbar_init();
@@ -332,11 +340,12 @@ __global__ void __launch_bounds__(Layout<NM, NT, NCW_, UPW_>::NTHREADS, 1)
 
     if (warp == L::W_WARP) {
         // ------------------------------------------------------------- producer
-        // One thread issues the W, x and mask boxes of a stage against one
-        // expected byte count.  (Separate producer warps arriving on the same
-        // barrier gave occasional wrong operands on B200; one did not.)
+        // One thread issues the W, x and mask boxes of a stage, each completing
+        // on a barrier of its own.  (Loads from several producer warps, or
+        // several loads completing on one barrier, gave occasional wrong
+        // operands on B200; one load per barrier from one thread did not.)
         if (lane == 0) {
-            const uint32_t bytes = (uint32_t)(L::W_BYTES + L::NKC * xr * 128 + (NM > 0 ? L::M_BYTES : 0));
+            const uint32_t xbytes = (uint32_t)(L::NKC * xr * 128);
             prefetch_tensormap(&tm_w);
             prefetch_tensormap(&tm_x);
             if (NM > 0)
@@ -348,14 +357,17 @@ __global__ void __launch_bounds__(Layout<NM, NT, NCW_, UPW_>::NTHREADS, 1)
                 const uint32_t ph = (uint32_t)(i / NSTAGES) & 1u;
                 if (!mbar_wait(&empty[s], ph ^ 1u))
                     break;
-                mbar_arrive_expect_tx(&full[s], bytes);
                 uint8_t *st = ring + s * STAGE;
                 const int k0 = ks * L::KS;
                 // boxes: W (0, k0/64, row0), x (0, k0/64, 0), masks (0, k0/128, row0)
+                mbar_arrive_expect_tx(&full[s], (uint32_t)L::W_BYTES);
                 tma_load_3d(st, &tm_w, &full[s], 0, k0 / 64, rb * ROWS);
-                tma_load_3d(st + L::X_OFF, &tm_x, &full[s], 0, k0 / 64, 0);
-                if constexpr (NM > 0)
-                    tma_load_3d(st + L::M_OFF, &tm_m, &full[s], 0, k0 / MASK_K, rb * ROWS);
+                mbar_arrive_expect_tx(&xfull[s], xbytes);
+                tma_load_3d(st + L::X_OFF, &tm_x, &xfull[s], 0, k0 / 64, 0);
+                if constexpr (NM > 0) {
+                    mbar_arrive_expect_tx(&mfull[s], (uint32_t)L::M_BYTES);
+                    tma_load_3d(st + L::M_OFF, &tm_m, &mfull[s], 0, k0 / MASK_K, rb * ROWS);
+                }
             }
         }
         return;
@@ -465,8 +477,13 @@ __global__ void __launch_bounds__(Layout<NM, NT, NCW_, UPW_>::NTHREADS, 1)
     for (int i = 0; i < sc.n; sc.next(i, rb, ks), ++i) {
         const int s = i % NSTAGES;
         const uint32_t ph = (uint32_t)(i / NSTAGES) & 1u;
-        if (ok && !mbar_wait_warp(&full[s], ph))
+        if (ok && !mbar_wait_warp3(&xfull[s], &full[s], NM > 0 ? &mfull[s] : nullptr, ph))
             ok = false;
+        // The stage was written through the async proxy (TMA) and is read
+        // below with ordinary loads: order the two proxies for this thread.
+        // (Without this fence, reads right after the wait occasionally saw
+        // stale operands on B200.)
+        fence_proxy_async_smem();
         if (ok) {
             const uint8_t *st = ring + s * STAGE;
             uint32_t wa[L::UPW][4], wb[L::UPW][4], xb[L::UPW][NT][4];

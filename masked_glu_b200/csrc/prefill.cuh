@@ -48,9 +48,9 @@ struct Cfg {
     static constexpr int MB = NM == 0 ? 0 : (BK * NM / 8 < 16 ? 16 : BK * NM / 8);  // mask bytes per row per stage
     static constexpr int M_BYTES = NJ * MB;
     static constexpr int STAGE = (A_BYTES + B_BYTES + M_BYTES + 1023) / 1024 * 1024;
-    static constexpr uint32_t TX = A_BYTES + NJ * BK * 2 + M_BYTES;
+    static constexpr uint32_t W_TX = NJ * BK * 2;  // bytes of one W box (the variant rows are built here)
     static constexpr int BAR_OFF = STAGES * STAGE;
-    static constexpr int SMEM = BAR_OFF + 256 + 1024;
+    static constexpr int SMEM = BAR_OFF + 512 + 1024;
     static constexpr int EC = NM >= 8 ? 8 : 16;  // epilogue columns per TMEM load round
     static_assert(N <= 256 && N % 16 == 0 && NJ % 8 == 0, "bad tile shape");
     static_assert(NJ % EC == 0, "epilogue chunking");
@@ -100,8 +100,11 @@ __global__ void __launch_bounds__(NTHREADS, 1) prefill_kernel(const __grid_const
     using C = Cfg<NM>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint64_t *full = reinterpret_cast<uint64_t *>(smem + C::BAR_OFF);
-    uint64_t *built = full + C::STAGES;
+    // one barrier per TMA load of a stage: x (A), W, masks
+    uint64_t *xfull = reinterpret_cast<uint64_t *>(smem + C::BAR_OFF);
+    uint64_t *full = xfull + C::STAGES;
+    uint64_t *mfull = full + C::STAGES;
+    uint64_t *built = mfull + C::STAGES;
     uint64_t *empty = built + C::STAGES;
     uint64_t *acc_full = empty + C::STAGES;
     uint64_t *acc_empty = acc_full + 2;
@@ -116,7 +119,9 @@ __global__ void __launch_bounds__(NTHREADS, 1) prefill_kernel(const __grid_const
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < C::STAGES; ++s) {
+            mbar_init(&xfull[s], 1);
             mbar_init(&full[s], 1);
+            mbar_init(&mfull[s], 1);
             mbar_init(&built[s], 4);
             mbar_init(&empty[s], 1);
         }
@@ -156,12 +161,16 @@ __global__ void __launch_bounds__(NTHREADS, 1) prefill_kernel(const __grid_const
                         break;
                     }
                     uint8_t *st = smem + s * C::STAGE;
-                    mbar_arrive_expect_tx(&full[s], C::TX);
-                    tma_load_2d(st, &tm_x, &full[s], kb * BK, m0);
+                    // each load completes on a barrier of its own (loads sharing a
+                    // barrier gave occasional wrong operands on B200)
+                    mbar_arrive_expect_tx(&xfull[s], C::A_BYTES);
+                    tma_load_2d(st, &tm_x, &xfull[s], kb * BK, m0);
+                    mbar_arrive_expect_tx(&full[s], C::W_TX);
                     tma_load_2d(st + C::A_BYTES, &tm_w, &full[s], kb * BK, n0);
                     if constexpr (NM > 0) {
                         const int mc = (kb * BK * NM / 8) / C::MB * C::MB;  // 16-byte aligned column
-                        tma_load_2d(st + C::A_BYTES + C::B_BYTES, &tm_m, &full[s], mc, n0);
+                        mbar_arrive_expect_tx(&mfull[s], C::M_BYTES);
+                        tma_load_2d(st + C::A_BYTES + C::B_BYTES, &tm_m, &mfull[s], mc, n0);
                     }
                 }
             }
@@ -182,7 +191,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) prefill_kernel(const __grid_const
                 for (int kb = 0; kb < nkb; ++kb, ++it) {
                     const int s = it % C::STAGES;
                     const uint32_t ph = (uint32_t)(it / C::STAGES) & 1u;
-                    if (!mbar_wait(NM > 0 ? &built[s] : &full[s], ph)) {
+                    if (!mbar_wait(NM > 0 ? &built[s] : &full[s], ph) || !mbar_wait(&xfull[s], ph)) {
                         ok = false;
                         break;
                     }
@@ -209,10 +218,11 @@ __global__ void __launch_bounds__(NTHREADS, 1) prefill_kernel(const __grid_const
                 for (int kb = 0; kb < nkb; ++kb, ++it) {
                     const int s = it % C::STAGES;
                     const uint32_t ph = (uint32_t)(it / C::STAGES) & 1u;
-                    if (!mbar_wait_warp(&full[s], ph)) {
+                    if (!mbar_wait_warp3(&full[s], &mfull[s], nullptr, ph)) {
                         ok = false;
                         break;
                     }
+                    fence_proxy_async_smem();  // TMA-written tiles are read with ordinary loads below
                     uint8_t *B = smem + s * C::STAGE + C::A_BYTES;
                     const uint8_t *Mt = B + C::B_BYTES;
                     const int moff = (kb * BK * NM / 8) % C::MB;  // nonzero only when NM = 1

@@ -101,6 +101,18 @@ __device__ __forceinline__ bool mbar_wait_warp(uint64_t *bar, uint32_t parity)
     return ok != 0;
 }
 
+// The same for the phase of up to three barriers (null ones are skipped):
+// lane 0 waits for each in turn, then one broadcast and warp synchronization.
+__device__ __forceinline__ bool mbar_wait_warp3(uint64_t *a, uint64_t *b, uint64_t *c, uint32_t parity)
+{
+    int ok = 1;
+    if ((threadIdx.x & 31) == 0)
+        ok = (mbar_wait(a, parity) && (!b || mbar_wait(b, parity)) && (!c || mbar_wait(c, parity))) ? 1 : 0;
+    ok = __shfl_sync(0xffffffffu, ok, 0);
+    __syncwarp();
+    return ok != 0;
+}
+
 // Make the calling thread hold `v` in a register here: every instruction that
 // produced it has completed (used to wait for outstanding loads).
 __device__ __forceinline__ void consume(uint32_t v) { asm volatile("" ::"r"(v) : "memory"); }

@@ -223,3 +223,42 @@ def test_decode_scratch_is_left_zeroed(T):
         counters = scratch[mglu.scratch_bytes(256) - 256:].cpu().numpy()
         assert not counters.any(), "scratch counters not reset"
     assert np.array_equal(outs[0], outs[1]) and np.array_equal(outs[1], outs[2]), "run-to-run difference"
+
+
+# Shapes on which an earlier form of the decode kernel gave intermittent wrong
+# rows (about one operand read in ten thousand, only when its consumer warps
+# outran the TMA): the dense down-projection with K = 14336, which mixes
+# data-parallel and split row blocks, n_m = 4 with a three-stage ring, and
+# n_m = 8 with two token blocks.  Every repeat must match the oracle and be
+# bit-identical to the first.
+@pytest.mark.parametrize("T", [1, 16])
+def test_dense_decode_repeatable_k14336(T):
+    rng = np.random.default_rng(900 + T)
+    hid = inputs.normal(rng, (T, 14336), 1.0, "bf16")
+    Wd = inputs.normal(rng, (4096, 14336), 0.02, "bf16")
+    hd, wd = to_device(hid), to_device(Wd)
+    ref = oracle.down(hid.values, Wd.values)
+    first = None
+    for rep in range(6):
+        y = to_f64(mglu.down_proj(hd, wd))
+        assert mglu.last_device_status() == 0
+        assert_close(y, ref, "bf16", f"dense decode K=14336 T={T} repeat {rep}")
+        if first is None:
+            first = y
+        assert np.array_equal(y, first), f"repeat {rep} differs from the first call"
+
+
+@pytest.mark.parametrize("n_m,T,d,h", [(4, 8, 2048, 8192), (4, 4, 2048, 8192), (2, 8, 2048, 4096),
+                                       (8, 16, 4096, 2048)])
+def test_decode_repeatable(n_m, T, d, h):
+    case = inputs.make_case(T, d, h, n_m, seed=950 + 31 * n_m + T)
+    x, W, packed, _ = device_case(case)
+    ref, _ = oracle.forward(case.x.values, case.W.values, oracle_packed(case), n_m, ACT["swish"])
+    first = None
+    for rep in range(8):
+        got = to_f64(mglu.forward(x, W, packed, n_m, "swish"))
+        assert mglu.last_device_status() == 0
+        assert_close(got, ref, "bf16", f"decode n_m={n_m} T={T} repeat {rep}")
+        if first is None:
+            first = got
+        assert np.array_equal(got, first), f"repeat {rep} differs from the first call"
