@@ -52,16 +52,15 @@ constexpr int BAR_SLOTS_FREE = 2;     // finisher arrives, consumers wait
 constexpr int MASK_K = 128;           // k covered by one row of a mask box
 
 // Default consumer warps / 32-k units per warp and stage, chosen by timing on
-// B200.  The math of a unit is bound by instruction issue, so more warps do
-// not make it faster; fewer warps that each take more units per stage mean
-// fewer accumulator slots to reduce and leave shared memory for a deeper
-// ring: one warp per SM quadrant with eight units (1024 k per stage) for
-// n_m <= 4, eight warps with two units (512 k) for n_m = 8 and for two token
-// blocks.
+// B200.  The math of a unit is bound by instruction issue, so more warps help
+// only by hiding the per-stage wait and load latency, while fewer warps leave
+// fewer accumulator slots to reduce and more shared memory for the ring:
+// eight warps with four units (1024 k per stage) for n_m <= 4, twelve with two
+// (768 k) for n_m = 8, eight with two (512 k) for two token blocks.
 template <int NM, int NT>
 struct DefaultShape {
-    static constexpr int NCW = NT == 2 ? 8 : NM == 8 ? 8 : 4;
-    static constexpr int UPW = NT == 2 ? 2 : NM == 8 ? 2 : 8;
+    static constexpr int NCW = NT == 2 ? 8 : NM == 8 ? 12 : 8;
+    static constexpr int UPW = NT == 2 ? 2 : NM == 8 ? 2 : 4;
 };
 
 constexpr int MAX_STAGES = 12;
