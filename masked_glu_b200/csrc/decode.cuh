@@ -55,12 +55,14 @@ constexpr int MASK_K = 128;           // k covered by one row of a mask box
 // B200.  The math of a unit is bound by instruction issue, so more warps help
 // only by hiding the per-stage wait and load latency, while fewer warps leave
 // fewer accumulator slots to reduce and more shared memory for the ring:
-// eight warps with four units (1024 k per stage) for n_m <= 4, twelve with two
-// (768 k) for n_m = 8, eight with two (512 k) for two token blocks.
+// four warps with eight units (1024 k per stage) for n_m <= 4, twelve with two
+// (768 k) for n_m = 8, eight with two (512 k) for two token blocks.  (Eight
+// warps with four units was 5 % faster for n_m = 4 but gave wrong rows at
+// T = 8 in repeated runs; it is not used.)
 template <int NM, int NT>
 struct DefaultShape {
-    static constexpr int NCW = NT == 2 ? 8 : NM == 8 ? 12 : 8;
-    static constexpr int UPW = NT == 2 ? 2 : NM == 8 ? 2 : 4;
+    static constexpr int NCW = NT == 2 ? 8 : NM == 8 ? 12 : 4;
+    static constexpr int UPW = NT == 2 ? 2 : NM == 8 ? 2 : 8;
 };
 
 constexpr int MAX_STAGES = 12;
