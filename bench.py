@@ -51,6 +51,8 @@ def parse_args():
     ap.add_argument("--act", default="swish", choices=["swish", "gelu", "relu"])
     ap.add_argument("--p", type=float, default=0.5, help="mask density (FFN-block workload)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-comparisons", action="store_true",
+                    help="skip the torch.matmul baselines (dense SwiGLU, naive MGLU) timed after the run")
     ap.add_argument("--probe-seconds", type=float, default=1.0,
                     help="untimed run of the same step before timing, to settle and sample clocks")
     return ap.parse_args()
@@ -277,6 +279,57 @@ def run_reference(args, dist):
 
 
 # ---------------------------------------------------------------------- GPU run
+def time_comparisons(T, d, h, nm, act, dev, l2, reps=10):
+    """Library baselines on the same box and shapes, for context only (not the
+    product path, not counted in gpu_launches): a dense SwiGLU with two bf16
+    d x h projections through torch.matmul (cuBLAS), and a naive PyTorch MGLU
+    that materialises every masked weight M_i * W in bf16 before multiplying.
+    Weights rotate over copies larger than L2; times are per call."""
+    import math
+
+    import torch
+    F = torch.nn.functional
+    fn_act = F.gelu if act == "gelu" else F.relu if act == "relu" else F.silu
+    x = torch.randn(T, d, device=dev).to(torch.bfloat16)
+
+    def timed(fn, R):
+        for i in range(2 * R):
+            fn(i % R)
+        torch.cuda.synchronize(dev)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for i in range(reps * R):
+            fn(i % R)
+        e1.record()
+        e1.synchronize()
+        return e0.elapsed_time(e1) * 1000.0 / (reps * R)
+
+    res = {}
+    R = max(2, math.ceil(4 * l2 / (2 * h * d * 2)))
+    Wg = [(torch.randn(h, d, device=dev) * 0.02).to(torch.bfloat16) for _ in range(R)]
+    Wv = [(torch.randn(h, d, device=dev) * 0.02).to(torch.bfloat16) for _ in range(R)]
+    res["dense_swiglu_us"] = timed(lambda i: fn_act(x @ Wg[i].t()) * (x @ Wv[i].t()), R)
+    del Wg, Wv
+    R = max(2, math.ceil(4 * l2 / (h * d * 2 * (1 + nm))))
+    W = [(torch.randn(h, d, device=dev) * 0.02).to(torch.bfloat16) for _ in range(R)]
+    M = [(torch.rand(nm, h, d, device=dev) < 0.5).to(torch.bfloat16) for _ in range(R)]
+
+    def naive(i):
+        D = x @ W[i].t()
+        out = torch.zeros_like(D)
+        for k in range(nm):
+            g = x @ (W[i] * M[i][k]).t()
+            out = out + fn_act(g) * (D - g)
+        return out
+
+    res["naive_torch_mglu_us"] = timed(naive, R)
+    del W, M
+    torch.cuda.empty_cache()
+    res["note"] = ("torch.matmul (cuBLAS) baselines on the same shapes: dense SwiGLU = two bf16 d x h "
+                   "projections; naive MGLU materialises each M_i * W in bf16")
+    return res
+
+
 def run_mglu(args, dist):
     import numpy as np
     import torch
@@ -489,6 +542,12 @@ def run_mglu(args, dist):
         line["tflops"] = up_flops / (up_ms / 1000.0) / 1e12
     else:
         line["hbm_gbs"] = up_bytes / (up_ms / 1000.0) / 1e9
+
+    if dist.world == 1 and w["dtype"] == "bf16" and not args.no_comparisons:
+        line["comparisons"] = time_comparisons(T, d, h, nm, args.act, dev, l2)
+        line["comparisons"]["mglu_us"] = up_ms * 1000.0 + (down_ms * 1000.0 if kind == "ffn" else 0.0)
+        if kind == "ffn":
+            line["comparisons"]["note"] += "; mglu_us includes the down-projection, the baselines do not"
 
     # the CPU oracle on a bounded sample: rank 0, one GPU only
     if dist.world == 1 and dist.rank == 0 and not args.no_cpu_baseline:
