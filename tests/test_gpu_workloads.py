@@ -99,3 +99,18 @@ def test_ffn_block_d4096_h14336_nm8(c5, T):
     ref = oracle.down_elems(hid, case.W_down.values, rows, cols)
     got = y[np.repeat(toks, case.d), cols]
     assert_close(got, ref, "bf16", f"ffn block T={T} p={p}", exact_check=False)
+
+
+# Edge sizes: the widest Llama-style FFN hidden (h = 53248) and a very deep
+# reduction (d = 16384), through the decode and tensor-core paths, checked on
+# whole output rows of chosen tokens plus random elements.
+@pytest.mark.parametrize("n_m,T,d,h", [(4, 1, 2048, 53248), (8, 16, 1024, 53248), (2, 5, 16384, 1024),
+                                       (4, 300, 16384, 512), (1, 33, 256, 53248)])
+def test_edge_sizes(n_m, T, d, h):
+    case = inputs.make_case(T, d, h, n_m, seed=4100 + n_m + T)
+    x, W, packed, _ = device_case(case)
+    got = to_f64(mglu.forward(x, W, packed, n_m, "swish"))
+    assert mglu.last_device_status() == 0
+    b, j = sample(T, h, [0, T - 1], 3000, seed=T + h)
+    ref, _ = oracle.forward_elems(case.x.values, case.W.values, oracle_packed(case), n_m, ACT["swish"], b, j)
+    assert_close(got[b, j], ref, "bf16", f"edge n_m={n_m} T={T} d={d} h={h}")
