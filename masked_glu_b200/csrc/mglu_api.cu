@@ -288,7 +288,7 @@ int launch_prefill(const void *x, int64_t T, int64_t d, const void *W, int64_t r
     const int64_t tiles = ((T + mglu::pf::BM - 1) / mglu::pf::BM) * ((rows + C::NJ - 1) / C::NJ);
     const int grid = (int)(tiles < sm_count(dev) ? tiles : sm_count(dev));
     (void)kernel;
-    return launch_pdl(mglu::pf::prefill_kernel<NM>, dim3((unsigned)grid), dim3(mglu::pf::NTHREADS), C::SMEM, s,
+    return launch_pdl(mglu::pf::prefill_kernel<NM>, dim3((unsigned)grid), dim3(mglu::pf::Cfg<NM>::NTHREADS), C::SMEM, s,
                       "prefill launch", tx, tw, tm, (int)T, (int)rows, (int)d, act,
                       reinterpret_cast<__nv_bfloat16 *>(out));
 }

@@ -14,9 +14,9 @@
 //   warp 0      TMA producer: x tile (128 tokens x 64 k), W tile (NJ x 64),
 //               packed-mask tile, into a ring of STAGES shared-memory stages
 //   warp 1      TMEM allocator and the single thread that issues tcgen05.mma
-//   warps 2-5   builders: write the NM masked copies of the W tile next to
+//   warps 2..    builders (8 warps for n_m <= 4, else 4): write the NM masked copies of the W tile next to
 //               it in shared memory (same 128-byte swizzle), then signal
-//   warps 6-9   epilogue: tcgen05.ld the accumulators, out = sum_i
+//   last 4 warps epilogue: tcgen05.ld the accumulators, out = sum_i
 //               act(g_i)(D - g_i), bf16 stores; overlaps the next tile's
 //               MMAs through a double-buffered accumulator
 #pragma once
@@ -31,7 +31,6 @@ namespace pf {
 
 constexpr int BM = 128;  // tokens per tile (UMMA M)
 constexpr int BK = 64;   // k per stage: one 128-byte swizzle atom of bf16
-constexpr int NTHREADS = 320;
 constexpr int TMEM_COLS = 512;
 constexpr int ACC_STRIDE = 256;  // TMEM columns between the two accumulator buffers
 
@@ -52,6 +51,11 @@ struct Cfg {
     static constexpr int BAR_OFF = STAGES * STAGE;
     static constexpr int SMEM = BAR_OFF + 512 + 1024;
     static constexpr int EC = NM >= 8 ? 8 : 16;  // epilogue columns per TMEM load round
+    // warps: 0 TMA, 1 TMEM + MMA, then NBW builders, then 4 epilogue warps.
+    // Eight builders were 7 % faster than four for n_m = 4 and 2 % slower for
+    // n_m = 8 (timed on B200); the dense kernel has nothing to build.
+    static constexpr int NBW = NM == 8 || NM == 0 ? 4 : 8;
+    static constexpr int NTHREADS = (2 + NBW + 4) * 32;
     static_assert(N <= 256 && N % 16 == 0 && NJ % 8 == 0, "bad tile shape");
     static_assert(NJ % EC == 0, "epilogue chunking");
     static_assert(SMEM <= 227 * 1024, "shared memory");
@@ -91,7 +95,7 @@ __device__ __forceinline__ void build_variants(uint8_t *B, int off, uint4 w, uin
 }
 
 template <int NM>
-__global__ void __launch_bounds__(NTHREADS, 1) prefill_kernel(const __grid_constant__ CUtensorMap tm_x,
+__global__ void __launch_bounds__(Cfg<NM>::NTHREADS, 1) prefill_kernel(const __grid_constant__ CUtensorMap tm_x,
                                                               const __grid_constant__ CUtensorMap tm_w,
                                                               const __grid_constant__ CUtensorMap tm_m, int T,
                                                               int rows, int d, int act,
@@ -122,7 +126,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) prefill_kernel(const __grid_const
             mbar_init(&xfull[s], 1);
             mbar_init(&full[s], 1);
             mbar_init(&mfull[s], 1);
-            mbar_init(&built[s], 4);
+            mbar_init(&built[s], C::NBW);
             mbar_init(&empty[s], 1);
         }
         for (int b = 0; b < 2; ++b) {
@@ -208,10 +212,10 @@ __global__ void __launch_bounds__(NTHREADS, 1) prefill_kernel(const __grid_const
                     umma_commit(&acc_full[b]);
             }
         }
-    } else if (warp < 6) {
+    } else if (warp < 2 + C::NBW) {
         // ---------------------------------------------------------- builders
         if constexpr (NM > 0) {
-            const int bt = threadIdx.x - 64;  // 0..127
+            const int bt = threadIdx.x - 64;  // 0 .. 32 * NBW - 1
             int it = 0;
             bool ok = true;
             for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
@@ -226,7 +230,7 @@ __global__ void __launch_bounds__(NTHREADS, 1) prefill_kernel(const __grid_const
                     uint8_t *B = smem + s * C::STAGE + C::A_BYTES;
                     const uint8_t *Mt = B + C::B_BYTES;
                     const int moff = (kb * BK * NM / 8) % C::MB;  // nonzero only when NM = 1
-                    for (int item = bt; item < C::NJ * 8; item += 128) {
+                    for (int item = bt; item < C::NJ * 8; item += 32 * C::NBW) {
                         const int r = item >> 3, c = item & 7;
                         const int off = r * 128 + ((c ^ (r & 7)) << 4);
                         const uint4 w = *reinterpret_cast<const uint4 *>(B + off);
