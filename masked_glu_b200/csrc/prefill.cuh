@@ -14,7 +14,7 @@
 //   warp 0      TMA producer: x tile (128 tokens x 64 k), W tile (NJ x 64),
 //               packed-mask tile, into a ring of STAGES shared-memory stages
 //   warp 1      TMEM allocator and the single thread that issues tcgen05.mma
-//   warps 2..    builders (8 warps for n_m <= 4, else 4): write the NM masked copies of the W tile next to
+//   warps 2..    builders (6 to 12 warps by n_m): write the NM masked copies of the W tile next to
 //               it in shared memory (same 128-byte swizzle), then signal
 //   last 4 warps epilogue: tcgen05.ld the accumulators, out = sum_i
 //               act(g_i)(D - g_i), bf16 stores; overlaps the next tile's
@@ -50,11 +50,15 @@ struct Cfg {
     static constexpr uint32_t W_TX = NJ * BK * 2;  // bytes of one W box (the variant rows are built here)
     static constexpr int BAR_OFF = STAGES * STAGE;
     static constexpr int SMEM = BAR_OFF + 512 + 1024;
-    static constexpr int EC = NM >= 8 ? 8 : 16;  // epilogue columns per TMEM load round
     // warps: 0 TMA, 1 TMEM + MMA, then NBW builders, then 4 epilogue warps.
-    // Eight builders were 7 % faster than four for n_m = 4 and 2 % slower for
-    // n_m = 8 (timed on B200); the dense kernel has nothing to build.
-    static constexpr int NBW = NM == 8 || NM == 0 ? 4 : 8;
+    // A stage has NJ * 8 build items (16-byte pieces of the W tile); builder
+    // counts that split them into whole rounds were fastest on B200 (n_m = 4:
+    // 384 items, 12 warps, 966 TFLOP/s against 842 with 4 warps); the dense
+    // kernel has nothing to build.
+    static constexpr int NBW = NM == 0 ? 4 : NM == 8 ? 6 : NM == 4 ? 12 : NM == 2 ? 10 : 8;
+    // epilogue columns per TMEM load round (8 where the register budget of the
+    // larger block is tight)
+    static constexpr int EC = NM >= 4 ? 8 : 16;
     static constexpr int NTHREADS = (2 + NBW + 4) * 32;
     static_assert(N <= 256 && N % 16 == 0 && NJ % 8 == 0, "bad tile shape");
     static_assert(NJ % EC == 0, "epilogue chunking");
