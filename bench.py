@@ -461,18 +461,18 @@ def run_mglu(args, dist):
     x_h.copy_(x.cpu())
     res = y if kind == "ffn" else out
     res_h = torch.empty(res.shape, dtype=tdt, pin_memory=True)
-    x_dev = torch.empty_like(x)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     stream = torch.cuda.current_stream(dev)
 
+    # the public host-buffer call: one library call per step copies x in,
+    # runs the kernels and copies the result out, in order on the stream
+    ws_host = torch.zeros(max(256, mglu.host_workspace_bytes(T, d, h, nm, tdt, kind == "ffn")), dtype=torch.uint8,
+                          device=dev)
+
     def e2e_step(i):
         r = i % R
-        x_dev.copy_(x_h, non_blocking=True)
-        if kind == "ffn":
-            mglu.forward_down(x_dev, Ws[r], pks[r], nm, Wds[r], args.act, workspace=ws, out=y)
-        else:
-            mglu.forward(x_dev, Ws[r], pks[r], nm, args.act, out=out, scratch=scratch)
-        res_h.copy_(res, non_blocking=True)
+        mglu.forward_host(x_h, Ws[r], pks[r], nm, args.act, W_down=Wds[r] if kind == "ffn" else None,
+                          out_host=res_h, workspace=ws_host)
 
     for i in range(args.warmup):
         e2e_step(i)
@@ -530,7 +530,7 @@ def run_mglu(args, dist):
         "gpu_launches": K * (2 if kind == "ffn" else 1),
         "timing": "device-side: one CUDA-graph replay of the K steps back to back (CUDA events around the "
                   "replay); kernel_us_isolated: a second replay with event nodes around each kernel; "
-                  "e2e: eager calls through the Python binding with pinned host copies",
+                  "e2e: one mglu_forward_host call per step (pinned host x in, kernels, pinned host result out)",
         "clocks": clocks,
         "host_us_per_forward_call": host_us,
         "device_status": status,

@@ -190,6 +190,35 @@ int mglu_forward_decode_static(const void *x, int64_t T, int64_t d,
                                const void *W, int64_t h, const uint8_t *packed,
                                int n_m, int act, void *out, void *stream);
 
+/*
+ * Device workspace mglu_forward_host needs: a staging copy of x, the device
+ * result, and the decode scratch (plus the hidden activation when
+ * with_down != 0).  0 for bad input.
+ */
+size_t mglu_host_workspace_bytes(int64_t T, int64_t d, int64_t h, int n_m,
+                                 int dtype, int with_down);
+
+/*
+ * The forward (W_down == NULL) or the FFN block (W_down != NULL) on HOST
+ * activations: copies x_host [T][d] to the device, runs mglu_forward or
+ * mglu_forward_down, and copies the result back to result_host ([T][h], or
+ * [T][d] with W_down), all in order on `stream` (cudaMemcpyAsync, then the
+ * kernels, then cudaMemcpyAsync).  W, packed and W_down are device pointers
+ * as for mglu_forward.  The call returns before the copies finish:
+ * x_host must stay unchanged and result_host is written when the stream
+ * reaches the end of the call (synchronize before reading it).  Pinned host
+ * memory (cudaHostAlloc) makes both copies asynchronous; pageable memory
+ * works but the copies then block the calling thread.
+ *   workspace: device, 256-byte aligned, >= mglu_host_workspace_bytes(...),
+ *   zero-filled before its first use (it holds the decode scratch).
+ * Nothing is allocated.  Errors: as mglu_forward / mglu_forward_down, plus
+ * INVALID for a missing or small workspace or a NULL host pointer.
+ */
+int mglu_forward_host(const void *x_host, int64_t T, int64_t d, const void *W,
+                      int64_t h, const uint8_t *packed, int n_m, int act,
+                      int dtype, const void *W_down, void *workspace,
+                      size_t workspace_bytes, void *result_host, void *stream);
+
 /* Which kernel family mglu_forward uses for T tokens of `dtype`. */
 int mglu_forward_path(int64_t T, int dtype);
 

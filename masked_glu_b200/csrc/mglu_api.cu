@@ -602,6 +602,60 @@ int mglu_forward_decode_static(const void *x, int64_t T, int64_t d, const void *
     return by_nm<DecodeF>(n_m, x, T, d, W, h, packed, act, out, ws, s);
 }
 
+size_t mglu_host_workspace_bytes(int64_t T, int64_t d, int64_t h, int n_m, int dtype, int with_down)
+{
+    if (T < 0 || d <= 0 || h <= 0 || (dtype != MGLU_BF16 && dtype != MGLU_F32))
+        return 0;
+    const size_t es = dtype == MGLU_BF16 ? 2u : 4u;
+    const size_t xb = ((size_t)T * (size_t)d * es + 255) / 256 * 256;
+    const size_t rb = ((size_t)T * (size_t)(with_down ? d : h) * es + 255) / 256 * 256;
+    const size_t rest = with_down ? mglu_workspace_bytes(T, d, h, n_m, dtype) : scratch_bytes(h);
+    return xb + rb + rest;
+}
+
+int mglu_forward_host(const void *x_host, int64_t T, int64_t d, const void *W, int64_t h, const uint8_t *packed,
+                      int n_m, int act, int dtype, const void *W_down, void *workspace, size_t workspace_bytes,
+                      void *result_host, void *stream)
+{
+    if (T < 0 || d <= 0 || h <= 0 || (dtype != MGLU_BF16 && dtype != MGLU_F32))
+        return MGLU_ERR_INVALID;
+    if (T == 0)
+        return MGLU_OK;
+    if (!x_host || !result_host || !workspace)
+        return MGLU_ERR_INVALID;
+    const int with_down = W_down != nullptr;
+    if (workspace_bytes < mglu_host_workspace_bytes(T, d, h, n_m, dtype, with_down))
+        return MGLU_ERR_INVALID;
+    if (!aligned(workspace, 256))
+        return MGLU_ERR_ALIGN;
+    const size_t es = dtype == MGLU_BF16 ? 2u : 4u;
+    const size_t xbytes = (size_t)T * (size_t)d * es;
+    const size_t rbytes = (size_t)T * (size_t)(with_down ? d : h) * es;
+    uint8_t *base = reinterpret_cast<uint8_t *>(workspace);
+    void *x_dev = base;
+    void *r_dev = base + (xbytes + 255) / 256 * 256;
+    uint8_t *rest = reinterpret_cast<uint8_t *>(r_dev) + (rbytes + 255) / 256 * 256;
+    const size_t rest_bytes = workspace_bytes - (size_t)(rest - base);
+    // every argument is checked before anything is queued
+    int rc = check_forward(x_dev, T, d, W, h, packed, n_m, act, dtype, with_down ? (const void *)rest : r_dev);
+    if (rc)
+        return rc;
+    if (with_down && (rc = check_down(rest, T, h, W_down, d, dtype, r_dev)))
+        return rc;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    cudaError_t e = cudaMemcpyAsync(x_dev, x_host, xbytes, cudaMemcpyHostToDevice, s);
+    if (e != cudaSuccess)
+        return cuda_fail(e, "copy x to the device");
+    rc = with_down ? mglu_forward_down(x_dev, T, d, W, h, packed, n_m, act, dtype, W_down, rest, rest_bytes, r_dev,
+                                       stream)
+                   : mglu_forward(x_dev, T, d, W, h, packed, n_m, act, dtype, r_dev, rest, rest_bytes, stream);
+    if (rc)
+        return rc;
+    if ((e = cudaMemcpyAsync(result_host, r_dev, rbytes, cudaMemcpyDeviceToHost, s)) != cudaSuccess)
+        return cuda_fail(e, "copy the result to the host");
+    return MGLU_OK;
+}
+
 int mglu_forward_path(int64_t T, int dtype) { return path_for(T, dtype); }
 
 int mglu_set_decode_max_tokens(int t)

@@ -60,6 +60,8 @@ def lib() -> ctypes.CDLL:
             "mglu_workspace_bytes": (SZ, [I64, I64, I64, I32, I32]),
             "mglu_forward_down": (I32, [P, I64, I64, P, I64, P, I32, I32, I32, P, P, SZ, P, P]),
             "mglu_forward_decode_static": (I32, [P, I64, I64, P, I64, P, I32, I32, P, P]),
+            "mglu_host_workspace_bytes": (SZ, [I64, I64, I64, I32, I32, I32]),
+            "mglu_forward_host": (I32, [P, I64, I64, P, I64, P, I32, I32, I32, P, P, SZ, P, P]),
             "mglu_forward_path": (I32, [I64, I32]),
             "mglu_set_decode_max_tokens": (I32, [I32]),
             "mglu_last_device_status": (I32, [P]),
@@ -98,6 +100,12 @@ def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:
         return None
     if not (t.is_cuda and t.is_contiguous()):
         raise ValueError("tensors must be contiguous and on a CUDA device")
+    return t.data_ptr()
+
+
+def _hptr(t: torch.Tensor) -> int:
+    if t.is_cuda or not t.is_contiguous():
+        raise ValueError("host tensors must be contiguous CPU tensors")
     return t.data_ptr()
 
 
@@ -219,6 +227,32 @@ def forward_down(x: torch.Tensor, W: torch.Tensor, packed: torch.Tensor, n_m: in
                                    _ptr(W_down), _ptr(workspace), workspace.numel() * workspace.element_size(),
                                    _ptr(out), _stream(stream)), "mglu_forward_down")
     return out
+
+
+def host_workspace_bytes(T: int, d: int, h: int, n_m: int, dtype=torch.bfloat16, with_down=False) -> int:
+    return int(lib().mglu_host_workspace_bytes(T, d, h, n_m, DTYPES[dtype], 1 if with_down else 0))
+
+
+def forward_host(x_host: torch.Tensor, W: torch.Tensor, packed: torch.Tensor, n_m: int, act="swish",
+                 W_down: Optional[torch.Tensor] = None, out_host: Optional[torch.Tensor] = None,
+                 workspace: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """The forward (or, with W_down, the FFN block) on host activations: one
+    library call copies x_host to the device, runs the kernels and copies the
+    result into out_host, in order on the stream.  Pin the host tensors for
+    asynchronous copies; out_host is valid after the stream synchronizes."""
+    T, d = x_host.shape
+    h = W.shape[0]
+    if x_host.is_cuda or (out_host is not None and out_host.is_cuda):
+        raise ValueError("x_host and out_host must be host tensors")
+    if out_host is None:
+        out_host = torch.empty((T, d if W_down is not None else h), dtype=x_host.dtype, pin_memory=True)
+    need = host_workspace_bytes(T, d, h, n_m, x_host.dtype, W_down is not None)
+    if workspace is None:
+        workspace = torch.zeros(max(need, 256), dtype=torch.uint8, device=W.device)
+    _check(lib().mglu_forward_host(_hptr(x_host), T, d, _ptr(W), h, _ptr(packed), n_m, _act(act), _dtype(x_host),
+                                   _ptr(W_down), _ptr(workspace), _nbytes(workspace), _hptr(out_host),
+                                   _stream(stream)), "mglu_forward_host")
+    return out_host
 
 
 def forward_path(T: int, dtype=torch.bfloat16) -> int:

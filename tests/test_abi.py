@@ -149,3 +149,20 @@ def test_decode_schedule_host_check(tmp_path):
                     "-o", str(exe), os.path.join(ROOT, "tests", "native", "sched_check.cpp")], check=True)
     r = subprocess.run([str(exe)], capture_output=True, text=True)
     assert r.returncode == 0 and r.stdout.strip() == "ok", r.stdout
+
+
+def test_forward_host_rejects_before_any_copy():
+    """Argument errors of the host-buffer entry point come back before any
+    copy or launch is queued (no device is touched)."""
+    L = mglu.lib()
+    p = ctypes.c_void_p(1 << 20)
+    need = L.mglu_host_workspace_bytes(2, 128, 64, 4, 0, 0)
+    assert need > 0
+    assert L.mglu_host_workspace_bytes(2, 128, 64, 4, 0, 1) > need   # the block also stages the hidden
+    args = lambda xh, ws, wsb, rh: L.mglu_forward_host(xh, 2, 128, p, 64, p, 4, 0, 0, None, ws, wsb, rh, None)
+    assert args(None, p, need, p) == -1                  # no host input
+    assert args(p, p, need, None) == -1                  # no host result
+    assert args(p, None, need, p) == -1                  # no workspace
+    assert args(p, p, need - 1, p) == -1                 # workspace too small
+    assert args(p, ctypes.c_void_p((1 << 20) + 16), need, p) == -3   # workspace not 256-byte aligned
+    assert L.mglu_forward_host(p, 0, 128, p, 64, p, 4, 0, 0, None, p, need, p, None) == 0   # T == 0: no-op

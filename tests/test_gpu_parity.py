@@ -262,3 +262,23 @@ def test_decode_repeatable(n_m, T, d, h):
         if first is None:
             first = got
         assert np.array_equal(got, first), f"repeat {rep} differs from the first call"
+
+
+@pytest.mark.parametrize("n_m,T,d,h,down", [(4, 1, 1024, 640, False), (8, 9, 512, 300, False),
+                                            (2, 40, 384, 200, False), (8, 16, 256, 1024, True),
+                                            (4, 200, 256, 512, True)])
+def test_forward_host_matches_device_calls(n_m, T, d, h, down):
+    """The host-buffer entry point gives the same bits as the device-pointer
+    calls (same kernels), with the copies done inside the library call."""
+    case = inputs.make_case(T, d, h, n_m, seed=1200 + T + n_m, with_down=down)
+    x, W, packed, Wd = device_case(case)
+    x_h = x.cpu().pin_memory()
+    if down:
+        want = mglu.forward_down(x, W, packed, n_m, Wd, "swish")
+        got = mglu.forward_host(x_h, W, packed, n_m, "swish", W_down=Wd)
+    else:
+        want = mglu.forward(x, W, packed, n_m, "swish")
+        got = mglu.forward_host(x_h, W, packed, n_m, "swish")
+    torch.cuda.synchronize()
+    assert mglu.last_device_status() == 0
+    assert torch.equal(got, want.cpu())
