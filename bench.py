@@ -92,12 +92,19 @@ def load_peaks():
 
 
 def kernel_source_hash():
+    """Hash of the CUDA sources with comments and blank space removed, so a
+    recorded ncu capture stays valid across comment edits but not across any
+    change to the code."""
+    import re
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "masked_glu_b200", "csrc")
     for name in sorted(os.listdir(csrc)):
         if name.endswith((".cu", ".cuh")):
-            with open(os.path.join(csrc, name), "rb") as f:
-                h.update(name.encode() + f.read())
+            with open(os.path.join(csrc, name)) as f:
+                text = f.read()
+            text = re.sub(r"/\*.*?\*/", " ", text, flags=re.S)
+            text = re.sub(r"//[^\n]*", " ", text)
+            h.update(name.encode() + " ".join(text.split()).encode())
     return h.hexdigest()[:16]
 
 

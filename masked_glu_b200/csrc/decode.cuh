@@ -6,35 +6,40 @@
 // are read exactly once and the masks are unpacked inside the kernel):
 //
 //  * Work is made of units (row block of ROWS = 16 rows of W, k-stage of
-//    KS = 512 (256 for 9..16 tokens)).  A persistent grid of one CTA per SM
-//    splits it evenly: every CTA gets the same number of whole row blocks
-//    (data-parallel part) plus an equal contiguous share of the units of the
-//    remaining row blocks (stream-K part), so all SMs stream the same number
-//    of bytes.  Each CTA does its stream-K share first, so the combining of
-//    row blocks split between CTAs overlaps the data-parallel part instead of
-//    trailing the kernel.
-//  * A producer warp streams the CTA's share through a deep ring of
-//    shared-memory stages with three TMA loads per stage, issued together by
-//    three lanes: the W tile (16 rows x KS, as KS/64 boxes of 64 k with the
-//    128-byte swizzle), the x tile (the T token rows x KS) and
-//    the packed-mask tile of the same rows and k.  It does not pause at
-//    row-block boundaries.
-//  * Sixteen consumer warps (eight for 9..16 tokens) each take 32 k of a stage.  A lane loads 8
-//    consecutive weights of two rows, turns each mask's bits into bf16x2 lane
-//    masks (pair_mask: two shifts and one prmt per register) and feeds W and
-//    the NM masked copies of W as the A operand of mma.sync m16n8k16, with
-//    the tokens as B.  One dense product D and NM gate products g_i
-//    accumulate in fp32; the value of mask i is D - g_i.  The tensor cores
-//    only do the k reduction here; HBM bandwidth bounds the kernel.
+//    KS k: 1024 for n_m <= 4, 768 for n_m = 8, 512 for 9..16 tokens).  A
+//    persistent grid of one CTA per SM splits it evenly: every CTA gets the
+//    same number of whole row blocks (data-parallel part) plus an equal
+//    contiguous share of the units of the remaining row blocks (stream-K
+//    part), so all SMs stream the same number of bytes.  Each CTA does its
+//    stream-K share first, so the combining of row blocks split between CTAs
+//    overlaps the data-parallel part instead of trailing the kernel.
+//  * One producer thread streams the CTA's share through a ring of
+//    shared-memory stages: per stage a W box (16 rows x KS, 128-byte
+//    swizzle), an x box (the token rows x KS) and a packed-mask box of the
+//    same rows and k, each completing on an mbarrier of its own.
+//  * The consumer warps (4 for n_m <= 4, 12 for n_m = 8, 8 for 9..16 tokens)
+//    each take 32 * UPW k of a stage.  A lane loads 8 consecutive weights of
+//    two rows, turns each mask's bits into bf16x2 masks (AND masks for
+//    n_m <= 4, exponent-bit scales for n_m = 8) and feeds W and the NM masked
+//    copies of W as the A operand of mma.sync m16n8k16, with the tokens as
+//    B.  One dense product D and NM gate products g_i accumulate in fp32;
+//    the value of mask i is D - g_i.  The SM's instruction issue (mask
+//    building plus the HMMAs) and the per-stage synchronization bound the
+//    kernel; every weight and mask byte is read once.
 //  * At the end of a row block the consumers drop their accumulators into
 //    shared-memory slots and carry on; a finisher warp adds the slots in a
 //    fixed order.  A row block whose k range lies inside one CTA is
 //    finished there: out = sum_i act(g_i) (D - g_i), rounded once to bf16.
 //    A row block split between CTAs (only at the two ends of a stream-K
-//    share) is finished by whichever of its CTAs arrives last: the others' partial
-//    sums come from a small global scratch, added in CTA order, so the result
-//    does not depend on arrival order.  The arrival counter is reset by the
-//    finishing CTA, leaving the scratch zeroed.
+//    share) is finished by whichever of its CTAs arrives last: the others'
+//    partial sums come from a small global scratch, added in CTA order, so
+//    the result does not depend on arrival order.  The arrival counter is
+//    reset by the finishing CTA, leaving the scratch zeroed.
+//  * The synchronization follows rules found necessary on B200 (each is
+//    stated where it applies): one TMA load per mbarrier, one producer
+//    thread, one polling lane per consumer warp, a proxy fence before
+//    ordinary loads of a TMA-written stage, and release of a stage only once
+//    its loads have returned.
 #pragma once
 #include <cstdint>
 #include <cuda_bf16.h>
