@@ -464,22 +464,30 @@ def run_mglu(args, dist):
     up_ms = ms_per_step if kind != "ffn" else dist.max(up_iso_ms, dev)
 
     # end to end: pinned host x in, result out, every step
-    x_h = torch.empty((T, d), dtype=tdt, pin_memory=True)
-    x_h.copy_(x.cpu())
     res = y if kind == "ffn" else out
-    res_h = torch.empty(res.shape, dtype=tdt, pin_memory=True)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     stream = torch.cuda.current_stream(dev)
 
-    # the public host-buffer call: one library call per step copies x in,
-    # runs the kernels and copies the result out, in order on the stream
-    ws_host = torch.zeros(max(256, mglu.host_workspace_bytes(T, d, h, nm, tdt, kind == "ffn")), dtype=torch.uint8,
-                          device=dev)
+    # The public host-buffer call: one library call per step copies that
+    # step's x in from pinned host memory, runs the kernels and copies the
+    # result out, in order on its stream.  Consecutive steps alternate over
+    # two streams (each with its own pinned buffers and workspace), as a
+    # serving loop pipelines requests: one step's copies overlap the other's
+    # kernels.
+    NS = 2
+    e2e_streams = [torch.cuda.Stream(dev) for _ in range(NS)]
+    x_hs = [torch.empty((T, d), dtype=tdt, pin_memory=True) for _ in range(NS)]
+    for xh in x_hs:
+        xh.copy_(x.cpu())
+    res_hs = [torch.empty(res.shape, dtype=tdt, pin_memory=True) for _ in range(NS)]
+    ws_need = max(256, mglu.host_workspace_bytes(T, d, h, nm, tdt, kind == "ffn"))
+    ws_hosts = [torch.zeros(ws_need, dtype=torch.uint8, device=dev) for _ in range(NS)]
+    x_h, res_h = x_hs[0], res_hs[0]
 
     def e2e_step(i):
-        r = i % R
-        mglu.forward_host(x_h, Ws[r], pks[r], nm, args.act, W_down=Wds[r] if kind == "ffn" else None,
-                          out_host=res_h, workspace=ws_host)
+        r, q = i % R, i % NS
+        mglu.forward_host(x_hs[q], Ws[r], pks[r], nm, args.act, W_down=Wds[r] if kind == "ffn" else None,
+                          out_host=res_hs[q], workspace=ws_hosts[q], stream=e2e_streams[q])
 
     for i in range(args.warmup):
         e2e_step(i)
@@ -494,8 +502,14 @@ def run_mglu(args, dist):
     dist.barrier()
     torch.cuda.synchronize(dev)
     e0.record(stream)
+    for st in e2e_streams:
+        st.wait_event(e0)
     for i in range(K):
         e2e_step(i)
+    for st in e2e_streams:
+        done = torch.cuda.Event()
+        done.record(st)
+        stream.wait_event(done)
     e1.record(stream)
     torch.cuda.synchronize(dev)
     dist.barrier()
@@ -537,7 +551,8 @@ def run_mglu(args, dist):
         "gpu_launches": K * (2 if kind == "ffn" else 1),
         "timing": "device-side: one CUDA-graph replay of the K steps back to back (CUDA events around the "
                   "replay); kernel_us_isolated: a second replay with event nodes around each kernel; "
-                  "e2e: one mglu_forward_host call per step (pinned host x in, kernels, pinned host result out)",
+                  "e2e: one mglu_forward_host call per step (pinned host x in, kernels, pinned host result "
+                  "out), consecutive steps alternating over two streams",
         "clocks": clocks,
         "host_us_per_forward_call": host_us,
         "device_status": status,
