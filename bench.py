@@ -221,9 +221,11 @@ def _num(s):
 
 
 # ---------------------------------------------------------------------- oracle timing
-def time_oracle(w, budget_s=10.0, max_tokens=None):
+def time_oracle(w, budget_s=10.0, max_tokens=None, single_s=3.0):
     """Time the float64 oracle on a bounded sample of the workload: whole
-    tokens (every output column of a token), as many as fit in ~budget_s."""
+    tokens (every output column of a token), as many as fit in ~budget_s on
+    all the oracle's OpenMP threads, then a shorter sample (~single_s) on one
+    thread."""
     import numpy as np
     import oracle
     from masked_glu_b200 import inputs
@@ -246,15 +248,29 @@ def time_oracle(w, budget_s=10.0, max_tokens=None):
     t0 = time.perf_counter()
     one_token()
     t1 = time.perf_counter() - t0
-    n = max(1, min(int(budget_s / max(t1, 1e-6)), max_tokens or T))
+    n = max(1, int(budget_s / max(t1, 1e-6)))
+    if max_tokens:
+        n = min(n, max_tokens)
     t0 = time.perf_counter()
     for _ in range(n):
         one_token()
     dt = time.perf_counter() - t0
-    cores = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
-    return {"value": n / dt, "unit": "tok/s", "cores": cores, "kind": "oracle",
-            "sample": f"{n} token(s) x all {h} output columns of {w['name']} (d={d}, n_m={nm}), "
-                      f"float64, OpenMP over columns"}, one_token
+    cores = oracle.max_threads()
+    res = {"value": n / dt, "unit": "tok/s", "cores": cores, "kind": "oracle",
+           "sample": f"{n} one-token forwards (all {h} output columns each) of {w['name']} "
+                     f"(d={d}, n_m={nm}), float64, OpenMP over columns, {dt:.1f} s wall"}
+    if single_s > 0:
+        oracle.set_threads(1)
+        try:
+            n1 = max(1, min(int(single_s / max(t1 * cores, 1e-6)), n))
+            t0 = time.perf_counter()
+            for _ in range(n1):
+                one_token()
+            res["single_thread_value"] = n1 / (time.perf_counter() - t0)
+            res["single_thread_sample"] = f"{n1} one-token forwards, same columns, 1 thread"
+        finally:
+            oracle.set_threads(cores)
+    return res, one_token
 
 
 def run_reference(args, dist):
@@ -263,7 +279,7 @@ def run_reference(args, dist):
     w["name"], w["act"], w["p"] = args.workload, args.act, args.p
     if dist.rank != 0:
         return
-    _, one = time_oracle(w, budget_s=0.5, max_tokens=1)
+    _, one = time_oracle(w, budget_s=0.5, max_tokens=1, single_s=0)
     for _ in range(args.warmup):
         one()
     t0 = time.perf_counter()
@@ -271,7 +287,8 @@ def run_reference(args, dist):
         one()
     dt = time.perf_counter() - t0
     tok_s = args.steps / dt
-    cores = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
+    import oracle
+    cores = oracle.max_threads()
     line = {
         "impl": "reference", "metric": METRIC, "value": tok_s, "unit": "tok/s", "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000 * dt / args.steps,

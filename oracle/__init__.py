@@ -26,5 +26,4 @@ from .core import (  # noqa: F401
     gate_value,
     pack_masks,
     packed_bytes,
-    unpack_masks,
-)
+    unpack_masks, max_threads, set_threads)

@@ -68,6 +68,10 @@ def _load():
             lib.oracle_down.restype = None
             lib.oracle_down_elems.argtypes = [P, i64, P, i64, P, P, P]
             lib.oracle_down_elems.restype = None
+            lib.oracle_max_threads.argtypes = []
+            lib.oracle_max_threads.restype = i32
+            lib.oracle_set_threads.argtypes = [i32]
+            lib.oracle_set_threads.restype = None
             _lib = lib
     return _lib
 
@@ -178,3 +182,13 @@ def down_elems(hid_rows, Wd, row_idx, c_idx):
     y = np.zeros(row_idx.size)
     _load().oracle_down_elems(_p(hid_rows), h, _p(Wd), row_idx.size, _p(row_idx), _p(c_idx), _p(y))
     return y
+
+
+def max_threads() -> int:
+    """OpenMP threads the oracle's loops use."""
+    return int(_load().oracle_max_threads())
+
+
+def set_threads(n: int) -> None:
+    """Set the oracle's OpenMP thread count (timing only; results do not depend on it)."""
+    _load().oracle_set_threads(int(n))

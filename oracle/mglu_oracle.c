@@ -45,6 +45,9 @@
 #include <stdint.h>
 #include <stdlib.h>
 #include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
 
 #define ORACLE_ACT_SWISH 0
 #define ORACLE_ACT_GELU 1
@@ -231,4 +234,25 @@ void oracle_down_elems(const double *hid, int64_t h, const double *Wd,
             acc += hr[j] * wc[j];
         y[e] = acc;
     }
+}
+
+/* Thread control for timing runs; no effect on any result (every output
+ * element is computed by one thread in the same order). */
+int oracle_max_threads(void)
+{
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}
+
+void oracle_set_threads(int n)
+{
+#ifdef _OPENMP
+    if (n > 0)
+        omp_set_num_threads(n);
+#else
+    (void)n;
+#endif
 }
