@@ -8,6 +8,9 @@ product library never loads it, and it never loads the product library.
   OpenMP over output columns, explicit bit-by-bit mask unpacking).
 * :mod:`oracle.brute` -- pure-Python loops over logical (d x h) tensors, used
   to cross-check the C oracle at tiny sizes.
+* :mod:`oracle.train` -- numpy float64 training path: mask binarisation
+  from logits and the straight-through backward (dx, dW, mask-logit
+  gradients), plus the down-projection backward.
 
 The method: "Masked Gated Linear Unit" (atlas.scime.ai summary page of the
 MGLU paper), "Approach" and "Key results" and the "Measured effects" rows on

@@ -67,3 +67,27 @@ def matmul_logical(a, b):
     """Plain triple loop a [m][n] @ b [n][p]."""
     m, n, p = len(a), len(b), len(b[0])
     return [[sum(a[r][t] * b[t][c] for t in range(n)) for c in range(p)] for r in range(m)]
+
+
+def mglu_logical_soft(x, W, M, act):
+    """The same sum with the mask entries taken as real numbers: the gate of
+    mask i sums x*W*M_i and its value sums x*W*(1 - M_i).  For 0/1 masks it is
+    ``mglu_logical``; with real entries it is the function that the
+    straight-through gradient of a mask entry differentiates."""
+    T, d, h, n_m = len(x), len(W), len(W[0]), len(M)
+    out = []
+    for b in range(T):
+        row = []
+        for j in range(h):
+            total = 0.0
+            for i in range(n_m):
+                gate = 0.0
+                value = 0.0
+                for k in range(d):
+                    p = x[b][k] * W[k][j]
+                    gate += p * M[i][k][j]
+                    value += p * (1.0 - M[i][k][j])
+                total += act_ref(act, gate) * value
+            row.append(total)
+        out.append(row)
+    return out
