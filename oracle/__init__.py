@@ -11,6 +11,7 @@ product library never loads it, and it never loads the product library.
 * :mod:`oracle.train` -- numpy float64 training path: mask binarisation
   from logits and the straight-through backward (dx, dW, mask-logit
   gradients), plus the down-projection backward.
+* :mod:`oracle.routed` -- per-token mask weights and top-k mask routing.
 
 The method: "Masked Gated Linear Unit" (atlas.scime.ai summary page of the
 MGLU paper), "Approach" and "Key results" and the "Measured effects" rows on
