@@ -133,3 +133,40 @@ def down_backward(hid, Wd, dy):
     Wd = np.asarray(Wd, dtype=np.float64)
     dy = np.asarray(dy, dtype=np.float64)
     return dy @ Wd, dy.T @ hid
+
+
+def backward_sampled(x, Ws, masks, a: int, dout, tokens, rows):
+    """The same gradients for a subset, at sizes where the full backward is
+    too slow: dx for the listed tokens (every column j enters), and dW and
+    the mask-logit gradients for the listed rows j of W (every token enters).
+
+    Returns (dx [len(tokens)][d], dWs [len(rows)][d], dM [n_m][len(rows)][d]).
+    Each piece is the chain rule of ``backward`` restricted to what it needs:
+    g_i and v_i of the listed tokens for dx, of the listed rows for dW, dM.
+    """
+    x = np.asarray(x, dtype=np.float64)
+    Ws = np.asarray(Ws, dtype=np.float64)
+    m = np.asarray(masks, dtype=np.float64)
+    dout = np.asarray(dout, dtype=np.float64)
+    tokens = np.asarray(tokens, dtype=np.int64)
+    rows = np.asarray(rows, dtype=np.int64)
+    n_m = m.shape[0]
+
+    xt = x[tokens]
+    g, v = gates_values(xt, Ws, m)
+    dx = np.zeros((tokens.size, x.shape[1]))
+    for i in range(n_m):
+        dg = dout[tokens] * act_grad(a, g[i]) * v[i]
+        dv = dout[tokens] * act(a, g[i])
+        dx += dg @ (m[i] * Ws) + dv @ ((1.0 - m[i]) * Ws)
+
+    Wr, mr = Ws[rows], m[:, rows]
+    g, v = gates_values(x, Wr, mr)
+    dWs = np.zeros((rows.size, x.shape[1]))
+    dM = np.zeros((n_m, rows.size, x.shape[1]))
+    for i in range(n_m):
+        dg = dout[:, rows] * act_grad(a, g[i]) * v[i]
+        dv = dout[:, rows] * act(a, g[i])
+        dWs += mr[i] * (dg.T @ x) + (1.0 - mr[i]) * (dv.T @ x)
+        dM[i] = Wr * ((dg - dv).T @ x)
+    return dx, dWs, dM

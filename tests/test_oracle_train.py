@@ -305,3 +305,16 @@ def test_block_backward_composes():
     dx, _, _ = train.backward(x, Ws, masks, a, dhid)
     g = _fd(lambda t: float(np.sum(dy * oracle.down(_c_forward(t, Ws, masks, a), Wd))), x)
     assert _close(dx, g)
+
+
+def test_sampled_backward_matches_full():
+    """The sampled form gives exactly the full backward's entries (same
+    arithmetic on the restricted operands), including repeated indices."""
+    for n_m, a in ((1, train.ACT_RELU), (4, train.ACT_SWISH), (8, train.ACT_GELU)):
+        x, Ws, masks, dout = _case(30 + n_m, 9, 32, 20, n_m)
+        dx, dWs, dM = train.backward(x, Ws, masks, a, dout)
+        tokens, rows = [0, 4, 8, 4], [19, 0, 7]
+        sx, sW, sM = train.backward_sampled(x, Ws, masks, a, dout, tokens, rows)
+        np.testing.assert_allclose(sx, dx[tokens], rtol=1e-12, atol=1e-12)
+        np.testing.assert_allclose(sW, dWs[rows], rtol=1e-12, atol=1e-12)
+        np.testing.assert_allclose(sM, dM[:, rows], rtol=1e-12, atol=1e-12)
