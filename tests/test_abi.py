@@ -166,3 +166,54 @@ def test_forward_host_rejects_before_any_copy():
     assert args(p, p, need - 1, p) == -1                 # workspace too small
     assert args(p, ctypes.c_void_p((1 << 20) + 16), need, p) == -3   # workspace not 256-byte aligned
     assert L.mglu_forward_host(p, 0, 128, p, 64, p, 4, 0, 0, None, p, need, p, None) == 0   # T == 0: no-op
+
+
+C_CALLER = r"""
+/* A plain C99 caller of the library: no CUDA headers, only mglu.h. */
+#include <stdio.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include "mglu.h"
+
+int main(void)
+{
+    /* malloc gives 16-byte aligned blocks on this platform, as the bf16 path requires */
+    uint16_t *x = malloc(128 * 2), *W = malloc(128 * 4 * 2), *out = malloc(4 * 2);
+    uint8_t *packed = malloc(256);
+    if (!x || !W || !out || !packed || ((uintptr_t)W | (uintptr_t)packed | (uintptr_t)x | (uintptr_t)out) % 16)
+        return 2;
+    /* host-side size queries */
+    printf("packed %zu\n", mglu_packed_bytes(4, 128, 4));
+    printf("scratch_nonzero %d\n", mglu_scratch_bytes(4) > 0);
+    printf("path %d %d\n", mglu_forward_path(1, MGLU_BF16), mglu_forward_path(64, MGLU_BF16));
+    /* rejected before any device work: unsupported n_m, bad act, d % 128 */
+    printf("nm3 %d\n", mglu_forward(x, 1, 128, W, 4, packed, 3, MGLU_ACT_SWISH, MGLU_BF16, out, 0, 0, 0));
+    printf("act9 %d\n", mglu_forward(x, 1, 128, W, 4, packed, 4, 9, MGLU_BF16, out, 0, 0, 0));
+    printf("d64 %d\n", mglu_forward(x, 1, 64, W, 4, packed, 4, MGLU_ACT_GELU, MGLU_BF16, out, 0, 0, 0));
+    printf("zeroT %d\n", mglu_forward(x, 0, 128, W, 4, packed, 4, MGLU_ACT_RELU, MGLU_BF16, out, 0, 0, 0));
+    printf("msg %s\n", mglu_status_string(MGLU_ERR_ALIGN));
+    printf("f32path %d\n", mglu_forward_path(1, MGLU_F32));
+    free(x), free(W), free(out), free(packed);
+    return 0;
+}
+"""
+
+
+def test_header_serves_a_plain_c99_caller(tmp_path):
+    """include/mglu.h compiles as strict C99 and a C program links against
+    libmglu.so and gets the documented host-side answers (no GPU needed)."""
+    mbuild.build()
+    src = tmp_path / "caller.c"
+    src.write_text(C_CALLER)
+    exe = tmp_path / "caller"
+    lib_dir = os.path.dirname(mglu.LIB_PATH)
+    subprocess.run(["gcc", "-std=c99", "-Wall", "-Wextra", "-Werror", "-pedantic", "-I", os.path.join(ROOT, "include"),
+                    str(src), "-o", str(exe), f"-L{lib_dir}", "-l:libmglu.so", f"-Wl,-rpath,{lib_dir}"],
+                   check=True)
+    out = subprocess.run([str(exe)], capture_output=True, text=True, check=True).stdout.split("\n")
+    got = dict(line.split(" ", 1) for line in out if line)
+    assert got["packed"] == str(128 * 4 * 4 // 8)
+    assert got["scratch_nonzero"] == "1"
+    assert got["path"] == "0 1" and got["f32path"] == "2"  # decode for 1 token, prefill for 64; fp32 path
+    assert got["nm3"] == "-2" and got["act9"] == "-1" and got["d64"] == "-3" and got["zeroT"] == "0"
+    assert got["msg"] == "alignment requirement not met"
