@@ -45,7 +45,7 @@ def explore(n_cons, n_stages, flushes, mutation=None):
     # writing: per stage, iteration whose load may be writing it (-1: none)
     # released: per iteration, consumer releases
     # cons: per consumer (i, pc, nflush, arrived_gen) ; pc in W, R, E, F1, F1w, F2, F3, DONE
-    # fin: (f, pc)  pc in A, Aw, B, C, DONE
+    # fin: (f, pc, gen)  pc in A (arrive on FULL), Aw (wait, then read the slots), C (arrive on FREE), DONE
     # full: (gen, count) ; free: (gen, count)
     # slot: per consumer, flush index written (-1 none) ; fin_read: last flush read (-1)
     init = (0, (), (-1,) * n_stages, (-1,) * n_stages, (0,) * N,
