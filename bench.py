@@ -8,7 +8,14 @@ A step is one pass of the hot path over one batch: for the decode and prefill
 workloads one ``mglu_forward`` call (mask-bit unpacking, the n_m + 1 products
 and the fused act-sum epilogue); for the FFN-block workload the up-projection
 plus the down-projection.  Mask packing happens once at weight-load time and
-is outside the timed region.  One JSON line is printed by rank 0.
+is outside the timed region.
+
+The headline workload is the n_m = 8 decode layer (d = 4096, h = 14336, one
+token).  With no --workload given, the run then times the other workloads of
+the suite the same way and adds them to the same JSON line as sub-records
+(``workloads``): the n_m = 4 decode layer, the 4096-token prefill with Swish
+and with GELU, and the FFN block at 1 and 2048 tokens.  One JSON line is
+printed by rank 0.
 
 Inputs are seeded synthetic tensors with the workload's shapes.  To keep every
 timed launch reading HBM, each step uses the next of R device copies of
@@ -20,6 +27,7 @@ from __future__ import annotations
 
 import argparse
 import csv
+import gc
 import hashlib
 import io
 import json
@@ -35,41 +43,69 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 METRIC = "MGLU fwd HBM GB/s & tok/s (decode), TFLOP/s (prefill) vs B200 roofline"
-DEFAULT_WORKLOAD = "decode_d2048_h8192_nm4"
+DEFAULT_WORKLOAD = "decode_d4096_h14336_nm8"
+# the rest of the default run: (workload, tokens, act)
+SUITE = [
+    ("decode_d2048_h8192_nm4", 1, "swish"),
+    ("prefill_T4096_d2048_h8192_nm4", 4096, "swish"),
+    ("prefill_T4096_d2048_h8192_nm4", 4096, "gelu"),
+    ("ffn_d4096_h14336_nm8", 1, "swish"),
+    ("ffn_d4096_h14336_nm8", 2048, "swish"),
+]
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+L2_POLICY = ("inputs larger than L2: each step reads the next of R rotating device copies of the weights "
+             "and packed masks, R x working set > 4 x L2")
 
 
 # ---------------------------------------------------------------------- setup
-def parse_args():
+def parse_args(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["mglu", "reference"], default="mglu")
-    ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    ap.add_argument("--workload", default=None,
+                    help=f"time only this workload (default: {DEFAULT_WORKLOAD} plus the suite)")
     ap.add_argument("--tokens", type=int, default=None, help="token count for the sweep workloads")
     ap.add_argument("--act", default="swish", choices=["swish", "gelu", "relu"])
     ap.add_argument("--p", type=float, default=0.5, help="mask density (FFN-block workload)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-comparisons", action="store_true",
                     help="skip the torch.matmul baselines (dense SwiGLU, naive MGLU) timed after the run")
+    ap.add_argument("--no-suite", action="store_true", help="time the headline workload only")
+    ap.add_argument("--tstar-sweep", action="store_true",
+                    help="also time the FFN block for T in 8..64 with the decode kernel allowed up to 16 tokens "
+                         "and with every T on the tensor-core kernel")
     ap.add_argument("--probe-seconds", type=float, default=1.0,
                     help="untimed run of the same step before timing, to settle and sample clocks")
-    return ap.parse_args()
+    args = ap.parse_args(argv)
+    args.suite = args.workload is None and not args.no_suite
+    if args.workload is None:
+        args.workload = DEFAULT_WORKLOAD
+    return args
 
 
-def workload_shape(args):
+def workload_shape(name, tokens=None, act="swish", p=0.5):
     from masked_glu_b200 import inputs
-    if args.workload not in inputs.WORKLOADS:
-        raise SystemExit(f"unknown workload {args.workload}; choose from {list(inputs.WORKLOADS)}")
-    w = dict(inputs.WORKLOADS[args.workload])
-    if args.tokens is not None:
-        w["T"] = args.tokens
-    w["kind"] = ("ffn" if args.workload.startswith("ffn") else
-                 "prefill" if args.workload.startswith("prefill") else
-                 "tiny" if args.workload.startswith("tiny") else "decode")
-    w["seed"] = inputs.WORKLOAD_SEEDS[args.workload] + (w["T"] if args.tokens is not None else 0)
+    if name not in inputs.WORKLOADS:
+        raise SystemExit(f"unknown workload {name}; choose from {list(inputs.WORKLOADS)}")
+    w = dict(inputs.WORKLOADS[name])
+    if tokens is not None:
+        w["T"] = tokens
+    w["kind"] = ("ffn" if name.startswith("ffn") else
+                 "prefill" if name.startswith("prefill") else
+                 "tiny" if name.startswith("tiny") else "decode")
+    w["seed"] = inputs.WORKLOAD_SEEDS[name] + (w["T"] if tokens is not None else 0)
+    w["name"], w["act"], w["p"] = name, act, p
     return w
+
+
+def config_of(w, world):
+    """The workload's description, identical in the GPU arm and the
+    reference arm."""
+    return {"workload": w["name"], "T": w["T"], "d": w["d"], "h": w["h"], "n_m": w["n_m"], "act": w["act"],
+            "p": w["p"] if w["kind"] == "ffn" else 0.5, "l2": L2_POLICY,
+            "parallelism": "replicas" if world > 1 else "single"}
 
 
 def algorithmic(w):
@@ -274,9 +310,10 @@ def time_oracle(w, budget_s=10.0, max_tokens=None, single_s=3.0):
 
 
 def run_reference(args, dist):
-    """The float64 oracle as it stands, on the host cores (rank 0 only)."""
-    w = workload_shape(args)
-    w["name"], w["act"], w["p"] = args.workload, args.act, args.p
+    """The float64 oracle as it stands, on the host cores (rank 0 only), on
+    the headline workload: each step is one token's forward (every output
+    column), a bounded sample of the workload."""
+    w = workload_shape(args.workload, args.tokens, args.act, args.p)
     if dist.rank != 0:
         return
     _, one = time_oracle(w, budget_s=0.5, max_tokens=1, single_s=0)
@@ -293,46 +330,49 @@ def run_reference(args, dist):
         "impl": "reference", "metric": METRIC, "value": tok_s, "unit": "tok/s", "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000 * dt / args.steps,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": args.workload, "T_per_step": 1, "d": w["d"], "h": w["h"], "n_m": w["n_m"],
-                   "act": args.act},
+        "config": config_of(w, args.gpus),
         "cpu_baseline": {"value": tok_s, "unit": "tok/s", "cores": cores, "kind": "oracle",
-                         "sample": f"one token (all {w['h']} columns) of {args.workload} per step"},
+                         "sample": f"one token (all {w['h']} columns) of {w['name']} per step; the config's l2 "
+                                   f"policy describes the GPU arm"},
         "e2e": {"value": tok_s, "unit": "tok/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
 
 
 # ---------------------------------------------------------------------- GPU run
-def time_comparisons(T, d, h, nm, act, dev, l2, reps=10):
+def time_comparisons(T, d, h, nm, act, dev, l2, reps=50, rounds=3):
     """Library baselines on the same box and shapes, for context only (not the
     product path, not counted in gpu_launches): a dense SwiGLU with two bf16
     d x h projections through torch.matmul (cuBLAS), and a naive PyTorch MGLU
     that materialises every masked weight M_i * W in bf16 before multiplying.
-    Weights rotate over copies larger than L2; times are per call."""
-    import math
-
+    Weights rotate over copies larger than L2; times are per call, the median
+    of `rounds` runs of reps x R calls."""
     import torch
     F = torch.nn.functional
     fn_act = F.gelu if act == "gelu" else F.relu if act == "relu" else F.silu
     x = torch.randn(T, d, device=dev).to(torch.bfloat16)
 
-    def timed(fn, R):
+    def timed(fn, R, n):
         for i in range(2 * R):
             fn(i % R)
         torch.cuda.synchronize(dev)
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record()
-        for i in range(reps * R):
-            fn(i % R)
-        e1.record()
-        e1.synchronize()
-        return e0.elapsed_time(e1) * 1000.0 / (reps * R)
+        res = []
+        for _ in range(rounds):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            for i in range(n * R):
+                fn(i % R)
+            e1.record()
+            e1.synchronize()
+            res.append(e0.elapsed_time(e1) * 1000.0 / (n * R))
+        return statistics.median(res), res
 
     res = {}
     R = max(2, math.ceil(4 * l2 / (2 * h * d * 2)))
     Wg = [(torch.randn(h, d, device=dev) * 0.02).to(torch.bfloat16) for _ in range(R)]
     Wv = [(torch.randn(h, d, device=dev) * 0.02).to(torch.bfloat16) for _ in range(R)]
-    res["dense_swiglu_us"] = timed(lambda i: fn_act(x @ Wg[i].t()) * (x @ Wv[i].t()), R)
+    res["dense_swiglu_us"], res["dense_swiglu_rounds_us"] = timed(
+        lambda i: fn_act(x @ Wg[i].t()) * (x @ Wv[i].t()), R, reps)
     del Wg, Wv
     R = max(2, math.ceil(4 * l2 / (h * d * 2 * (1 + nm))))
     W = [(torch.randn(h, d, device=dev) * 0.02).to(torch.bfloat16) for _ in range(R)]
@@ -346,35 +386,27 @@ def time_comparisons(T, d, h, nm, act, dev, l2, reps=10):
             out = out + fn_act(g) * (D - g)
         return out
 
-    res["naive_torch_mglu_us"] = timed(naive, R)
+    res["naive_torch_mglu_us"], res["naive_torch_mglu_rounds_us"] = timed(naive, R, max(3, reps // 10))
     del W, M
     torch.cuda.empty_cache()
     res["note"] = ("torch.matmul (cuBLAS) baselines on the same shapes: dense SwiGLU = two bf16 d x h "
-                   "projections; naive MGLU materialises each M_i * W in bf16")
+                   "projections; naive MGLU materialises each M_i * W in bf16; median of "
+                   f"{rounds} rounds")
     return res
 
 
-def run_mglu(args, dist):
+def measure(args, dist, w, dev, *, sample_clocks):
+    """Time one workload: K steps replayed as one CUDA graph (device time,
+    max over ranks), per-kernel times from a second replay with event nodes,
+    and the end-to-end rate through the host-buffer entry point."""
     import numpy as np
     import torch
 
-    from masked_glu_b200 import build as mbuild
     from masked_glu_b200 import inputs, mglu
-
-    if args.warmup < 3:
-        raise SystemExit("--warmup must be >= 3")
-    w = workload_shape(args)
-    w["name"], w["act"], w["p"] = args.workload, args.act, args.p
-    torch.cuda.set_device(dist.local)
-    dev = torch.device("cuda", dist.local)
-    dist.init("nccl")
-    mbuild.build()
-    mglu.lib()
-    mglu.set_decode_max_tokens(16)
 
     T, d, h, nm = w["T"], w["d"], w["h"], w["n_m"]
     kind = w["kind"]
-    case = inputs.make_case(T, d, h, nm, seed=w["seed"] + 7919 * dist.rank, p=args.p, dtype=w["dtype"],
+    case = inputs.make_case(T, d, h, nm, seed=w["seed"] + 7919 * dist.rank, p=w["p"], dtype=w["dtype"],
                             with_down=(kind == "ffn"))
     tdt = torch.float32 if w["dtype"] == "f32" else torch.bfloat16
 
@@ -388,6 +420,7 @@ def run_mglu(args, dist):
     pk0 = mglu.pack_masks(torch.from_numpy(case.masks).to(dev))
     Wd0 = up(case.W_down) if kind == "ffn" else None
     del case
+    gc.collect()
     up_bytes, up_flops, down_bytes, down_flops = algorithmic(w)
     working = up_bytes + (down_bytes if kind == "ffn" else 0)
     l2 = torch.cuda.get_device_properties(dev).L2_cache_size
@@ -400,15 +433,14 @@ def run_mglu(args, dist):
     Wds = ([Wd0] + [Wd0.clone() for _ in range(R - 1)]) if kind == "ffn" else None
     out = torch.empty((T, h), dtype=tdt, device=dev)
     y = torch.empty((T, d), dtype=tdt, device=dev) if kind == "ffn" else None
-    ws = (torch.zeros(max(256, mglu.workspace_bytes(T, d, h, nm, tdt)), dtype=torch.uint8, device=dev)
-          if kind == "ffn" else None)
     scratch = torch.zeros(mglu.scratch_bytes(max(d, h)), dtype=torch.uint8, device=dev)
+
     def step(i, ev=None):
         """One step on the current stream; ev = events bracketing its kernels."""
         r = i % R
         if ev is not None:
             ev[0].record()
-        mglu.forward(x, Ws[r], pks[r], nm, args.act, out=out, scratch=scratch)
+        mglu.forward(x, Ws[r], pks[r], nm, w["act"], out=out, scratch=scratch)
         if ev is not None:
             ev[1].record()
         if kind == "ffn":
@@ -421,12 +453,12 @@ def run_mglu(args, dist):
         step(i)
     torch.cuda.synchronize(dev)
     if mglu.last_device_status() != 0:
-        raise SystemExit("device status error during warm-up")
+        raise SystemExit(f"device status error during warm-up of {w['name']}")
 
     # The K timed steps are captured once as a CUDA graph and replayed: the
     # kernels run back to back (each may start its prologue while the
     # previous one drains, as in a decode loop).  A second graph with event
-    # nodes around each kernel gives the up/down split of a block step.
+    # nodes around each kernel gives the per-kernel split of a step.
     K = args.steps
     cap = torch.cuda.Stream(dev)
 
@@ -446,8 +478,9 @@ def run_mglu(args, dist):
     torch.cuda.synchronize(dev)
 
     # an untimed run of the same graph to settle and sample clocks
-    sampler = ClockSampler(dist.local)
-    sampler.start()
+    sampler = ClockSampler(dist.local) if sample_clocks else None
+    if sampler:
+        sampler.start()
     t_end = time.perf_counter() + args.probe_seconds
     while time.perf_counter() < t_end:
         graph.replay()
@@ -462,7 +495,7 @@ def run_mglu(args, dist):
     t1.record()
     torch.cuda.synchronize(dev)
     dist.barrier()
-    clocks = sampler.stop()
+    clocks = sampler.stop() if sampler else None
     status = mglu.last_device_status()
     total_ms = dist.max(t0.elapsed_time(t1), dev)
     ms_per_step = total_ms / K
@@ -480,17 +513,14 @@ def run_mglu(args, dist):
     # one-kernel step the back-to-back period; for the block its isolated time
     up_ms = ms_per_step if kind != "ffn" else dist.max(up_iso_ms, dev)
 
-    # end to end: pinned host x in, result out, every step
+    # End to end through the public host-buffer call: one library call per
+    # step copies that step's x in from pinned host memory, runs the kernels
+    # and copies the result out, in order on its stream.  Consecutive steps
+    # alternate over two streams (each with its own pinned buffers and
+    # workspace), as a serving loop pipelines requests: one step's copies
+    # overlap the other's kernels.
     res = y if kind == "ffn" else out
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     stream = torch.cuda.current_stream(dev)
-
-    # The public host-buffer call: one library call per step copies that
-    # step's x in from pinned host memory, runs the kernels and copies the
-    # result out, in order on its stream.  Consecutive steps alternate over
-    # two streams (each with its own pinned buffers and workspace), as a
-    # serving loop pipelines requests: one step's copies overlap the other's
-    # kernels.
     NS = 2
     e2e_streams = [torch.cuda.Stream(dev) for _ in range(NS)]
     x_hs = [torch.empty((T, d), dtype=tdt, pin_memory=True) for _ in range(NS)]
@@ -499,23 +529,22 @@ def run_mglu(args, dist):
     res_hs = [torch.empty(res.shape, dtype=tdt, pin_memory=True) for _ in range(NS)]
     ws_need = max(256, mglu.host_workspace_bytes(T, d, h, nm, tdt, kind == "ffn"))
     ws_hosts = [torch.zeros(ws_need, dtype=torch.uint8, device=dev) for _ in range(NS)]
-    x_h, res_h = x_hs[0], res_hs[0]
 
     def e2e_step(i):
         r, q = i % R, i % NS
-        mglu.forward_host(x_hs[q], Ws[r], pks[r], nm, args.act, W_down=Wds[r] if kind == "ffn" else None,
+        mglu.forward_host(x_hs[q], Ws[r], pks[r], nm, w["act"], W_down=Wds[r] if kind == "ffn" else None,
                           out_host=res_hs[q], workspace=ws_hosts[q], stream=e2e_streams[q])
 
     for i in range(args.warmup):
         e2e_step(i)
     torch.cuda.synchronize(dev)
-    # host cost of one public call (no device sync inside the loop)
     n_host = 50
     h0 = time.perf_counter()
     for i in range(n_host):
-        mglu.forward(x, Ws[i % R], pks[i % R], nm, args.act, out=out, scratch=scratch)
+        mglu.forward(x, Ws[i % R], pks[i % R], nm, w["act"], out=out, scratch=scratch)
     host_us = (time.perf_counter() - h0) / n_host * 1e6
     torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     dist.barrier()
     torch.cuda.synchronize(dev)
     e0.record(stream)
@@ -532,9 +561,11 @@ def run_mglu(args, dist):
     dist.barrier()
     e2e_ms = dist.max(e0.elapsed_time(e1), dev)
     e2e_value = dist.world * T * K / (e2e_ms / 1000.0)
+    status = status or mglu.last_device_status()
 
     peaks, peak_src = load_peaks()
-    if kind in ("decode", "ffn", "tiny") and T <= 16:
+    decode = T <= 16 and w["dtype"] != "f32"
+    if decode or kind == "tiny":
         achieved = up_bytes / (up_ms / 1000.0) / 1e9
         roof = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                 "frac": achieved / peaks["hbm_gbs"], "peak_source": f"{peak_src} hbm_gbs (copy)"}
@@ -542,51 +573,150 @@ def run_mglu(args, dist):
         achieved = up_flops / (up_ms / 1000.0) / 1e12
         pk = peaks["bf16_tflops"]
         roof = {"bound": "tensor", "achieved": achieved, "peak": pk, "unit": "TFLOP/s",
-                "frac": achieved / pk, "peak_source": f"{peak_src} bf16_tflops (burst, kernel timed alone)"}
-    roof["traffic"] = recorded_traffic(args.workload, T)
-    roof["kernel"] = "mglu up-projection (decode)" if (T <= 16 and w["dtype"] != "f32") else \
-        "mglu up-projection (tcgen05)" if w["dtype"] != "f32" else "mglu fp32"
+                "frac": achieved / pk, "peak_source": f"{peak_src} bf16_tflops (burst, kernel timed alone)",
+                "frac_of_sustained": achieved / peaks.get("bf16_tflops_sustained", pk)}
+    roof["traffic"] = recorded_traffic(w["name"], T)
+    roof["kernel"] = ("mglu up-projection (decode)" if decode else
+                      "mglu up-projection (tcgen05)" if w["dtype"] != "f32" else "mglu fp32")
     roof["kernel_us"] = up_ms * 1000.0
     roof["kernel_us_isolated"] = up_iso_ms * 1000.0
     roof["algorithmic_bytes"] = up_bytes
     roof["algorithmic_flops"] = up_flops
 
-    line = {
-        "metric": METRIC, "value": value, "unit": "tok/s", "n_gpus": dist.world, "steps": K,
-        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": w["dtype"],
-        "data": "synthetic: x ~ N(0,1), W ~ N(0,0.02^2), Bernoulli(p) masks, seeded PCG64",
-        "config": {"workload": args.workload, "T": T, "d": d, "h": h, "n_m": nm, "act": args.act,
-                   "p": args.p if kind == "ffn" else 0.5,
-                   "l2": f"inputs larger than L2: {R} rotating device copies of W and packed masks"
-                         f"{' and W_down' if kind == 'ffn' else ''} ({R * working / 1e6:.0f} MB vs "
-                         f"{l2 / 1e6:.0f} MB L2)",
-                   "parallelism": "replicas" if dist.world > 1 else "single"},
+    rec = {
+        "value": value, "unit": "tok/s", "ms_per_step": ms_per_step, "dtype": w["dtype"],
+        "config": config_of(w, dist.world),
         "roofline": roof,
-        "e2e": {"value": e2e_value, "unit": "tok/s", "h2d_bytes_per_step": x_h.numel() * x_h.element_size(),
-                "d2h_bytes_per_step": res_h.numel() * res_h.element_size()},
+        "e2e": {"value": e2e_value, "unit": "tok/s", "h2d_bytes_per_step": x_hs[0].numel() * x_hs[0].element_size(),
+                "d2h_bytes_per_step": res_hs[0].numel() * res_hs[0].element_size()},
         "gpu_launches": K * (2 if kind == "ffn" else 1),
-        "timing": "device-side: one CUDA-graph replay of the K steps back to back (CUDA events around the "
-                  "replay); kernel_us_isolated: a second replay with event nodes around each kernel; "
-                  "e2e: one mglu_forward_host call per step (pinned host x in, kernels, pinned host result "
-                  "out), consecutive steps alternating over two streams",
-        "clocks": clocks,
         "host_us_per_forward_call": host_us,
         "device_status": status,
+        "rotating_copies": R,
+        "working_set_mb": R * working / 1e6,
     }
+    if clocks is not None:
+        rec["clocks"] = clocks
     if kind == "ffn":
-        line["down_kernel_us"] = down_ms * 1000.0
-        line["down_gbs"] = down_bytes / (down_ms / 1000.0) / 1e9
-    if kind == "prefill" or T > 16:
-        line["tflops"] = up_flops / (up_ms / 1000.0) / 1e12
+        rec["down_kernel_us"] = down_ms * 1000.0
+        rec["down_gbs"] = down_bytes / (down_ms / 1000.0) / 1e9
+        rec["down_tflops"] = down_flops / (down_ms / 1000.0) / 1e12
+    if decode:
+        rec["hbm_gbs"] = up_bytes / (up_ms / 1000.0) / 1e9
     else:
-        line["hbm_gbs"] = up_bytes / (up_ms / 1000.0) / 1e9
+        rec["tflops"] = up_flops / (up_ms / 1000.0) / 1e12
+    extra = {"l2": l2}
+    del Ws, pks, Wds, x, out, y, scratch, ws_hosts
+    gc.collect()
+    torch.cuda.empty_cache()
+    return rec, extra
+
+
+def tstar_sweep(args, dist, dev):
+    """Device time of the FFN block (up + down) at T = 8..64 with the decode
+    kernel allowed up to 16 tokens and with every T on the tensor-core kernel:
+    where the two cross is the dispatch point."""
+    import numpy as np
+    import torch
+
+    from masked_glu_b200 import inputs, mglu
+
+    w = workload_shape("ffn_d4096_h14336_nm8", 64)
+    d, h, nm = w["d"], w["h"], w["n_m"]
+    case = inputs.make_case(64, d, h, nm, seed=w["seed"], with_down=True)
+
+    def up(t):
+        return torch.from_numpy(t.storage.view(np.int16)).view(torch.bfloat16).to(dev)
+
+    x64, W0, Wd0 = up(case.x), up(case.W), up(case.W_down)
+    pk0 = mglu.pack_masks(torch.from_numpy(case.masks).to(dev))
+    del case
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    R = max(2, math.ceil(4 * l2 / (W0.numel() * 4 + pk0.numel())))
+    Ws = [W0] + [W0.clone() for _ in range(R - 1)]
+    pks = [pk0] + [pk0.clone() for _ in range(R - 1)]
+    Wds = [Wd0] + [Wd0.clone() for _ in range(R - 1)]
+    scratch = torch.zeros(mglu.scratch_bytes(max(d, h)), dtype=torch.uint8, device=dev)
+    rows = []
+    prev = mglu.set_decode_max_tokens(16)
+    try:
+        for T in (8, 12, 16, 24, 32, 48, 64):
+            x = x64[:T].contiguous()
+            hid = torch.empty((T, h), dtype=torch.bfloat16, device=dev)
+            yy = torch.empty((T, d), dtype=torch.bfloat16, device=dev)
+            row = {"T": T}
+            for limit in (16, 0):
+                if limit == 16 and T > 16:
+                    continue
+                mglu.set_decode_max_tokens(limit)
+
+                def blk(i):
+                    mglu.forward(x, Ws[i % R], pks[i % R], nm, "swish", out=hid, scratch=scratch)
+                    mglu.down_proj(hid, Wds[i % R], out=yy, scratch=scratch)
+
+                for i in range(2 * R):
+                    blk(i)
+                torch.cuda.synchronize(dev)
+                n = 8 * R
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record()
+                for i in range(n):
+                    blk(i)
+                e1.record()
+                e1.synchronize()
+                row["decode_us" if limit == 16 else "tensor_core_us"] = dist.max(e0.elapsed_time(e1) * 1000 / n, dev)
+            rows.append(row)
+    finally:
+        mglu.set_decode_max_tokens(prev)
+    del Ws, pks, Wds, scratch
+    torch.cuda.empty_cache()
+    return {"what": "FFN block d=4096 h=14336 n_m=8, up + down per call, weights rotating over copies > 4x L2, "
+                    "eager back-to-back calls", "rows": rows}
+
+
+def run_mglu(args, dist):
+    import torch
+
+    from masked_glu_b200 import build as mbuild
+    from masked_glu_b200 import mglu
+
+    if args.warmup < 3:
+        raise SystemExit("--warmup must be >= 3")
+    torch.cuda.set_device(dist.local)
+    dev = torch.device("cuda", dist.local)
+    dist.init("nccl")
+    mbuild.build()
+    mglu.lib()
+    mglu.set_decode_max_tokens(16)
+
+    w = workload_shape(args.workload, args.tokens, args.act, args.p)
+    rec, extra = measure(args, dist, w, dev, sample_clocks=True)
+    line = {"metric": METRIC, "value": rec["value"], "unit": "tok/s", "n_gpus": dist.world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": rec["ms_per_step"], "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": w["dtype"],
+            "data": "synthetic: x ~ N(0,1), W ~ N(0,0.02^2), Bernoulli(p) masks, seeded PCG64"}
+    line.update({k: v for k, v in rec.items() if k not in line})
+    line["timing"] = ("device-side: one CUDA-graph replay of the K steps back to back (CUDA events around the "
+                      "replay); kernel_us_isolated: a second replay with event nodes around each kernel; e2e: one "
+                      "mglu_forward_host call per step (pinned host x in, kernels, pinned host result out), "
+                      "consecutive steps alternating over two streams")
 
     if dist.world == 1 and w["dtype"] == "bf16" and not args.no_comparisons:
-        line["comparisons"] = time_comparisons(T, d, h, nm, args.act, dev, l2)
-        line["comparisons"]["mglu_us"] = up_ms * 1000.0 + (down_ms * 1000.0 if kind == "ffn" else 0.0)
-        if kind == "ffn":
+        line["comparisons"] = time_comparisons(w["T"], w["d"], w["h"], w["n_m"], w["act"], dev, extra["l2"])
+        line["comparisons"]["mglu_us"] = rec["roofline"]["kernel_us"] + rec.get("down_kernel_us", 0.0)
+        if w["kind"] == "ffn":
             line["comparisons"]["note"] += "; mglu_us includes the down-projection, the baselines do not"
+
+    if args.suite:
+        subs = []
+        for name, T, act in SUITE:
+            ws = workload_shape(name, T if name.startswith("ffn") else None, act, 0.5)
+            r, _ = measure(args, dist, ws, dev, sample_clocks=True)
+            subs.append(r)
+        line["workloads"] = subs
+        line["gpu_launches_all_workloads"] = line["gpu_launches"] + sum(r["gpu_launches"] for r in subs)
+    if args.tstar_sweep:
+        line["tstar_sweep"] = tstar_sweep(args, dist, dev)
 
     # the CPU oracle on a bounded sample: rank 0, one GPU only
     if dist.world == 1 and dist.rank == 0 and not args.no_cpu_baseline:

@@ -58,7 +58,7 @@ extern "C" {
 typedef enum {
     MGLU_OK = 0,
     MGLU_ERR_INVALID = -1,     /* null pointer, negative size, bad act/dtype, small workspace */
-    MGLU_ERR_UNSUPPORTED = -2, /* n_m not in {1,2,4,8} */
+    MGLU_ERR_UNSUPPORTED = -2, /* n_m not in {1,2,4,8}; T > 16 on the decode-only entry point */
     MGLU_ERR_ALIGN = -3,       /* a pointer or size alignment rule above is broken */
     MGLU_ERR_CUDA = -4,        /* a CUDA runtime call or a kernel launch failed */
     MGLU_ERR_TIMEOUT = -5      /* a device-side bounded wait gave up (see mglu_last_device_status) */
@@ -134,17 +134,21 @@ int mglu_down_proj(const void *hid, int64_t T, int64_t h, const void *W_down,
                    int64_t d, int dtype, void *y, void *scratch,
                    size_t scratch_bytes, void *stream);
 
-/* Workspace bytes mglu_forward_down needs: the hidden activation [T][h] in
- * the path's dtype (rounded up to 256 bytes) followed by the decode scratch
- * for max(d, h) rows.  Zero-fill it before its first use, as for scratch. */
+/* Workspace bytes mglu_forward_down needs: the decode scratch for
+ * max(d, h) rows (mglu_scratch_bytes) at the START of the workspace, then the
+ * hidden activation [T][h] in the path's dtype (rounded up to 256 bytes).
+ * The scratch's place does not depend on T, so one workspace serves calls of
+ * any token count on the same layer shape.  Zero-fill it before its first
+ * use, as for scratch; zero-fill it again before using it for a layer with a
+ * larger max(d, h), whose scratch reaches into bytes that held activations. */
 size_t mglu_workspace_bytes(int64_t T, int64_t d, int64_t h, int n_m, int dtype);
 
 /*
  * The FFN block: y = MGLU(x) W_down^T.  The hidden activation is written to
- * the start of the caller's workspace (dtype of the path; bf16 rounding
+ * the workspace after the decode scratch (dtype of the path; bf16 rounding
  * happens once, as in mglu_forward) and then multiplied by W_down, both on
- * `stream`.  workspace_bytes must be >= mglu_workspace_bytes(...) (else
- * INVALID).
+ * `stream`.  workspace: device, 16-byte aligned, workspace_bytes >=
+ * mglu_workspace_bytes(...) (else INVALID / ALIGN).
  */
 int mglu_forward_down(const void *x, int64_t T, int64_t d, const void *W,
                       int64_t h, const uint8_t *packed, int n_m, int act,
@@ -191,9 +195,10 @@ int mglu_forward_decode_static(const void *x, int64_t T, int64_t d,
                                int n_m, int act, void *out, void *stream);
 
 /*
- * Device workspace mglu_forward_host needs: a staging copy of x, the device
- * result, and the decode scratch (plus the hidden activation when
- * with_down != 0).  0 for bad input.
+ * Device workspace mglu_forward_host needs: the decode scratch for max(d, h)
+ * rows at its start (whether or not W_down is given, so its place never
+ * moves), then a staging copy of x, the device result and, when
+ * with_down != 0, the hidden activation.  0 for bad input.
  */
 size_t mglu_host_workspace_bytes(int64_t T, int64_t d, int64_t h, int n_m,
                                  int dtype, int with_down);

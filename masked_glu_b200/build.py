@@ -10,6 +10,7 @@ machine without a GPU (calls then fail with MGLU_ERR_CUDA).
 from __future__ import annotations
 
 import glob
+import hashlib
 import os
 import subprocess
 import sys
@@ -19,6 +20,7 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libmglu.so")
+STAMP = LIB + ".sha256"  # hash of the sources and flags the library was built from
 
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",
@@ -37,11 +39,30 @@ def _deps():
             + [os.path.join(INCLUDE, "mglu.h")])
 
 
+def source_hash() -> str:
+    """SHA-256 over every source the library depends on, the compiler flags
+    and the nvcc version: the library is rebuilt whenever any of them
+    changes, whatever the files' modification times say."""
+    h = hashlib.sha256()
+    h.update(" ".join(NVCC_FLAGS).encode())
+    h.update(os.environ.get("NVCC", "nvcc").encode())
+    try:
+        ver = subprocess.run([os.environ.get("NVCC", "nvcc"), "--version"], capture_output=True, text=True).stdout
+    except OSError:
+        ver = ""
+    h.update(ver.encode())
+    for p in sorted(_deps()):
+        h.update(os.path.relpath(p, ROOT).encode())
+        with open(p, "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
 def up_to_date() -> bool:
-    if not os.path.exists(LIB):
+    if not (os.path.exists(LIB) and os.path.exists(STAMP)):
         return False
-    t = os.path.getmtime(LIB)
-    return all(os.path.getmtime(p) <= t for p in _deps())
+    with open(STAMP) as f:
+        return f.read().strip() == source_hash()
 
 
 def build(force: bool = False, verbose: bool = False) -> str:
@@ -54,8 +75,12 @@ def build(force: bool = False, verbose: bool = False) -> str:
     if verbose:
         cmd.insert(1, "-Xptxas=-v")
         print(" ".join(cmd), file=sys.stderr)
+    digest = source_hash()
     subprocess.run(cmd, check=True)
     os.replace(tmp, LIB)
+    with open(STAMP + ".tmp", "w") as f:
+        f.write(digest + "\n")
+    os.replace(STAMP + ".tmp", STAMP)
     return LIB
 
 

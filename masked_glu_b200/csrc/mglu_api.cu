@@ -6,6 +6,7 @@
 
 #include <cstdint>
 #include <cstdio>
+#include <atomic>
 #include <cstring>
 #include <mutex>
 
@@ -20,7 +21,7 @@
 namespace {
 
 thread_local char g_last_cuda_error[256] = "";
-int g_decode_max_tokens = 16;
+std::atomic<int> g_decode_max_tokens{16};
 constexpr int kMaxDevices = 64;
 
 int cuda_fail(cudaError_t e, const char *what)
@@ -49,15 +50,18 @@ int current_device(int *dev)
     return MGLU_OK;
 }
 
+// SM count per device, cached; concurrent first calls may both query, and
+// both store the same value.
 int sm_count(int dev)
 {
-    static int cache[kMaxDevices] = {0};
-    if (cache[dev] == 0) {
-        int n = 0;
+    static std::atomic<int> cache[kMaxDevices];
+    int n = cache[dev].load(std::memory_order_relaxed);
+    if (n == 0) {
         cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-        cache[dev] = n > 0 ? n : 148;
+        n = n > 0 ? n : 148;
+        cache[dev].store(n, std::memory_order_relaxed);
     }
-    return cache[dev];
+    return n;
 }
 
 // cuTensorMapEncodeTiled through the runtime's driver entry point, so the
@@ -169,18 +173,24 @@ int make_chunked_map(CUtensorMap *m, CUtensorMapDataType dt, const void *base, u
     return make_map_n(m, dt, base, 3, dims, strides, box, sw);
 }
 
+std::mutex g_attr_mu;
+
 // Raise the kernel's dynamic shared-memory limit once per device (one flag
-// array per kernel instantiation).
+// array per kernel instantiation; host threads making their first call at
+// once serialize on a mutex).
 template <auto Kernel>
 int ensure_smem(int bytes, int dev)
 {
-    static bool done[kMaxDevices] = {false};
-    if (!done[dev]) {
+    static std::atomic<bool> done[kMaxDevices];
+    if (done[dev].load(std::memory_order_acquire))
+        return MGLU_OK;
+    std::lock_guard<std::mutex> lock(g_attr_mu);
+    if (!done[dev].load(std::memory_order_relaxed)) {
         const cudaError_t e =
             cudaFuncSetAttribute(reinterpret_cast<const void *>(Kernel), cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
         if (e != cudaSuccess)
             return cuda_fail(e, "cudaFuncSetAttribute");
-        done[dev] = true;
+        done[dev].store(true, std::memory_order_release);
     }
     return MGLU_OK;
 }
@@ -359,6 +369,10 @@ int run_product(const void *x, int64_t T, int64_t d, const void *W, int64_t rows
 }
 
 size_t scratch_bytes(int64_t rows) { return rows > 0 ? (size_t)mglu::dec::workspace_bytes(rows) : 0; }
+
+size_t round256(size_t n) { return (n + 255) / 256 * 256; }
+
+size_t dtype_bytes(int dtype) { return dtype == MGLU_BF16 ? 2u : 4u; }
 
 // The decode kernel needs its scratch; other paths ignore it.
 int check_scratch(int64_t T, int dtype, int64_t rows, const void *ws, size_t ws_bytes)
@@ -545,29 +559,34 @@ size_t mglu_workspace_bytes(int64_t T, int64_t d, int64_t h, int n_m, int dtype)
     (void)n_m;
     if (T < 0 || d <= 0 || h <= 0 || (dtype != MGLU_BF16 && dtype != MGLU_F32))
         return 0;
-    const size_t hid = ((size_t)T * (size_t)h * (dtype == MGLU_BF16 ? 2u : 4u) + 255) / 256 * 256;
-    return hid + scratch_bytes(d > h ? d : h);
+    return scratch_bytes(d > h ? d : h) + round256((size_t)T * (size_t)h * dtype_bytes(dtype));
 }
 
 int mglu_forward_down(const void *x, int64_t T, int64_t d, const void *W, int64_t h, const uint8_t *packed, int n_m,
                       int act, int dtype, const void *W_down, void *workspace, size_t workspace_bytes, void *y,
                       void *stream)
 {
-    int rc = check_forward(x, T, d, W, h, packed, n_m, act, dtype, workspace);
-    if (rc)
-        return rc;
-    if ((rc = check_down(workspace, T, h, W_down, d, dtype, y)))
-        return rc;
+    if (T < 0 || d <= 0 || h <= 0 || (dtype != MGLU_BF16 && dtype != MGLU_F32))
+        return MGLU_ERR_INVALID;
     if (T > 0 && (!workspace || workspace_bytes < mglu_workspace_bytes(T, d, h, n_m, dtype)))
         return MGLU_ERR_INVALID;
+    // workspace: the decode scratch first (its place does not depend on T),
+    // then the hidden activation
+    uint8_t *scratch = reinterpret_cast<uint8_t *>(workspace);
+    uint8_t *hid = scratch + scratch_bytes(d > h ? d : h);
+    int rc = check_forward(x, T, d, W, h, packed, n_m, act, dtype, T > 0 ? hid : nullptr);
+    if (rc)
+        return rc;
+    if ((rc = check_down(hid, T, h, W_down, d, dtype, y)))
+        return rc;
     if (T == 0)
         return MGLU_OK;
-    const size_t hid = ((size_t)T * (size_t)h * (dtype == MGLU_BF16 ? 2u : 4u) + 255) / 256 * 256;
-    void *scratch = reinterpret_cast<uint8_t *>(workspace) + hid;
+    if (!aligned(workspace, 16))
+        return MGLU_ERR_ALIGN;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    if ((rc = run_product(x, T, d, W, h, packed, n_m, act, dtype, workspace, scratch, s)))
+    if ((rc = run_product(x, T, d, W, h, packed, n_m, act, dtype, hid, scratch, s)))
         return rc;
-    return run_product(workspace, T, h, W_down, d, nullptr, 0, 0, dtype, y, scratch, s);
+    return run_product(hid, T, h, W_down, d, nullptr, 0, 0, dtype, y, scratch, s);
 }
 
 int mglu_forward_decode_static(const void *x, int64_t T, int64_t d, const void *W, int64_t h,
@@ -604,13 +623,14 @@ int mglu_forward_decode_static(const void *x, int64_t T, int64_t d, const void *
 
 size_t mglu_host_workspace_bytes(int64_t T, int64_t d, int64_t h, int n_m, int dtype, int with_down)
 {
+    (void)n_m;
     if (T < 0 || d <= 0 || h <= 0 || (dtype != MGLU_BF16 && dtype != MGLU_F32))
         return 0;
-    const size_t es = dtype == MGLU_BF16 ? 2u : 4u;
-    const size_t xb = ((size_t)T * (size_t)d * es + 255) / 256 * 256;
-    const size_t rb = ((size_t)T * (size_t)(with_down ? d : h) * es + 255) / 256 * 256;
-    const size_t rest = with_down ? mglu_workspace_bytes(T, d, h, n_m, dtype) : scratch_bytes(h);
-    return xb + rb + rest;
+    const size_t es = dtype_bytes(dtype);
+    const size_t xb = round256((size_t)T * (size_t)d * es);
+    const size_t rb = round256((size_t)T * (size_t)(with_down ? d : h) * es);
+    const size_t hb = with_down ? round256((size_t)T * (size_t)h * es) : 0;
+    return scratch_bytes(d > h ? d : h) + xb + rb + hb;
 }
 
 int mglu_forward_host(const void *x_host, int64_t T, int64_t d, const void *W, int64_t h, const uint8_t *packed,
@@ -628,28 +648,28 @@ int mglu_forward_host(const void *x_host, int64_t T, int64_t d, const void *W, i
         return MGLU_ERR_INVALID;
     if (!aligned(workspace, 256))
         return MGLU_ERR_ALIGN;
-    const size_t es = dtype == MGLU_BF16 ? 2u : 4u;
+    const size_t es = dtype_bytes(dtype);
     const size_t xbytes = (size_t)T * (size_t)d * es;
     const size_t rbytes = (size_t)T * (size_t)(with_down ? d : h) * es;
-    uint8_t *base = reinterpret_cast<uint8_t *>(workspace);
-    void *x_dev = base;
-    void *r_dev = base + (xbytes + 255) / 256 * 256;
-    uint8_t *rest = reinterpret_cast<uint8_t *>(r_dev) + (rbytes + 255) / 256 * 256;
-    const size_t rest_bytes = workspace_bytes - (size_t)(rest - base);
+    // workspace: the decode scratch (sized for max(d, h) rows whatever the
+    // call, so its place never moves), the staged x, the result, the hidden
+    uint8_t *scratch = reinterpret_cast<uint8_t *>(workspace);
+    uint8_t *x_dev = scratch + scratch_bytes(d > h ? d : h);
+    uint8_t *r_dev = x_dev + round256(xbytes);
+    uint8_t *hid = r_dev + round256(rbytes);
     // every argument is checked before anything is queued
-    int rc = check_forward(x_dev, T, d, W, h, packed, n_m, act, dtype, with_down ? (const void *)rest : r_dev);
+    int rc = check_forward(x_dev, T, d, W, h, packed, n_m, act, dtype, with_down ? (const void *)hid : r_dev);
     if (rc)
         return rc;
-    if (with_down && (rc = check_down(rest, T, h, W_down, d, dtype, r_dev)))
+    if (with_down && (rc = check_down(hid, T, h, W_down, d, dtype, r_dev)))
         return rc;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     cudaError_t e = cudaMemcpyAsync(x_dev, x_host, xbytes, cudaMemcpyHostToDevice, s);
     if (e != cudaSuccess)
         return cuda_fail(e, "copy x to the device");
-    rc = with_down ? mglu_forward_down(x_dev, T, d, W, h, packed, n_m, act, dtype, W_down, rest, rest_bytes, r_dev,
-                                       stream)
-                   : mglu_forward(x_dev, T, d, W, h, packed, n_m, act, dtype, r_dev, rest, rest_bytes, stream);
-    if (rc)
+    if ((rc = run_product(x_dev, T, d, W, h, packed, n_m, act, dtype, with_down ? hid : r_dev, scratch, s)))
+        return rc;
+    if (with_down && (rc = run_product(hid, T, h, W_down, d, nullptr, 0, 0, dtype, r_dev, scratch, s)))
         return rc;
     if ((e = cudaMemcpyAsync(result_host, r_dev, rbytes, cudaMemcpyDeviceToHost, s)) != cudaSuccess)
         return cuda_fail(e, "copy the result to the host");
@@ -662,9 +682,7 @@ int mglu_set_decode_max_tokens(int t)
 {
     if (t < 0 || t > 16)
         return MGLU_ERR_INVALID;
-    const int prev = g_decode_max_tokens;
-    g_decode_max_tokens = t;
-    return prev;
+    return g_decode_max_tokens.exchange(t);
 }
 
 int mglu_last_device_status(void *stream)
@@ -690,7 +708,7 @@ const char *mglu_status_string(int status)
     switch (status) {
     case MGLU_OK: return "ok";
     case MGLU_ERR_INVALID: return "invalid argument";
-    case MGLU_ERR_UNSUPPORTED: return "unsupported n_m";
+    case MGLU_ERR_UNSUPPORTED: return "unsupported n_m, or too many tokens for the decode-only entry point";
     case MGLU_ERR_ALIGN: return "alignment requirement not met";
     case MGLU_ERR_CUDA: return "CUDA error";
     case MGLU_ERR_TIMEOUT: return "device wait timed out";

@@ -20,7 +20,8 @@ def test_reference_arm_prints_one_contract_line():
     assert d["steps"] == 2 and d["warmup"] == 3
     assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["cores"] >= 1
     assert d["e2e"] == {"value": d["value"], "unit": "tok/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
-    assert d["config"]["workload"] == "decode_d2048_h8192_nm4"
+    assert d["config"]["workload"] == "decode_d4096_h14336_nm8"
+    assert set(d["config"]) >= {"T", "d", "h", "n_m", "act", "p", "l2", "parallelism"}
 
 
 def test_warmup_below_three_is_refused_by_the_gpu_arm():

@@ -282,3 +282,32 @@ def test_forward_host_matches_device_calls(n_m, T, d, h, down):
     torch.cuda.synchronize()
     assert mglu.last_device_status() == 0
     assert torch.equal(got, want.cpu())
+
+
+def test_workspace_reused_across_token_counts_and_block_modes():
+    """One workspace reused by FFN-block calls of different token counts
+    (tensor-core hidden write, then decode), and by host-buffer calls with and
+    without the down-projection: the decode scratch sits at the start of the
+    workspace, so activations written by one call never land on the arrival
+    counters a later call reads.  Every result must equal the same call made
+    on a fresh zero-filled workspace."""
+    d, h, n_m = 256, 1024, 8
+    case = inputs.make_case(512, d, h, n_m, seed=1300, with_down=True)
+    x, W, packed, Wd = device_case(case)
+    ws = torch.zeros(mglu.workspace_bytes(512, d, h, n_m), dtype=torch.uint8, device="cuda")
+    for T in (512, 1, 9, 512, 1):
+        xt = x[:T].contiguous()
+        got = mglu.forward_down(xt, W, packed, n_m, Wd, "swish", workspace=ws)
+        want = mglu.forward_down(xt, W, packed, n_m, Wd, "swish")
+        torch.cuda.synchronize()
+        assert mglu.last_device_status() == 0
+        assert torch.equal(got, want), f"T={T} on a reused workspace differs"
+    hws = torch.zeros(mglu.host_workspace_bytes(512, d, h, n_m, torch.bfloat16, True), dtype=torch.uint8,
+                      device="cuda")
+    for T, down in ((512, True), (1, False), (16, True), (3, False), (1, True)):
+        xh = x[:T].cpu().pin_memory()
+        got = mglu.forward_host(xh, W, packed, n_m, "swish", W_down=Wd if down else None, workspace=hws)
+        want = mglu.forward_host(xh, W, packed, n_m, "swish", W_down=Wd if down else None)
+        torch.cuda.synchronize()
+        assert mglu.last_device_status() == 0
+        assert torch.equal(got, want), f"host call T={T} down={down} on a reused workspace differs"
