@@ -34,11 +34,13 @@
  *        out     [T][h]
  *        W_down  [d][h]            nn.Linear(h, d).weight
  *        y       [T][d]
- *  - bf16 path (dtype MGLU_BF16): x, W, out, W_down, y are bf16; products are
- *    exact and accumulate in fp32; the result is rounded to bf16 once.
+ *  - bf16 path (dtype MGLU_BF16): x, W, out, W_down, y are bf16; every
+ *    product x*W is exact and they accumulate in fp32, at any input scale
+ *    within bf16's range (masks select or negate whole bf16 values, no
+ *    rescaling); the result is rounded to bf16 once.
  *    Requirements (else MGLU_ERR_ALIGN): every pointer 16-byte aligned and
- *    d % 128 == 0 (rows of W and of packed mask bits are then moved in whole
- *    128-element pieces; Llama-style FFN widths satisfy it).
+ *    d % 8 == 0 (a row of W then starts on 16 bytes, and each 8-weight piece
+ *    owns whole bytes of mask bits).  The down-projection needs h % 8 == 0.
  *  - fp32 path (dtype MGLU_F32): x, W, out, W_down, y are float; plain fp32
  *    FMA on CUDA cores (never TF32); any d, h; 4-byte aligned pointers.
  *  - Supported n_m: 1, 2, 4, 8 (else MGLU_ERR_UNSUPPORTED).  T == 0 is a
@@ -86,11 +88,26 @@ size_t mglu_packed_bytes(int n_m, int64_t d, int64_t h);
  *   packed out : mglu_packed_bytes(n_m, d, h) bytes, every byte written
  *                (unused high bits of a partial last byte are 0).
  * Requirements: packed 16-byte aligned.  Any d and h are accepted; the bf16
- * forward additionally needs d % 128 == 0.
+ * forward additionally needs d % 8 == 0.
  * Errors: INVALID, UNSUPPORTED, ALIGN, CUDA.
  */
 int mglu_pack_masks(const uint8_t *masks, int n_m, int64_t d, int64_t h,
                     uint8_t *packed, void *stream);
+
+/*
+ * Pack the masks straight from their training-time logits ("Masked Gated
+ * Linear Unit", "Limitations": the masks are held as FP16 logits while
+ * training, and binary in the forward): M_i[j,k] = 1 where the logit is
+ * greater than zero, else 0.  +0, -0, negative values and NaN give 0;
+ * positive subnormals and +infinity give 1.
+ *   logits in  : [n_m][h][d] IEEE binary16 (uint16 bit patterns), device,
+ *                2-byte aligned (16-byte aligned with (h*d) % 8 == 0 for
+ *                vector loads).
+ *   packed out : as mglu_pack_masks (same format, every byte written).
+ * Errors: INVALID, UNSUPPORTED, ALIGN, CUDA.
+ */
+int mglu_pack_mask_logits(const void *logits, int n_m, int64_t d, int64_t h,
+                          uint8_t *packed, void *stream);
 
 /* Exact inverse of mglu_pack_masks: writes [n_m][h][d] bytes, each 0 or 1. */
 int mglu_unpack_masks(const uint8_t *packed, int n_m, int64_t d, int64_t h,
@@ -109,7 +126,11 @@ int mglu_unpack_masks(const uint8_t *packed, int n_m, int64_t d, int64_t h,
 size_t mglu_scratch_bytes(int64_t rows);
 
 /*
- * MGLU up-projection with the act-and-sum epilogue fused: out = MGLU(x).
+ * MGLU up-projection with the act-and-sum epilogue fused: out = MGLU(x)
+ * ("Masked Gated Linear Unit", "Approach": one shared W, n_m binary masks
+ * splitting it into gate and value parts, the gated products summed; and
+ * "Problem": at decode the layer is bound by reading W, so the masks are
+ * unpacked inside the kernel that reads it).
  * Reads each weight and its mask bits once per pass; for T up to the decode
  * limit (16 by default) one pass serves all tokens; above it a tensor-core
  * (tcgen05) kernel tiles tokens and weights.
@@ -125,10 +146,10 @@ int mglu_forward(const void *x, int64_t T, int64_t d, const void *W, int64_t h,
 
 /*
  * The FFN down-projection alone, a dense product (MGLU replaces only the two
- * GLU projections; "Masked Gated Linear Unit", summary line):
+ * GLU projections; "Masked Gated Linear Unit", "Problem"):
  *   y[b,c] = sum_j hid[b,j] * W_down[c,j]
  *   hid [T][h], W_down [d][h], y [T][d], scratch: mglu_scratch_bytes(d).
- * bf16 requirements: 16-byte aligned pointers, h % 64 == 0.
+ * bf16 requirements: 16-byte aligned pointers, h % 8 == 0.
  */
 int mglu_down_proj(const void *hid, int64_t T, int64_t h, const void *W_down,
                    int64_t d, int dtype, void *y, void *scratch,
@@ -144,7 +165,9 @@ int mglu_down_proj(const void *hid, int64_t T, int64_t h, const void *W_down,
 size_t mglu_workspace_bytes(int64_t T, int64_t d, int64_t h, int n_m, int dtype);
 
 /*
- * The FFN block: y = MGLU(x) W_down^T.  The hidden activation is written to
+ * The FFN block: y = MGLU(x) W_down^T ("Masked Gated Linear Unit", "Problem":
+ * the GLU is the gated half of a transformer FFN, followed by its dense
+ * down-projection).  The hidden activation is written to
  * the workspace after the decode scratch (dtype of the path; bf16 rounding
  * happens once, as in mglu_forward) and then multiplied by W_down, both on
  * `stream`.  workspace: device, 16-byte aligned, workspace_bytes >=
@@ -174,7 +197,7 @@ int mglu_forward_down(const void *x, int64_t T, int64_t d, const void *W,
  * cudaFree or other allocating call on this path.
  *
  *   Arguments and layouts as mglu_forward with dtype MGLU_BF16 (same
- *   alignment and d % 128 rules).  T must be in 0..16 (T == 0 is a no-op),
+ *   alignment and d % 8 rules).  T must be in 0..16 (T == 0 is a no-op),
  *   else MGLU_ERR_UNSUPPORTED.  h must be <= MGLU_STATIC_SCRATCH_MAX_ROWS,
  *   else MGLU_ERR_INVALID, with the limit stated in mglu_last_cuda_error().
  *   The decode kernel runs for every T in 1..16, whatever

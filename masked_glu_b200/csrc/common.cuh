@@ -77,4 +77,54 @@ MGLU_HD uint32_t pair_mask(uint32_t lo, uint32_t hi)
     return prmt_any(v0, v1, sel);
 }
 
+// ---------------------------------------------------------------- mask logits
+// Mask bit of an IEEE binary16 mask logit ("Masked Gated Linear Unit",
+// "Limitations": masks are held as FP16 logits while training): 1 where the
+// logit is greater than zero, i.e. for the bit patterns 0x0001 (the smallest
+// subnormal) through 0x7C00 (+infinity); +0, -0, every negative value and
+// every NaN give 0.
+MGLU_HD uint32_t logit_bit(uint32_t h16) { return ((h16 - 1u) & 0xFFFFu) < 0x7C00u ? 1u : 0u; }
+
+// ---------------------------------------------------------------- sign flips
+// The decode kernel applies mask i to a bf16 pair by flipping signs: it
+// accumulates h_i = x (S_i . W) with S_i = +1 where mask i is set and -1
+// where it is clear, so g_i = (D + h_i) / 2 and v_i = (D - h_i) / 2 with the
+// dense product D = x W.  One LOP3 per pair and mask builds the operand.
+//
+// group_bits<NM, S>: the mask bits of weights 4S .. 4S+3 of an 8-weight
+// chunk (lo/hi as for pair_mask), rearranged so that mask I of weight 4S
+// sits at bit I, of weight 4S+2 at bit 8+I, of weight 4S+1 at bit 16+I and
+// of weight 4S+3 at bit 24+I.  Shifting the result left by 15-I then puts
+// mask I of the pair (4S, 4S+1) at bits 15 and 31 (the pair's sign bits),
+// shifting by 7-I does so for the pair (4S+2, 4S+3).
+template <int NM, int S>
+MGLU_HD uint32_t group_bits(uint32_t lo, uint32_t hi)
+{
+    static_assert(S == 0 || S == 1, "two groups of four weights per chunk");
+    if constexpr (NM == 8) {
+        // one byte per weight: bytes [b0 b1 b2 b3] -> [b0 b2 b1 b3]
+        return prmt_any(S == 0 ? lo : hi, 0u, 0x3120u);
+    } else {
+        uint32_t n = lo;  // one nibble per weight, weight w in nibble w
+        if constexpr (NM == 2) {
+            // 2-bit fields -> nibbles
+            n = (n | (n << 8)) & 0x00FF00FFu;
+            n = (n | (n << 4)) & 0x0F0F0F0Fu;
+            n = (n | (n << 2)) & 0x33333333u;
+        } else if constexpr (NM == 1) {
+            // bits -> nibbles
+            n = (n | (n << 12)) & 0x000F000Fu;
+            n = (n | (n << 6)) & 0x03030303u;
+            n = (n | (n << 3)) & 0x11111111u;
+        }
+        const uint32_t even = n & 0x0F0F0F0Fu;         // weights 0 2 4 6, one per byte
+        const uint32_t odd = (n >> 4) & 0x0F0F0F0Fu;   // weights 1 3 5 7
+        return prmt_any(even, odd, S == 0 ? 0x5410u : 0x7632u);
+    }
+}
+
+// A bf16 pair with the sign of each half flipped where the matching bit of
+// m (bit 15 for the low half, bit 31 for the high half) is clear.
+MGLU_HD uint32_t flip_pair(uint32_t w, uint32_t m) { return w ^ (~m & 0x80008000u); }
+
 }  // namespace mglu

@@ -159,20 +159,6 @@ int make_map(CUtensorMap *m, CUtensorMapDataType dt, const void *base, uint64_t 
     return make_map_n(m, dt, base, 2, dims, strides, box, sw);
 }
 
-// 3-D view of a row-major [outer][inner] matrix as (element of a chunk of
-// `cw` elements, chunk, row): a box {cw, box_chunks, box_rows} lands in shared
-// memory as box_rows consecutive rows of box_chunks chunks.  Strides grow with
-// the dimension, as in a plain 2-D view.  inner % cw == 0.
-int make_chunked_map(CUtensorMap *m, CUtensorMapDataType dt, const void *base, uint64_t inner, uint64_t outer,
-                     uint64_t row_bytes, uint32_t cw, uint32_t esize, uint32_t box_chunks, uint32_t box_rows,
-                     CUtensorMapSwizzle sw)
-{
-    const uint64_t dims[3] = {cw, inner / cw, outer};
-    const uint64_t strides[2] = {(uint64_t)cw * esize, row_bytes};
-    const uint32_t box[3] = {cw, box_chunks, box_rows};
-    return make_map_n(m, dt, base, 3, dims, strides, box, sw);
-}
-
 std::mutex g_attr_mu;
 
 // Raise the kernel's dynamic shared-memory limit once per device (one flag
@@ -229,22 +215,6 @@ int launch_decode(const void *x, int64_t T, int64_t d, const void *W, int64_t ro
     int dev = 0, rc = current_device(&dev);
     if (rc)
         return rc;
-    CUtensorMap tw, tx, tm;
-    if ((rc = make_chunked_map(&tw, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, W, d, rows, d * 2, 64, 2, L::NKC,
-                               mglu::dec::ROWS, CU_TENSOR_MAP_SWIZZLE_128B)))
-        return rc;
-    const int xr = (int)(T < L::XR ? T : L::XR);  // token rows the x box loads
-    if ((rc = make_chunked_map(&tx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, x, d, T, d * 2, 64, 2, L::NKC, (uint32_t)xr,
-                               CU_TENSOR_MAP_SWIZZLE_128B)))
-        return rc;
-    if (NM > 0) {
-        if ((rc = make_chunked_map(&tm, CU_TENSOR_MAP_DATA_TYPE_UINT8, packed, d * NM / 8, rows, d * NM / 8,
-                                   L::M_BOX > 0 ? L::M_BOX : 16, 1, L::M_CHUNKS, mglu::dec::ROWS,
-                                   mglu::dec::mask_swizzle_mode<L::M_BOX>())))
-            return rc;
-    } else {
-        tm = tw;  // not read
-    }
     if ((rc = ensure_smem<mglu::dec::decode_kernel<NM, NT>>(L::SMEM, dev)))
         return rc;
     const int64_t rb = (rows + mglu::dec::ROWS - 1) / mglu::dec::ROWS;
@@ -257,8 +227,9 @@ int launch_decode(const void *x, int64_t T, int64_t d, const void *W, int64_t ro
     float *ws_part = reinterpret_cast<float *>(ws);
     int *ws_count = reinterpret_cast<int *>(reinterpret_cast<uint8_t *>(ws) + mglu::dec::part_bytes());
     return launch_pdl(mglu::dec::decode_kernel<NM, NT>, dim3((unsigned)grid), dim3(L::NTHREADS), L::SMEM, s,
-                      "decode launch", tw, tx, tm, (int)T, xr, (int)rows, (int)d, act, ws_part, ws_count,
-                      reinterpret_cast<__nv_bfloat16 *>(out));
+                      "decode launch", reinterpret_cast<const __nv_bfloat16 *>(x),
+                      reinterpret_cast<const __nv_bfloat16 *>(W), packed, (int)T, (int)rows, (int)d, act, ws_part,
+                      ws_count, reinterpret_cast<__nv_bfloat16 *>(out));
 }
 
 template <int NM>
@@ -285,7 +256,10 @@ int launch_prefill(const void *x, int64_t T, int64_t d, const void *W, int64_t r
     if ((rc = make_map(&tw, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, W, d, rows, d * 2, mglu::pf::BK, C::NJ,
                        CU_TENSOR_MAP_SWIZZLE_128B)))
         return rc;
-    if (NM > 0) {
+    // a tensor map needs 16-byte row strides; other packed rows are read by
+    // the builder warps directly
+    const int mask_direct = NM > 0 && (d * NM / 8) % 16 != 0;
+    if (NM > 0 && !mask_direct) {
         if ((rc = make_map(&tm, CU_TENSOR_MAP_DATA_TYPE_UINT8, packed, d * NM / 8, rows, d * NM / 8, C::MB, C::NJ,
                            CU_TENSOR_MAP_SWIZZLE_NONE)))
             return rc;
@@ -300,7 +274,7 @@ int launch_prefill(const void *x, int64_t T, int64_t d, const void *W, int64_t r
     (void)kernel;
     return launch_pdl(mglu::pf::prefill_kernel<NM>, dim3((unsigned)grid), dim3(mglu::pf::Cfg<NM>::NTHREADS), C::SMEM, s,
                       "prefill launch", tx, tw, tm, (int)T, (int)rows, (int)d, act,
-                      reinterpret_cast<__nv_bfloat16 *>(out));
+                      reinterpret_cast<__nv_bfloat16 *>(out), packed, mask_direct);
 }
 
 // ------------------------------------------------------------------ fp32
@@ -409,8 +383,8 @@ int check_forward(const void *x, int64_t T, int64_t d, const void *W, int64_t h,
     if (dtype == MGLU_BF16) {
         if (!aligned(W, 16) || !aligned(packed, 16) || (T > 0 && (!aligned(x, 16) || !aligned(out, 16))))
             return MGLU_ERR_ALIGN;
-        if (d % 128 != 0)
-            return MGLU_ERR_ALIGN;
+        if (d % 8 != 0)
+            return MGLU_ERR_ALIGN;  // rows of W start on 16 bytes and a lane's 8 weights share their mask bytes
     } else {
         if (!aligned(W, 4) || (T > 0 && (!aligned(x, 4) || !aligned(out, 4))))
             return MGLU_ERR_ALIGN;
@@ -429,8 +403,8 @@ int check_down(const void *hid, int64_t T, int64_t h, const void *Wd, int64_t d,
     if (dtype == MGLU_BF16) {
         if (!aligned(Wd, 16) || (T > 0 && (!aligned(hid, 16) || !aligned(y, 16))))
             return MGLU_ERR_ALIGN;
-        if (h % 64 != 0)
-            return MGLU_ERR_ALIGN;
+        if (h % 8 != 0)
+            return MGLU_ERR_ALIGN;  // rows of W_down start on 16 bytes
     } else {
         if (!aligned(Wd, 4) || (T > 0 && (!aligned(hid, 4) || !aligned(y, 4))))
             return MGLU_ERR_ALIGN;
@@ -453,6 +427,20 @@ int pack_dispatch(const uint8_t *in, int64_t d, int64_t h, uint8_t *outp, bool u
     else
         mglu::pack_kernel<NM><<<(unsigned)blocks, 256, 0, s>>>(in, hd, nbytes, outp, vec);
     return check_launch(unpack ? "unpack launch" : "pack launch");
+}
+
+template <int NM>
+int pack_logits_dispatch(const uint16_t *in, int64_t d, int64_t h, uint8_t *outp, cudaStream_t s)
+{
+    const int64_t hd = h * d;
+    const int64_t nbytes = (hd * NM + 7) / 8;
+    const int64_t chunks = (nbytes + 15) / 16;
+    const int vec = (hd % 8 == 0) && aligned(in, 16);
+    const int64_t blocks = (chunks + 255) / 256;
+    if (blocks > 0x7FFFFFFF)
+        return MGLU_ERR_INVALID;
+    mglu::pack_logits_kernel<NM><<<(unsigned)blocks, 256, 0, s>>>(in, hd, nbytes, outp, vec);
+    return check_launch("pack logits launch");
 }
 
 int pack_common(const uint8_t *in, int n_m, int64_t d, int64_t h, uint8_t *outp, bool unpack, void *stream)
@@ -523,6 +511,26 @@ size_t mglu_packed_bytes(int n_m, int64_t d, int64_t h)
 int mglu_pack_masks(const uint8_t *masks, int n_m, int64_t d, int64_t h, uint8_t *packed, void *stream)
 {
     return pack_common(masks, n_m, d, h, packed, false, stream);
+}
+
+int mglu_pack_mask_logits(const void *logits, int n_m, int64_t d, int64_t h, uint8_t *packed, void *stream)
+{
+    if (d <= 0 || h <= 0 || !logits || !packed)
+        return MGLU_ERR_INVALID;
+    if (!nm_supported(n_m))
+        return MGLU_ERR_UNSUPPORTED;
+    if (!aligned(packed, 16) || !aligned(logits, 2))
+        return MGLU_ERR_ALIGN;
+    if (h > ((int64_t)1 << 62) / d)
+        return MGLU_ERR_INVALID;
+    const uint16_t *in = reinterpret_cast<const uint16_t *>(logits);
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    switch (n_m) {
+    case 1: return pack_logits_dispatch<1>(in, d, h, packed, s);
+    case 2: return pack_logits_dispatch<2>(in, d, h, packed, s);
+    case 4: return pack_logits_dispatch<4>(in, d, h, packed, s);
+    default: return pack_logits_dispatch<8>(in, d, h, packed, s);
+    }
 }
 
 int mglu_unpack_masks(const uint8_t *packed, int n_m, int64_t d, int64_t h, uint8_t *masks, void *stream)
@@ -702,6 +710,17 @@ int mglu_last_device_status(void *stream)
 }
 
 const char *mglu_last_cuda_error(void) { return g_last_cuda_error; }
+
+#ifdef MGLU_TEST_HOOKS
+// Test-hook build only (not part of the product ABI): nonzero stops the
+// tensor-core kernel's producer after its first stage on the current device.
+int mglu_test_set_stall(int on)
+{
+    const int v = on ? 1 : 0;
+    const cudaError_t e = cudaMemcpyToSymbol(mglu::g_test_stall_producer, &v, sizeof(int));
+    return e == cudaSuccess ? MGLU_OK : cuda_fail(e, "set test stall");
+}
+#endif
 
 const char *mglu_status_string(int status)
 {

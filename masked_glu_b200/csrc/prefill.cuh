@@ -98,12 +98,36 @@ __device__ __forceinline__ void build_variants(uint8_t *B, int off, uint4 w, uin
     }
 }
 
+// Mask bits of an 8-weight chunk read straight from global memory (NM bytes
+// at byte offset (row * d + k) * NM / 8; zero outside the matrix).
+template <int NM>
+__device__ __forceinline__ uint2 load_mask_global(const uint8_t *packed, int row, int k, int rows, int d)
+{
+    if (row >= rows || k >= d)
+        return make_uint2(0u, 0u);
+    const uint8_t *p = packed + ((int64_t)row * d + k) * NM / 8;
+    if constexpr (NM == 8)
+        return __ldg(reinterpret_cast<const uint2 *>(p));
+    else if constexpr (NM == 4)
+        return make_uint2(__ldg(reinterpret_cast<const unsigned int *>(p)), 0u);
+    else if constexpr (NM == 2)
+        return make_uint2(__ldg(reinterpret_cast<const unsigned short *>(p)), 0u);
+    else
+        return make_uint2(__ldg(p), 0u);
+}
+
+// mask_direct != 0: the packed rows are not 16-byte strided (d * NM / 8 is
+// not a multiple of 16), so no tensor map can describe them; the builders
+// then read each chunk's mask bits from global memory (issued before they
+// wait for the W tile, so the two latencies overlap) instead of a staged
+// mask tile.
 template <int NM>
 __global__ void __launch_bounds__(Cfg<NM>::NTHREADS, 1) prefill_kernel(const __grid_constant__ CUtensorMap tm_x,
                                                               const __grid_constant__ CUtensorMap tm_w,
                                                               const __grid_constant__ CUtensorMap tm_m, int T,
                                                               int rows, int d, int act,
-                                                              __nv_bfloat16 *__restrict__ out)
+                                                              __nv_bfloat16 *__restrict__ out,
+                                                              const uint8_t *__restrict__ packed, int mask_direct)
 {
     using C = Cfg<NM>;
     extern __shared__ uint8_t smem_raw[];
@@ -116,7 +140,8 @@ __global__ void __launch_bounds__(Cfg<NM>::NTHREADS, 1) prefill_kernel(const __g
     uint64_t *empty = built + C::STAGES;
     uint64_t *acc_full = empty + C::STAGES;
     uint64_t *acc_empty = acc_full + 2;
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(acc_empty + 2);
+    uint64_t *drain = acc_empty + 2;  // the MMA issuer's last commit: every MMA has completed
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(drain + 1);
 
     pdl_launch_dependents();
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -137,6 +162,7 @@ __global__ void __launch_bounds__(Cfg<NM>::NTHREADS, 1) prefill_kernel(const __g
             mbar_init(&acc_full[b], 1);
             mbar_init(&acc_empty[b], 4);
         }
+        mbar_init(drain, 1);
         fence_mbar_init();
     }
     if (warp == 1) {
@@ -162,6 +188,12 @@ __global__ void __launch_bounds__(Cfg<NM>::NTHREADS, 1) prefill_kernel(const __g
                 const int m0 = (tile % num_m) * BM;
                 const int n0 = (tile / num_m) * C::NJ;
                 for (int kb = 0; kb < nkb; ++kb, ++it) {
+#ifdef MGLU_TEST_HOOKS
+                    if (it >= 1 && *(volatile int *)&g_test_stall_producer) {
+                        ok = false;  // stop issuing: the consumers' waits run out
+                        break;
+                    }
+#endif
                     const int s = it % C::STAGES;
                     const uint32_t ph = (uint32_t)(it / C::STAGES) & 1u;
                     if (!mbar_wait(&empty[s], ph ^ 1u)) {
@@ -169,18 +201,30 @@ __global__ void __launch_bounds__(Cfg<NM>::NTHREADS, 1) prefill_kernel(const __g
                         break;
                     }
                     uint8_t *st = smem + s * C::STAGE;
-                    // each load completes on a barrier of its own (loads sharing a
-                    // barrier gave occasional wrong operands on B200)
+                    // each load completes on a barrier of its own
                     mbar_arrive_expect_tx(&xfull[s], C::A_BYTES);
                     tma_load_2d(st, &tm_x, &xfull[s], kb * BK, m0);
                     mbar_arrive_expect_tx(&full[s], C::W_TX);
                     tma_load_2d(st + C::A_BYTES, &tm_w, &full[s], kb * BK, n0);
                     if constexpr (NM > 0) {
-                        const int mc = (kb * BK * NM / 8) / C::MB * C::MB;  // 16-byte aligned column
-                        mbar_arrive_expect_tx(&mfull[s], C::M_BYTES);
-                        tma_load_2d(st + C::A_BYTES + C::B_BYTES, &tm_m, &mfull[s], mc, n0);
+                        if (!mask_direct) {
+                            const int mc = (kb * BK * NM / 8) / C::MB * C::MB;  // 16-byte aligned column
+                            mbar_arrive_expect_tx(&mfull[s], C::M_BYTES);
+                            tma_load_2d(st + C::A_BYTES + C::B_BYTES, &tm_m, &mfull[s], mc, n0);
+                        }
                     }
                 }
+            }
+            // Before the CTA may exit, every load issued must have landed: the
+            // last STAGES iterations' barriers have completed their phase (at
+            // once when the consumers took them; after a timeout, bounded).
+            for (int j = it - C::STAGES < 0 ? 0 : it - C::STAGES; j < it; ++j) {
+                const int s = j % C::STAGES;
+                const uint32_t ph = (uint32_t)(j / C::STAGES) & 1u;
+                mbar_wait(&xfull[s], ph);
+                mbar_wait(&full[s], ph);
+                if (NM > 0 && !mask_direct)
+                    mbar_wait(&mfull[s], ph);
             }
         }
     } else if (warp == 1) {
@@ -215,18 +259,34 @@ __global__ void __launch_bounds__(Cfg<NM>::NTHREADS, 1) prefill_kernel(const __g
                 if (ok)
                     umma_commit(&acc_full[b]);
             }
+            // every MMA issued has completed before TMEM is released
+            umma_commit(drain);
+            mbar_wait(drain, 0);
         }
     } else if (warp < 2 + C::NBW) {
         // ---------------------------------------------------------- builders
         if constexpr (NM > 0) {
             const int bt = threadIdx.x - 64;  // 0 .. 32 * NBW - 1
+            constexpr int ITEMS = C::NJ * 8;   // 16-byte pieces of a W tile
+            constexpr int MAXI = (ITEMS + 32 * C::NBW - 1) / (32 * C::NBW);
             int it = 0;
             bool ok = true;
             for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+                const int n0 = (tile / num_m) * C::NJ;
                 for (int kb = 0; kb < nkb; ++kb, ++it) {
                     const int s = it % C::STAGES;
                     const uint32_t ph = (uint32_t)(it / C::STAGES) & 1u;
-                    if (!mbar_wait_warp3(&full[s], &mfull[s], nullptr, ph)) {
+                    uint2 mg[MAXI];
+                    if (mask_direct) {
+#pragma unroll
+                        for (int q = 0; q < MAXI; ++q) {
+                            const int item = bt + q * 32 * C::NBW;
+                            mg[q] = item < ITEMS ? load_mask_global<NM>(packed, n0 + (item >> 3), kb * BK + 8 * (item & 7),
+                                                                        rows, d)
+                                                 : make_uint2(0u, 0u);
+                        }
+                    }
+                    if (!mbar_wait_warp3(&full[s], mask_direct ? nullptr : &mfull[s], nullptr, ph)) {
                         ok = false;
                         break;
                     }
@@ -234,13 +294,22 @@ __global__ void __launch_bounds__(Cfg<NM>::NTHREADS, 1) prefill_kernel(const __g
                     uint8_t *B = smem + s * C::STAGE + C::A_BYTES;
                     const uint8_t *Mt = B + C::B_BYTES;
                     const int moff = (kb * BK * NM / 8) % C::MB;  // nonzero only when NM = 1
-                    for (int item = bt; item < C::NJ * 8; item += 32 * C::NBW) {
-                        const int r = item >> 3, c = item & 7;
-                        const int off = r * 128 + ((c ^ (r & 7)) << 4);
-                        const uint4 w = *reinterpret_cast<const uint4 *>(B + off);
-                        uint32_t lo, hi;
-                        load_mask_bytes<NM>(Mt + r * C::MB + moff + c * NM, lo, hi);
-                        build_variants<NM, 0>(B, off, w, lo, hi);
+#pragma unroll
+                    for (int q = 0; q < MAXI; ++q) {
+                        const int item = bt + q * 32 * C::NBW;
+                        if (item < ITEMS) {
+                            const int r = item >> 3, c = item & 7;
+                            const int off = r * 128 + ((c ^ (r & 7)) << 4);
+                            const uint4 w = *reinterpret_cast<const uint4 *>(B + off);
+                            uint32_t lo, hi;
+                            if (mask_direct) {
+                                lo = mg[q].x;
+                                hi = mg[q].y;
+                            } else {
+                                load_mask_bytes<NM>(Mt + r * C::MB + moff + c * NM, lo, hi);
+                            }
+                            build_variants<NM, 0>(B, off, w, lo, hi);
+                        }
                     }
                     fence_proxy_async_smem();  // generic-proxy writes -> visible to the tensor core
                     __syncwarp();

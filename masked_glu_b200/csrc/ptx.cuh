@@ -65,9 +65,17 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity)
 }
 
 // Wait for the phase with the given parity to complete, for at most about
-// one second of wall time.  Returns false (and records MGLU_ERR_TIMEOUT) if
-// the wait gave up.  Every wait in this library goes through here.
+// one second of wall time (20 ms in the test-hook build, whose tests make a
+// wait run out on purpose).  Returns false (and records MGLU_ERR_TIMEOUT) if
+// the wait gave up.  Every mbarrier wait in this library goes through here.
+#ifdef MGLU_TEST_HOOKS
+constexpr uint64_t kWaitLimitNs = 20000000ull;
+// Test hook: when nonzero, the tensor-core kernel's producer issues the
+// loads of its first stage only, so every later wait of the CTA runs out.
+__device__ int g_test_stall_producer;
+#else
 constexpr uint64_t kWaitLimitNs = 1000000000ull;
+#endif
 
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity)
 {
@@ -112,10 +120,6 @@ __device__ __forceinline__ bool mbar_wait_warp3(uint64_t *a, uint64_t *b, uint64
     __syncwarp();
     return ok != 0;
 }
-
-// Make the calling thread hold `v` in a register here: every instruction that
-// produced it has completed (used to wait for outstanding loads).
-__device__ __forceinline__ void consume(uint32_t v) { asm volatile("" ::"r"(v) : "memory"); }
 
 // ---------------------------------------------------------------- dependent launch
 // Kernels are launched with programmatic stream serialization: the next

@@ -93,6 +93,15 @@ struct Sched {
         return 2 * c + ((uint32_t)(rb - rb_sk0) * (uint32_t)nst <= sk_begin(c) ? 0 : 1);
     }
     MGLU_HD bool contributes(int c) const { return sk_begin(c + 1) > sk_begin(c); }
+    // number of units i at which flush_at(i, .) holds: the row blocks the
+    // stream-K share touches plus the whole row blocks
+    MGLU_HD int flushes() const
+    {
+        int f = q;
+        if (n_sk > 0)
+            f += (int)((sk_b + (uint32_t)n_sk - 1u) / (uint32_t)nst - sk_b / (uint32_t)nst) + 1;
+        return f;
+    }
 };
 
 }  // namespace dec

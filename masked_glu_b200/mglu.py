@@ -54,6 +54,7 @@ def lib() -> ctypes.CDLL:
             "mglu_packed_bytes": (SZ, [I32, I64, I64]),
             "mglu_pack_masks": (I32, [P, I32, I64, I64, P, P]),
             "mglu_unpack_masks": (I32, [P, I32, I64, I64, P, P]),
+            "mglu_pack_mask_logits": (I32, [P, I32, I64, I64, P, P]),
             "mglu_scratch_bytes": (SZ, [I64]),
             "mglu_forward": (I32, [P, I64, I64, P, I64, P, I32, I32, I32, P, P, SZ, P]),
             "mglu_down_proj": (I32, [P, I64, I64, P, I64, I32, P, P, SZ, P]),
@@ -128,6 +129,17 @@ def pack_masks(masks: torch.Tensor, stream=None) -> torch.Tensor:
     n_m, h, d = masks.shape
     out = torch.empty(packed_bytes(n_m, d, h), dtype=torch.uint8, device=masks.device)
     _check(lib().mglu_pack_masks(_ptr(masks), n_m, d, h, _ptr(out), _stream(stream)), "mglu_pack_masks")
+    return out
+
+
+def pack_mask_logits(logits: torch.Tensor, stream=None) -> torch.Tensor:
+    """logits [n_m][h][d] float16 on the GPU -> packed stream of the masks
+    logit > 0."""
+    if logits.dtype != torch.float16:
+        raise ValueError("mask logits must be float16")
+    n_m, h, d = logits.shape
+    out = torch.empty(packed_bytes(n_m, d, h), dtype=torch.uint8, device=logits.device)
+    _check(lib().mglu_pack_mask_logits(_ptr(logits), n_m, d, h, _ptr(out), _stream(stream)), "mglu_pack_mask_logits")
     return out
 
 

@@ -3,7 +3,8 @@
 // exactly one CTA; a row block is either finished inside one CTA or is a
 // stream-K row block whose contributors (counted by Sched::contributors) are
 // exactly the CTAs that flush a part of it; their scratch slots are distinct
-// and each CTA uses each of its two slots for at most one row block.
+// and each CTA uses each of its two slots for at most one row block; and
+// Sched::flushes() counts a CTA's flushes exactly.
 // Prints "ok" and exits 0 on success.
 #include <cstdio>
 #include <map>
@@ -27,9 +28,10 @@ static int check(int rows, int d, int ks_width, int G)
     for (int c = 0; c < G; ++c) {
         Sched sc;
         sc.init(rows, d, ks_width, G, c);
-        int rb, ks, cur_rb = -1, seg_start = 0;
+        int rb, ks, cur_rb = -1, seg_start = 0, nflush = 0;
         sc.start(rb, ks);
         for (int i = 0; i < sc.n; sc.next(i, rb, ks), ++i) {
+            nflush += sc.flush_at(i, ks) ? 1 : 0;
             if (rb < 0 || rb >= RB || ks < 0 || ks >= nst) {
                 std::printf("unit out of range rows=%d d=%d G=%d c=%d rb=%d ks=%d\n", rows, d, G, c, rb, ks);
                 return 1;
@@ -74,6 +76,11 @@ static int check(int rows, int d, int ks_width, int G)
             }
             cur_rb = -1;  // the next unit starts a new segment
         }
+        if (nflush != sc.flushes()) {
+            std::printf("CTA %d flushes %d times, flushes() says %d (rows=%d d=%d ks=%d G=%d)\n", c, nflush,
+                        sc.flushes(), rows, d, ks_width, G);
+            return 1;
+        }
     }
     for (size_t u = 0; u < seen.size(); ++u)
         if (seen[u] != 1) {
@@ -108,7 +115,7 @@ static int check(int rows, int d, int ks_width, int G)
 int main()
 {
     const int rows_list[] = {1, 16, 40, 200, 1024, 4096, 8192, 14336, 2000};
-    const int d_list[] = {128, 640, 2048, 4096, 14336};
+    const int d_list[] = {8, 128, 200, 640, 2048, 4096, 14336};
     const int ks_list[] = {256, 384, 512, 768, 1024};
     const int g_list[] = {1, 7, 64, 148, 296, 320};
     for (int rows : rows_list)

@@ -85,11 +85,9 @@ def test_forward_rejects_bad_arguments(L):
     assert fwd(L, W=A + 2) == mglu.ERR_ALIGN
     assert fwd(L, pk=A + 4) == mglu.ERR_ALIGN
     assert fwd(L, out=A + 8) == mglu.ERR_ALIGN
-    assert fwd(L, d=100) == mglu.ERR_ALIGN             # d % 128
-    assert fwd(L, d=192) == mglu.ERR_ALIGN
-    assert fwd(L, d=200, n_m=8) == mglu.ERR_ALIGN      # d * n_m % 128
-    assert fwd(L, d=64, n_m=1) == mglu.ERR_ALIGN
-    assert fwd(L, d=80, n_m=4) == mglu.ERR_ALIGN
+    assert fwd(L, d=100) == mglu.ERR_ALIGN             # d % 8
+    assert fwd(L, d=4) == mglu.ERR_ALIGN
+    assert fwd(L, d=1026, n_m=1) == mglu.ERR_ALIGN
     # fp32 path: 4-byte alignment only
     assert fwd(L, dtype=1, x=A + 2) == mglu.ERR_ALIGN
     # decode scratch: required (and sized for h) on the decode path only
@@ -108,8 +106,8 @@ def test_forward_zero_tokens_is_a_noop(L):
 
 def test_down_and_block_reject_bad_arguments(L):
     big = 1 << 30
-    assert L.mglu_down_proj(A, 1, 100, A, 64, 0, A, A, big, None) == mglu.ERR_ALIGN  # h % 64
-    assert L.mglu_down_proj(A, 1, 96, A, 64, 0, A, A, big, None) == mglu.ERR_ALIGN
+    assert L.mglu_down_proj(A, 1, 100, A, 64, 0, A, A, big, None) == mglu.ERR_ALIGN  # h % 8
+    assert L.mglu_down_proj(A, 1, 12, A, 64, 0, A, A, big, None) == mglu.ERR_ALIGN
     assert L.mglu_down_proj(None, 1, 128, A, 64, 0, A, A, big, None) == mglu.ERR_INVALID
     assert L.mglu_down_proj(A, 1, 128, A, 64, 5, A, A, big, None) == mglu.ERR_INVALID
     assert L.mglu_down_proj(A, 1, 128, A, 64, 0, A, None, 0, None) == mglu.ERR_INVALID  # decode needs scratch
@@ -138,6 +136,33 @@ def test_mask_expansion_host_check(tmp_path):
                     "-o", str(exe), os.path.join(ROOT, "tests", "native", "pair_mask_check.cpp")], check=True)
     r = subprocess.run([str(exe)], capture_output=True, text=True)
     assert r.returncode == 0 and r.stdout.strip() == "ok", r.stdout
+
+
+def test_sign_flip_host_check(tmp_path):
+    """The decode kernel's sign-flip operand construction (group_bits and
+    flip_pair in csrc/common.cuh), compiled for the host and checked against
+    the packed-format definition for every n_m, group, pair and mask."""
+    exe = tmp_path / "flip_check"
+    subprocess.run(["g++", "-std=c++17", "-O1", "-I", os.path.join(ROOT, "masked_glu_b200", "csrc"),
+                    "-o", str(exe), os.path.join(ROOT, "tests", "native", "flip_check.cpp")], check=True)
+    r = subprocess.run([str(exe)], capture_output=True, text=True)
+    assert r.returncode == 0 and r.stdout.strip() == "ok", r.stdout
+
+
+def test_logit_bit_rule_on_every_fp16_pattern(tmp_path):
+    """The mask-logit bit rule (logit_bit in csrc/common.cuh), compiled for
+    the host and evaluated on all 65536 binary16 patterns, equals numpy's
+    IEEE comparison logit > 0 (so +-0 and NaN give 0, +inf and positive
+    subnormals give 1)."""
+    import numpy as np
+    exe = tmp_path / "logit_bit_check"
+    subprocess.run(["g++", "-std=c++17", "-O1", "-I", os.path.join(ROOT, "masked_glu_b200", "csrc"),
+                    "-o", str(exe), os.path.join(ROOT, "tests", "native", "logit_bit_check.cpp")], check=True)
+    out = subprocess.run([str(exe)], capture_output=True, text=True, check=True).stdout.strip()
+    got = np.frombuffer(out.encode(), dtype=np.uint8) - ord("0")
+    with np.errstate(invalid="ignore"):
+        want = (np.arange(65536, dtype=np.uint16).view(np.float16) > 0).astype(np.uint8)
+    assert got.shape == want.shape and np.array_equal(got, want)
 
 
 def test_decode_schedule_host_check(tmp_path):
@@ -186,10 +211,10 @@ int main(void)
     printf("packed %zu\n", mglu_packed_bytes(4, 128, 4));
     printf("scratch_nonzero %d\n", mglu_scratch_bytes(4) > 0);
     printf("path %d %d\n", mglu_forward_path(1, MGLU_BF16), mglu_forward_path(64, MGLU_BF16));
-    /* rejected before any device work: unsupported n_m, bad act, d % 128 */
+    /* rejected before any device work: unsupported n_m, bad act, d % 8 */
     printf("nm3 %d\n", mglu_forward(x, 1, 128, W, 4, packed, 3, MGLU_ACT_SWISH, MGLU_BF16, out, 0, 0, 0));
     printf("act9 %d\n", mglu_forward(x, 1, 128, W, 4, packed, 4, 9, MGLU_BF16, out, 0, 0, 0));
-    printf("d64 %d\n", mglu_forward(x, 1, 64, W, 4, packed, 4, MGLU_ACT_GELU, MGLU_BF16, out, 0, 0, 0));
+    printf("d60 %d\n", mglu_forward(x, 1, 60, W, 4, packed, 4, MGLU_ACT_GELU, MGLU_BF16, out, 0, 0, 0));
     printf("zeroT %d\n", mglu_forward(x, 0, 128, W, 4, packed, 4, MGLU_ACT_RELU, MGLU_BF16, out, 0, 0, 0));
     printf("msg %s\n", mglu_status_string(MGLU_ERR_ALIGN));
     printf("f32path %d\n", mglu_forward_path(1, MGLU_F32));
@@ -215,5 +240,5 @@ def test_header_serves_a_plain_c99_caller(tmp_path):
     assert got["packed"] == str(128 * 4 * 4 // 8)
     assert got["scratch_nonzero"] == "1"
     assert got["path"] == "0 1" and got["f32path"] == "2"  # decode for 1 token, prefill for 64; fp32 path
-    assert got["nm3"] == "-2" and got["act9"] == "-1" and got["d64"] == "-3" and got["zeroT"] == "0"
+    assert got["nm3"] == "-2" and got["act9"] == "-1" and got["d60"] == "-3" and got["zeroT"] == "0"
     assert got["msg"] == "alignment requirement not met"

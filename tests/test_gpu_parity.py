@@ -311,3 +311,60 @@ def test_workspace_reused_across_token_counts_and_block_modes():
         torch.cuda.synchronize()
         assert mglu.last_device_status() == 0
         assert torch.equal(got, want), f"host call T={T} down={down} on a reused workspace differs"
+
+
+# ------------------------------------------------------------------ widths that are multiples of 8 only
+# The bf16 path accepts any d % 8 == 0 (and h % 8 == 0 for the down-projection).
+# Packed mask rows of d * n_m / 8 bytes that are not 16-byte strided cannot be
+# described by a tensor map; the tensor-core kernel then reads them directly.
+@pytest.mark.parametrize("n_m,T,d,h", [
+    (4, 1, 200, 100), (1, 3, 200, 64), (8, 9, 72, 50), (2, 16, 8, 24),        # decode
+    (2, 40, 200, 100), (1, 150, 136, 70), (4, 40, 1000, 64), (8, 40, 1000, 72),  # prefill, masks read directly
+    (8, 40, 1008, 72), (4, 129, 96, 130),                                       # prefill, ragged last k block
+])
+def test_widths_multiple_of_8(n_m, T, d, h):
+    case = inputs.make_case(T, d, h, n_m, seed=1400 + n_m + T + d + h)
+    got = run_forward(case, "swish")
+    ref, _ = oracle.forward(case.x.values, case.W.values, oracle_packed(case), n_m, ACT["swish"])
+    assert_close(got, ref, "bf16", f"d%8 n_m={n_m} T={T} d={d} h={h}")
+
+
+@pytest.mark.parametrize("T,h,d", [(1, 200, 40), (9, 72, 136), (40, 200, 72)])
+def test_down_proj_h_multiple_of_8(T, h, d):
+    rng = np.random.default_rng(1500 + T + h + d)
+    hid = inputs.normal(rng, (T, h), 1.0, "bf16")
+    Wd = inputs.normal(rng, (d, h), 0.02, "bf16")
+    big, y = guarded((T, d), torch.bfloat16)
+    mglu.down_proj(to_device(hid), to_device(Wd), out=y)
+    check_guards(big)
+    assert_close(to_f64(y), oracle.down(hid.values, Wd.values), "bf16", f"down h%8 T={T} h={h}")
+
+
+# ------------------------------------------------------------------ scale range
+def _scaled(case, e):
+    """The case with x multiplied by 2^e (exact for bf16 values in range)."""
+    vals, bits = inputs.round_bf16(case.x.values * 2.0 ** e)
+    assert np.array_equal(vals, case.x.values * 2.0 ** e)
+    case.x = inputs.Tensor(vals, bits, "bf16")
+    return case
+
+
+@pytest.mark.parametrize("n_m,T", [(8, 1), (8, 9), (4, 3), (8, 40)])
+@pytest.mark.parametrize("e", [-60, 60])
+def test_extreme_input_scale_matches_oracle(n_m, T, e):
+    """Masks select or negate whole weights, so every product is exact at
+    any input scale: outputs at x * 2^-60 and x * 2^60 still meet the bar."""
+    case = _scaled(inputs.make_case(T, 512, 96, n_m, seed=1600 + n_m + T), e)
+    got = run_forward(case, "swish")
+    ref, _ = oracle.forward(case.x.values, case.W.values, oracle_packed(case), n_m, ACT["swish"])
+    assert_close(got, ref, "bf16", f"scale 2^{e} n_m={n_m} T={T}")
+
+
+@pytest.mark.parametrize("n_m,T", [(8, 1), (4, 16), (8, 40)])
+def test_relu_is_homogeneous_of_degree_two(n_m, T):
+    """ReLU gating: out(c x) = c^2 out(x) exactly for c = 2^-40 (powers of two
+    scale every product, sum and rounding exactly while values stay normal)."""
+    base = inputs.make_case(T, 512, 96, n_m, seed=1700 + n_m + T)
+    got1 = run_forward(base, "relu")
+    got2 = run_forward(_scaled(inputs.make_case(T, 512, 96, n_m, seed=1700 + n_m + T), -40), "relu")
+    assert np.array_equal(got2, got1 * 2.0 ** -80)

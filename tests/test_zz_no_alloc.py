@@ -37,7 +37,7 @@ def test_rejects_before_any_launch():
     assert str(MAX_ROWS) in mglu.last_cuda_error()
     assert L.mglu_forward_decode_static(p, 17, 128, p, 64, p, 4, 0, p, None) == -2  # UNSUPPORTED
     assert L.mglu_forward_decode_static(p, 1, 128, p, 64, p, 3, 0, p, None) == -2
-    assert L.mglu_forward_decode_static(p, 1, 96, p, 64, p, 4, 0, p, None) == -3  # d % 128
+    assert L.mglu_forward_decode_static(p, 1, 100, p, 64, p, 4, 0, p, None) == -3  # d % 8
     assert L.mglu_forward_decode_static(p, 0, 128, p, 64, p, 4, 0, p, None) == 0  # T == 0: no-op
 
 
