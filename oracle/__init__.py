@@ -21,6 +21,7 @@ from .core import (  # noqa: F401
     ACT_GELU,
     ACT_RELU,
     ACT_SWISH,
+    GATE_DENSE,
     activation,
     build,
     down,

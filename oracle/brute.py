@@ -24,10 +24,12 @@ def act_ref(act: int, z: float) -> float:
     raise ValueError(act)
 
 
-def mglu_logical(x, W, M, act):
+def mglu_logical(x, W, M, act, dense_gate=False):
     """x: T lists of d floats; W: d lists of h floats; M: n_m x d x h of 0/1.
 
-    Returns T lists of h floats."""
+    dense_gate: the "Remove the gate mask (dense gate)" ablation ("Measured
+    effects", last row), read as: every gate is the whole product x W and
+    each value keeps its mask.  Returns T lists of h floats."""
     T, d, h, n_m = len(x), len(W), len(W[0]), len(M)
     out = []
     for b in range(T):
@@ -38,9 +40,9 @@ def mglu_logical(x, W, M, act):
                 gate = 0.0
                 value = 0.0
                 for k in range(d):
-                    if M[i][k][j]:
+                    if M[i][k][j] or dense_gate:
                         gate += x[b][k] * W[k][j]
-                    else:
+                    if not M[i][k][j]:
                         value += x[b][k] * W[k][j]
                 total += act_ref(act, gate) * value
             row.append(total)

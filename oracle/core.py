@@ -23,6 +23,8 @@ import numpy as np
 ACT_SWISH = 0
 ACT_GELU = 1
 ACT_RELU = 2
+# OR-ed into act: the dense-gate ablation, out = sum_i act(x W) * v_i
+GATE_DENSE = 16
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _SRC = os.path.join(_HERE, "mglu_oracle.c")

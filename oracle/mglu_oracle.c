@@ -52,6 +52,11 @@
 #define ORACLE_ACT_SWISH 0
 #define ORACLE_ACT_GELU 1
 #define ORACLE_ACT_RELU 2
+/* Flag OR-ed into act: the "dense gate" ablation ("Measured effects", last
+ * row: "Remove the gate mask (dense gate)").  Reading: the gate of every mask
+ * is the whole product x W (no mask), the value keeps its mask:
+ *     out[b,j] = sum_i act(sum_k x[b,k] W[k,j]) * v_i[b,j]                  */
+#define ORACLE_GATE_DENSE 16
 
 /* Gating activation ("Measured effects": Swish is the default, GELU and ReLU
  * are the ablation rows).  Swish with beta = 1 (SiLU, as in SwiGLU); GELU in
@@ -155,9 +160,11 @@ static double oracle_element(const double *x, int64_t d, const double *Ws,
 {
     double g[8], v[8], D, absw, resid;
     oracle_gate_value(x, d, Ws, packed, n_m, b, j, &D, g, v, &absw, &resid);
+    const int dense_gate = (act & ORACLE_GATE_DENSE) != 0;
+    const int a = act & ~ORACLE_GATE_DENSE;
     double acc = 0.0;
     for (int i = 0; i < n_m; ++i)
-        acc += oracle_act(act, g[i]) * v[i];
+        acc += oracle_act(a, dense_gate ? D : g[i]) * v[i];
     *out = acc;
     return absw > 0.0 ? resid / absw : resid;
 }
@@ -169,7 +176,8 @@ double oracle_forward(const double *x, int64_t T, int64_t d, const double *Ws,
                       int64_t h, const uint8_t *packed, int n_m, int act,
                       double *out)
 {
-    if (n_m < 1 || n_m > 8 || act < 0 || act > 2)
+    const int a = act & ~ORACLE_GATE_DENSE;
+    if (n_m < 1 || n_m > 8 || a < 0 || a > 2)
         return -1.0;
     double worst = 0.0;
 #pragma omp parallel for schedule(dynamic, 4) reduction(max : worst)
@@ -189,7 +197,8 @@ double oracle_forward_elems(const double *x, int64_t d, const double *Ws,
                             const int64_t *b_idx, const int64_t *j_idx,
                             double *out)
 {
-    if (n_m < 1 || n_m > 8 || act < 0 || act > 2)
+    const int a = act & ~ORACLE_GATE_DENSE;
+    if (n_m < 1 || n_m > 8 || a < 0 || a > 2)
         return -1.0;
     double worst = 0.0;
 #pragma omp parallel for schedule(dynamic, 16) reduction(max : worst)
