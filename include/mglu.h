@@ -67,6 +67,13 @@ typedef enum {
 } mglu_status;
 
 typedef enum { MGLU_ACT_SWISH = 0, MGLU_ACT_GELU = 1, MGLU_ACT_RELU = 2 } mglu_act;
+
+/* OR into act for the dense-gate ablation ("Masked Gated Linear Unit",
+ * "Measured effects", last row, "Remove the gate mask (dense gate)"): the
+ * gate of every mask is the whole product x W, each value keeps its mask,
+ *     out[b,j] = sum_{i<n_m} act((x W)[b,j]) * v_i[b,j].
+ * Accepted wherever an act is (forward, FFN block, host and static calls). */
+#define MGLU_GATE_DENSE 16
 typedef enum { MGLU_BF16 = 0, MGLU_F32 = 1 } mglu_dtype;
 
 /* Kernel families mglu_forward can launch (see mglu_forward_path). */
@@ -135,7 +142,8 @@ size_t mglu_scratch_bytes(int64_t rows);
  * limit (16 by default) one pass serves all tokens; above it a tensor-core
  * (tcgen05) kernel tiles tokens and weights.
  *   x [T][d], W [h][d], packed (from mglu_pack_masks with the same n_m, d, h),
- *   act in mglu_act, dtype in mglu_dtype, out [T][h],
+ *   act in mglu_act (optionally | MGLU_GATE_DENSE), dtype in mglu_dtype,
+ *   out [T][h],
  *   scratch / scratch_bytes: see mglu_scratch_bytes(h).
  * Errors: INVALID (also: scratch missing or too small on the decode path),
  * UNSUPPORTED, ALIGN, CUDA.

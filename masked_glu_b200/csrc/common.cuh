@@ -12,6 +12,10 @@
 namespace mglu {
 
 enum { ACT_SWISH = 0, ACT_GELU = 1, ACT_RELU = 2 };
+// Flag OR-ed into act: the dense-gate ablation ("Masked Gated Linear Unit",
+// "Measured effects", last row, "Remove the gate mask (dense gate)"): every
+// gate is the whole product x W, each value keeps its mask.
+enum { GATE_DENSE = 16, ACT_MASK = 15 };
 
 #ifdef __CUDACC__
 // Gating activation ("Masked Gated Linear Unit", "Measured effects": Swish

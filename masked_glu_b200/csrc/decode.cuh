@@ -216,13 +216,15 @@ __device__ __forceinline__ float out_value(int act, const float (&acc)[NM + 1][N
         return acc[0][t][r];
     } else {
         const float D = acc[0][t][r];
+        const bool dense_gate = (act & GATE_DENSE) != 0;
+        const int a = act & ACT_MASK;
         float o = 0.f;
 #pragma unroll
         for (int i = 0; i < NM; ++i) {
             const float h = acc[1 + i][t][r];
             const float g = 0.5f * (D + h);  // x (M_i . W)
             const float v = 0.5f * (D - h);  // x ((1 - M_i) . W)
-            o += act_fn(act, g) * v;
+            o += act_fn(a, dense_gate ? D : g) * v;
         }
         return o;
     }

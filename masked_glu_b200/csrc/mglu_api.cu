@@ -374,7 +374,7 @@ int check_forward(const void *x, int64_t T, int64_t d, const void *W, int64_t h,
 {
     if (!sizes_ok(T, d, h))
         return MGLU_ERR_INVALID;
-    if (act < 0 || act > 2 || (dtype != MGLU_BF16 && dtype != MGLU_F32))
+    if ((act & ~MGLU_GATE_DENSE) < 0 || (act & ~MGLU_GATE_DENSE) > 2 || (dtype != MGLU_BF16 && dtype != MGLU_F32))
         return MGLU_ERR_INVALID;
     if (!nm_supported(n_m))
         return MGLU_ERR_UNSUPPORTED;

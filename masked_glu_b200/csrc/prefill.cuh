@@ -354,6 +354,8 @@ __global__ void __launch_bounds__(Cfg<NM>::NTHREADS, 1) prefill_kernel(const __g
                                 tmem_ld_x8(tbase + (1 + i) * C::NJ + jc + 8 * h8,
                                            *reinterpret_cast<uint32_t(*)[8]>(&gv[i][8 * h8]));
                         tmem_wait_ld();
+                        const bool dense_gate = (act & GATE_DENSE) != 0;
+                        const int a = act & ACT_MASK;
 #pragma unroll
                         for (int e = 0; e < C::EC; ++e) {
                             const float D = __uint_as_float(dv[e]);
@@ -361,7 +363,7 @@ __global__ void __launch_bounds__(Cfg<NM>::NTHREADS, 1) prefill_kernel(const __g
 #pragma unroll
                             for (int i = 0; i < NM; ++i) {
                                 const float gi = __uint_as_float(gv[i][e]);
-                                acc += act_fn(act, gi) * (D - gi);
+                                acc += act_fn(a, dense_gate ? D : gi) * (D - gi);
                             }
                             o[e] = acc;
                         }

@@ -80,7 +80,7 @@ __global__ void __launch_bounds__(256) simt_f32_kernel(const float *__restrict__
                 for (int t = 0; t < kSimtTokens; ++t)
                     if (t == lane)
                         g = gate[i][t];
-                o += act_fn(act, g) * (D - g);
+                o += act_fn(act & ACT_MASK, (act & GATE_DENSE) ? D : g) * (D - g);
             }
         }
         out[(t0 + lane) * h + j] = o;

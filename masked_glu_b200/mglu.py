@@ -20,6 +20,7 @@ HEADER = os.path.join(os.path.dirname(_PKG), "include", "mglu.h")
 
 OK, ERR_INVALID, ERR_UNSUPPORTED, ERR_ALIGN, ERR_CUDA, ERR_TIMEOUT = 0, -1, -2, -3, -4, -5
 ACTS = {"swish": 0, "gelu": 1, "relu": 2}
+GATE_DENSE = 16  # OR-ed into act: the dense-gate ablation (act names may end in "+dense_gate")
 DTYPES = {torch.bfloat16: 0, torch.float32: 1}
 PATH_DECODE, PATH_PREFILL, PATH_F32 = 0, 1, 2
 
@@ -117,7 +118,12 @@ def _dtype(t: torch.Tensor) -> int:
 
 
 def _act(act) -> int:
-    return ACTS[act] if isinstance(act, str) else int(act)
+    if isinstance(act, str):
+        name, _, flag = act.partition("+")
+        if flag not in ("", "dense_gate"):
+            raise ValueError(f"unknown act modifier {flag!r}")
+        return ACTS[name] | (GATE_DENSE if flag else 0)
+    return int(act)
 
 
 def packed_bytes(n_m: int, d: int, h: int) -> int:

@@ -225,12 +225,11 @@ def test_decode_scratch_is_left_zeroed(T):
     assert np.array_equal(outs[0], outs[1]) and np.array_equal(outs[1], outs[2]), "run-to-run difference"
 
 
-# Shapes on which an earlier form of the decode kernel gave intermittent wrong
-# rows (about one operand read in ten thousand, only when its consumer warps
-# outran the TMA): the dense down-projection with K = 14336, which mixes
-# data-parallel and split row blocks, n_m = 4 with a three-stage ring, and
-# n_m = 8 with two token blocks.  Every repeat must match the oracle and be
-# bit-identical to the first.
+# Repeat tests: every repeat must match the oracle and be bit-identical to
+# the first call.  The shapes are those on which an earlier decode kernel
+# (a TMA ring shared by all warps of a CTA) gave intermittent wrong rows: the
+# dense down-projection with K = 14336, which mixes data-parallel and split
+# row blocks; n_m = 4 with eight tokens; n_m = 8 with two token blocks.
 @pytest.mark.parametrize("T", [1, 16])
 def test_dense_decode_repeatable_k14336(T):
     rng = np.random.default_rng(900 + T)
@@ -248,14 +247,14 @@ def test_dense_decode_repeatable_k14336(T):
         assert np.array_equal(y, first), f"repeat {rep} differs from the first call"
 
 
-@pytest.mark.parametrize("n_m,T,d,h", [(4, 8, 2048, 8192), (4, 4, 2048, 8192), (2, 8, 2048, 4096),
-                                       (8, 16, 4096, 2048)])
-def test_decode_repeatable(n_m, T, d, h):
+@pytest.mark.parametrize("n_m,T,d,h,reps", [(4, 8, 2048, 8192, 40), (4, 4, 2048, 8192, 8), (2, 8, 2048, 4096, 8),
+                                            (8, 16, 4096, 2048, 8), (8, 1, 4096, 14336, 8)])
+def test_decode_repeatable(n_m, T, d, h, reps):
     case = inputs.make_case(T, d, h, n_m, seed=950 + 31 * n_m + T)
     x, W, packed, _ = device_case(case)
     ref, _ = oracle.forward(case.x.values, case.W.values, oracle_packed(case), n_m, ACT["swish"])
     first = None
-    for rep in range(8):
+    for rep in range(reps):
         got = to_f64(mglu.forward(x, W, packed, n_m, "swish"))
         assert mglu.last_device_status() == 0
         assert_close(got, ref, "bf16", f"decode n_m={n_m} T={T} repeat {rep}")
@@ -368,3 +367,17 @@ def test_relu_is_homogeneous_of_degree_two(n_m, T):
     got1 = run_forward(base, "relu")
     got2 = run_forward(_scaled(inputs.make_case(T, 512, 96, n_m, seed=1700 + n_m + T), -40), "relu")
     assert np.array_equal(got2, got1 * 2.0 ** -80)
+
+
+# ------------------------------------------------------------------ dense-gate ablation
+@pytest.mark.parametrize("n_m,T,d,h,dtype", [(4, 1, 512, 200, "bf16"), (8, 9, 256, 96, "bf16"),
+                                             (4, 150, 384, 200, "bf16"), (1, 40, 256, 64, "bf16"),
+                                             (2, 5, 100, 37, "f32")])
+@pytest.mark.parametrize("act", ["swish", "gelu", "relu"])
+def test_dense_gate_matches_oracle(n_m, T, d, h, dtype, act):
+    """act | MGLU_GATE_DENSE: out = sum_i act(x W) v_i, on the decode, the
+    tensor-core and the fp32 kernels."""
+    case = inputs.make_case(T, d, h, n_m, seed=1900 + n_m + T + d, dtype=dtype)
+    got = run_forward(case, act + "+dense_gate")
+    ref, _ = oracle.forward(case.x.values, case.W.values, oracle_packed(case), n_m, ACT[act] | oracle.GATE_DENSE)
+    assert_close(got, ref, dtype, f"dense gate {act} n_m={n_m} T={T}")
