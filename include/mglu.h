@@ -152,6 +152,44 @@ int mglu_forward(const void *x, int64_t T, int64_t d, const void *W, int64_t h,
                  const uint8_t *packed, int n_m, int act, int dtype, void *out,
                  void *scratch, size_t scratch_bytes, void *stream);
 
+/* Weightings of routed masks (see mglu_route_topk). */
+typedef enum { MGLU_ROUTE_HARD = 0, MGLU_ROUTE_SOFTMAX = 1 } mglu_route_mode;
+
+/*
+ * Mask routing ("Masked Gated Linear Unit", "Measured effects": each token
+ * routed to only 1, or 2, of its 4 masks instead of summing all of them).
+ * The page defines no router; here one linear map scores the masks per
+ * token, r[b,i] = sum_k x[b,k] W_r[i,k] (fp32 accumulation, no bias), the k
+ * highest scores are kept (of equal scores the lower mask index; a NaN score
+ * never beats a number), and the token's mask weights are written:
+ *   MGLU_ROUTE_HARD:    1 for each kept mask, 0 otherwise;
+ *   MGLU_ROUTE_SOFTMAX: the softmax of all n_m scores for each kept mask,
+ *                       0 otherwise (as a mixture-of-experts router scales
+ *                       an expert by its probability).
+ *   x [T][d] and W_r [n_m][d] in dtype (MGLU_BF16 or MGLU_F32, aligned to
+ *   their element size); weights [T][n_m] float (written); scores
+ *   [T][n_m] float (written, may be NULL).  0 <= k <= n_m.
+ * The weights feed mglu_forward_weighted.  Errors: INVALID, UNSUPPORTED,
+ * ALIGN, CUDA.
+ */
+int mglu_route_topk(const void *x, int64_t T, int64_t d, const void *W_r,
+                    int n_m, int k, int mode, int dtype, float *weights,
+                    float *scores, void *stream);
+
+/*
+ * mglu_forward with per-token mask weights, the forward of routed masks:
+ *     out[b,j] = sum_{i<n_m} w[b,i] act(g_i[b,j]) v_i[b,j]
+ * (w = 1 everywhere is mglu_forward).  mask_weights: [T][n_m] float, device,
+ * 4-byte aligned; any values.  On the decode kernel (T <= the decode limit)
+ * a mask whose weight is 0 for every token of the call skips its products,
+ * so top-k routing with k < n_m does less arithmetic (the weights and mask
+ * bits are still read once).  Other arguments and errors as mglu_forward.
+ */
+int mglu_forward_weighted(const void *x, int64_t T, int64_t d, const void *W,
+                          int64_t h, const uint8_t *packed, int n_m, int act,
+                          int dtype, const float *mask_weights, void *out,
+                          void *scratch, size_t scratch_bytes, void *stream);
+
 /*
  * The FFN down-projection alone, a dense product (MGLU replaces only the two
  * GLU projections; "Masked Gated Linear Unit", "Problem"):

@@ -144,7 +144,8 @@ __device__ __forceinline__ uint2 ld_mask_chunk(const uint8_t *p)
 }
 
 // One stage's operands of one lane: 8 weights of rows g and g + 8, their
-// mask bits, and 8 values of x for each token block.
+// mask bits (loaded P stages ahead), and 8 values of x for each token block
+// (loaded one stage ahead: x is read from L1 or L2, not HBM).
 template <int NM, int NT>
 struct Operands {
     uint4 wa, wb;
@@ -172,20 +173,24 @@ __device__ __forceinline__ uint32_t u4(const uint4 &v, int q)
 }
 
 // h_I += x (S_I . W) for k16 sub-step S of the unit, then the next mask.
-template <int NM, int NT, int S, int I>
+// With ROUTED, masks whose bit in `used` is clear (no token of the call
+// gives them a nonzero weight) skip their products.
+template <int NM, int NT, bool ROUTED, int S, int I>
 struct FlipLoop {
     static __device__ __forceinline__ void run(float (&acc)[NM + 1][NT][4], const Operands<NM, NT> &o, uint32_t ra,
-                                               uint32_t rb)
+                                               uint32_t rb, uint32_t used)
     {
         if constexpr (I < NM) {
-            const uint32_t a0 = flip_pair(u4(o.wa, 2 * S), shl_fma<15 - I>(ra));
-            const uint32_t a1 = flip_pair(u4(o.wb, 2 * S), shl_fma<15 - I>(rb));
-            const uint32_t a2 = flip_pair(u4(o.wa, 2 * S + 1), shl_fma<7 - I>(ra));
-            const uint32_t a3 = flip_pair(u4(o.wb, 2 * S + 1), shl_fma<7 - I>(rb));
+            if (!ROUTED || ((used >> I) & 1u)) {
+                const uint32_t a0 = flip_pair(u4(o.wa, 2 * S), shl_fma<15 - I>(ra));
+                const uint32_t a1 = flip_pair(u4(o.wb, 2 * S), shl_fma<15 - I>(rb));
+                const uint32_t a2 = flip_pair(u4(o.wa, 2 * S + 1), shl_fma<7 - I>(ra));
+                const uint32_t a3 = flip_pair(u4(o.wb, 2 * S + 1), shl_fma<7 - I>(rb));
 #pragma unroll
-            for (int t = 0; t < NT; ++t)
-                mma_bf16_16816(acc[1 + I][t], a0, a1, a2, a3, u4(o.xv[t], 2 * S), u4(o.xv[t], 2 * S + 1));
-            FlipLoop<NM, NT, S, I + 1>::run(acc, o, ra, rb);
+                for (int t = 0; t < NT; ++t)
+                    mma_bf16_16816(acc[1 + I][t], a0, a1, a2, a3, u4(o.xv[t], 2 * S), u4(o.xv[t], 2 * S + 1));
+            }
+            FlipLoop<NM, NT, ROUTED, S, I + 1>::run(acc, o, ra, rb, used);
         }
     }
 };
@@ -195,8 +200,8 @@ struct FlipLoop {
 // inside the MMA is a permutation of the physical k that depends only on c
 // and S; x (operand B) is loaded with the same permutation, so every sum is
 // unchanged.
-template <int NM, int NT, int S>
-__device__ __forceinline__ void unit_step(float (&acc)[NM + 1][NT][4], const Operands<NM, NT> &o)
+template <int NM, int NT, bool ROUTED, int S>
+__device__ __forceinline__ void unit_step(float (&acc)[NM + 1][NT][4], const Operands<NM, NT> &o, uint32_t used)
 {
 #pragma unroll
     for (int t = 0; t < NT; ++t)
@@ -205,12 +210,15 @@ __device__ __forceinline__ void unit_step(float (&acc)[NM + 1][NT][4], const Ope
     if constexpr (NM > 0) {
         const uint32_t ra = group_bits<NM, S>(o.ma.x, o.ma.y);
         const uint32_t rb = group_bits<NM, S>(o.mb.x, o.mb.y);
-        FlipLoop<NM, NT, S, 0>::run(acc, o, ra, rb);
+        FlipLoop<NM, NT, ROUTED, S, 0>::run(acc, o, ra, rb, used);
     }
 }
 
+// The output of one (row, token): sum_i w_i act(g_i) v_i, with the token's
+// mask weights w (NULL: every weight 1).
 template <int NM, int NT>
-__device__ __forceinline__ float out_value(int act, const float (&acc)[NM + 1][NT][4], int t, int r)
+__device__ __forceinline__ float out_value(int act, const float (&acc)[NM + 1][NT][4], int t, int r,
+                                           const float *__restrict__ w)
 {
     if constexpr (NM == 0) {
         return acc[0][t][r];
@@ -224,7 +232,7 @@ __device__ __forceinline__ float out_value(int act, const float (&acc)[NM + 1][N
             const float h = acc[1 + i][t][r];
             const float g = 0.5f * (D + h);  // x (M_i . W)
             const float v = 0.5f * (D - h);  // x ((1 - M_i) . W)
-            o += act_fn(a, dense_gate ? D : g) * v;
+            o += (w ? w[i] : 1.0f) * (act_fn(a, dense_gate ? D : g) * v);
         }
         return o;
     }
@@ -260,11 +268,15 @@ __device__ __forceinline__ void add_slot(float (&acc)[NM + 1][NT][4], const floa
 // slots per CTA (first and last row block of its stream-K share), then one
 // arrival counter per row block.  Counters must be zero on entry and are
 // zero again when the kernel completes.
-template <int NM, int NT, int NW_ = DefaultShape<NM, NT>::NW, int P_ = DefaultShape<NM, NT>::P>
+//
+// ROUTED: per-token mask weights mw [T][NM] scale each mask's term, and a
+// mask that no token of the call weights (all its weights zero) skips its
+// products (the weight stream is read in full either way).
+template <int NM, int NT, bool ROUTED = false, int NW_ = DefaultShape<NM, NT>::NW, int P_ = DefaultShape<NM, NT>::P>
 __global__ void __launch_bounds__(Layout<NM, NT, NW_, P_>::NTHREADS, 1)
     decode_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__restrict__ W,
                   const uint8_t *__restrict__ packed, int T, int rows, int d, int act, float *__restrict__ ws_part,
-                  int *__restrict__ ws_count, __nv_bfloat16 *__restrict__ out)
+                  int *__restrict__ ws_count, __nv_bfloat16 *__restrict__ out, const float *__restrict__ mw)
 {
     using L = Layout<NM, NT, NW_, P_>;
     extern __shared__ __align__(16) float slots[];  // two sets of NW slots
@@ -280,6 +292,15 @@ __global__ void __launch_bounds__(Layout<NM, NT, NW_, P_>::NTHREADS, 1)
         return;
     pdl_wait();
 
+    // masks some token of the call weights
+    uint32_t used = (1u << NM) - 1u;
+    if constexpr (ROUTED) {
+        uint32_t u = 0;
+        for (int e = lane; e < T * NM; e += 32)
+            u |= (mw[e] != 0.0f ? 1u : 0u) << (e % NM);
+        used = __reduce_or_sync(0xffffffffu, u);
+    }
+
     // ----------------------------------------------------------------- consumers
     // This warp's 32-k unit of stage ks starts at k = ks * KS + 32 * warp;
     // this lane's 8 weights at k = that + 8 * c.
@@ -289,14 +310,11 @@ __global__ void __launch_bounds__(Layout<NM, NT, NW_, P_>::NTHREADS, 1)
 #pragma unroll
     for (int t = 0; t < NT; ++t)
         xrow[t] = 8 * t + g < T ? 8 * t + g : T - 1;  // lanes of absent tokens repeat the last one
-    auto load = [&](Operands<NM, NT> &o, int rb, int ks) {
+    auto load_w = [&](Operands<NM, NT> &o, int rb, int ks) {
         const int k = ks * L::KS + kl;
         const int ra = rb * ROWS + g, rbb = ra + 8;
         o.wa = o.wb = make_uint4(0u, 0u, 0u, 0u);
         o.ma = o.mb = make_uint2(0u, 0u);
-#pragma unroll
-        for (int t = 0; t < NT; ++t)
-            o.xv[t] = make_uint4(0u, 0u, 0u, 0u);
         if (k < d) {  // d % 8 == 0: a lane's 8 weights are all in range or all out
             if (ra < rows) {
                 o.wa = ld_stream_16(W + (int64_t)ra * d + k);
@@ -308,10 +326,13 @@ __global__ void __launch_bounds__(Layout<NM, NT, NW_, P_>::NTHREADS, 1)
                 if constexpr (NM > 0)
                     o.mb = ld_mask_chunk<NM>(packed + (int64_t)rbb * mrow + (int64_t)k * NM / 8);
             }
-#pragma unroll
-            for (int t = 0; t < NT; ++t)
-                o.xv[t] = ld_cached_16(x + (int64_t)xrow[t] * d + k);
         }
+    };
+    auto load_x = [&](Operands<NM, NT> &o, int ks) {
+        const int k = ks * L::KS + kl;
+#pragma unroll
+        for (int t = 0; t < NT; ++t)
+            o.xv[t] = k < d ? ld_cached_16(x + (int64_t)xrow[t] * d + k) : make_uint4(0u, 0u, 0u, 0u);
     };
 
     const int nflushes = sc.flushes();
@@ -371,7 +392,8 @@ __global__ void __launch_bounds__(Layout<NM, NT, NW_, P_>::NTHREADS, 1)
                     const int row = g + 8 * (r >> 1);
                     const int tok = 8 * t + 2 * c + (r & 1);
                     if (row0 + row < rows && tok < T)
-                        out[(int64_t)tok * rows + row0 + row] = __float2bfloat16_rn(out_value<NM, NT>(act, acc, t, r));
+                        out[(int64_t)tok * rows + row0 + row] = __float2bfloat16_rn(
+                            out_value<NM, NT>(act, acc, t, r, ROUTED ? mw + (int64_t)tok * NM : nullptr));
                 }
         }
         zero_acc<NM, NT>(acc);
@@ -381,16 +403,17 @@ __global__ void __launch_bounds__(Layout<NM, NT, NW_, P_>::NTHREADS, 1)
     zero_acc<NM, NT>(acc);
     Operands<NM, NT> buf[L::P];
 
-    // the load cursor runs P stages ahead of the compute cursor
+    // the weight cursor runs P stages ahead of the compute cursor, x one
     int rb_c, ks_c, rb_l, ks_l;
     sc.start(rb_c, ks_c);
     rb_l = rb_c, ks_l = ks_c;
 #pragma unroll
     for (int b = 0; b < L::P; ++b) {
         if (b < sc.n)
-            load(buf[b], rb_l, ks_l);
+            load_w(buf[b], rb_l, ks_l);
         sc.next(b, rb_l, ks_l);
     }
+    load_x(buf[0], ks_c);
 
     int nflush = 0;
     for (int i0 = 0; i0 < sc.n; i0 += L::P) {
@@ -399,9 +422,16 @@ __global__ void __launch_bounds__(Layout<NM, NT, NW_, P_>::NTHREADS, 1)
             const int i = i0 + b;
             if (i >= sc.n)
                 break;
+            {
+                // x of the next stage
+                int rb_n = rb_c, ks_n = ks_c;
+                sc.next(i, rb_n, ks_n);
+                if (i + 1 < sc.n)
+                    load_x(buf[(b + 1) % L::P], ks_n);
+            }
             if (ks_c * L::KS + 32 * warp < d) {
-                unit_step<NM, NT, 0>(acc, buf[b]);
-                unit_step<NM, NT, 1>(acc, buf[b]);
+                unit_step<NM, NT, ROUTED, 0>(acc, buf[b], used);
+                unit_step<NM, NT, ROUTED, 1>(acc, buf[b], used);
             }
             // the flush comes before this buffer's refill, so the finisher's
             // work does not hold the consumed stage's registers
@@ -430,7 +460,7 @@ __global__ void __launch_bounds__(Layout<NM, NT, NW_, P_>::NTHREADS, 1)
             }
             const int il = i + L::P;
             if (il < sc.n) {
-                load(buf[b], rb_l, ks_l);
+                load_w(buf[b], rb_l, ks_l);
                 sc.next(il, rb_l, ks_l);
             }
             sc.next(i, rb_c, ks_c);

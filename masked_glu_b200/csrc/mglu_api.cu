@@ -16,6 +16,7 @@
 #include "pack.cuh"
 #include "prefill.cuh"
 #include "ptx.cuh"
+#include "route.cuh"
 #include "simt.cuh"
 
 namespace {
@@ -205,9 +206,9 @@ int launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, int smem, cudaSt
 }
 
 // ------------------------------------------------------------------ decode
-template <int NM, int NT>
+template <int NM, int NT, bool ROUTED>
 int launch_decode(const void *x, int64_t T, int64_t d, const void *W, int64_t rows, const uint8_t *packed, int act,
-                  void *out, void *ws, cudaStream_t s)
+                  void *out, void *ws, cudaStream_t s, const float *mw)
 {
     using L = mglu::dec::Layout<NM, NT>;
     if (d >= ((int64_t)1 << 22) || rows >= ((int64_t)1 << 27))
@@ -215,7 +216,7 @@ int launch_decode(const void *x, int64_t T, int64_t d, const void *W, int64_t ro
     int dev = 0, rc = current_device(&dev);
     if (rc)
         return rc;
-    if ((rc = ensure_smem<mglu::dec::decode_kernel<NM, NT>>(L::SMEM, dev)))
+    if ((rc = ensure_smem<mglu::dec::decode_kernel<NM, NT, ROUTED>>(L::SMEM, dev)))
         return rc;
     const int64_t rb = (rows + mglu::dec::ROWS - 1) / mglu::dec::ROWS;
     const int64_t units = rb * ((d + L::KS - 1) / L::KS);
@@ -226,24 +227,29 @@ int launch_decode(const void *x, int64_t T, int64_t d, const void *W, int64_t ro
         grid = units;
     float *ws_part = reinterpret_cast<float *>(ws);
     int *ws_count = reinterpret_cast<int *>(reinterpret_cast<uint8_t *>(ws) + mglu::dec::part_bytes());
-    return launch_pdl(mglu::dec::decode_kernel<NM, NT>, dim3((unsigned)grid), dim3(L::NTHREADS), L::SMEM, s,
+    return launch_pdl(mglu::dec::decode_kernel<NM, NT, ROUTED>, dim3((unsigned)grid), dim3(L::NTHREADS), L::SMEM, s,
                       "decode launch", reinterpret_cast<const __nv_bfloat16 *>(x),
                       reinterpret_cast<const __nv_bfloat16 *>(W), packed, (int)T, (int)rows, (int)d, act, ws_part,
-                      ws_count, reinterpret_cast<__nv_bfloat16 *>(out));
+                      ws_count, reinterpret_cast<__nv_bfloat16 *>(out), mw);
 }
 
 template <int NM>
 int decode_nt(const void *x, int64_t T, int64_t d, const void *W, int64_t rows, const uint8_t *packed, int act,
-              void *out, void *ws, cudaStream_t s)
+              void *out, void *ws, cudaStream_t s, const float *mw)
 {
-    return T <= 8 ? launch_decode<NM, 1>(x, T, d, W, rows, packed, act, out, ws, s)
-                  : launch_decode<NM, 2>(x, T, d, W, rows, packed, act, out, ws, s);
+    if constexpr (NM > 0) {
+        if (mw)
+            return T <= 8 ? launch_decode<NM, 1, true>(x, T, d, W, rows, packed, act, out, ws, s, mw)
+                          : launch_decode<NM, 2, true>(x, T, d, W, rows, packed, act, out, ws, s, mw);
+    }
+    return T <= 8 ? launch_decode<NM, 1, false>(x, T, d, W, rows, packed, act, out, ws, s, nullptr)
+                  : launch_decode<NM, 2, false>(x, T, d, W, rows, packed, act, out, ws, s, nullptr);
 }
 
 // ------------------------------------------------------------------ prefill
 template <int NM>
 int launch_prefill(const void *x, int64_t T, int64_t d, const void *W, int64_t rows, const uint8_t *packed, int act,
-                   void *out, void *, cudaStream_t s)
+                   void *out, void *, cudaStream_t s, const float *mw)
 {
     using C = mglu::pf::Cfg<NM>;
     int dev = 0, rc = current_device(&dev);
@@ -274,20 +280,20 @@ int launch_prefill(const void *x, int64_t T, int64_t d, const void *W, int64_t r
     (void)kernel;
     return launch_pdl(mglu::pf::prefill_kernel<NM>, dim3((unsigned)grid), dim3(mglu::pf::Cfg<NM>::NTHREADS), C::SMEM, s,
                       "prefill launch", tx, tw, tm, (int)T, (int)rows, (int)d, act,
-                      reinterpret_cast<__nv_bfloat16 *>(out), packed, mask_direct);
+                      reinterpret_cast<__nv_bfloat16 *>(out), packed, mask_direct, mw);
 }
 
 // ------------------------------------------------------------------ fp32
 template <int NM>
 int launch_simt(const void *x, int64_t T, int64_t d, const void *W, int64_t rows, const uint8_t *packed, int act,
-                void *out, void *, cudaStream_t s)
+                void *out, void *, cudaStream_t s, const float *mw)
 {
     const dim3 grid((unsigned)((rows + 7) / 8), (unsigned)((T + mglu::kSimtTokens - 1) / mglu::kSimtTokens));
     if (grid.y > 65535u)
         return MGLU_ERR_INVALID;
     mglu::simt_f32_kernel<NM><<<grid, 256, 0, s>>>(reinterpret_cast<const float *>(x), T, d,
                                                      reinterpret_cast<const float *>(W), rows, packed, act,
-                                                     reinterpret_cast<float *>(out));
+                                                     reinterpret_cast<float *>(out), mw);
     return check_launch("fp32 launch");
 }
 
@@ -331,14 +337,14 @@ int path_for(int64_t T, int dtype)
 // One product of the library: out[T][rows] from x[T][d] and W[rows][d] with
 // n_m masks (n_m = 0: dense).  Arguments already validated.
 int run_product(const void *x, int64_t T, int64_t d, const void *W, int64_t rows, const uint8_t *packed, int n_m,
-                int act, int dtype, void *out, void *ws, cudaStream_t s)
+                int act, int dtype, void *out, void *ws, cudaStream_t s, const float *mw = nullptr)
 {
     if (T == 0)
         return MGLU_OK;
     switch (path_for(T, dtype)) {
-    case MGLU_PATH_F32: return by_nm<SimtF>(n_m, x, T, d, W, rows, packed, act, out, ws, s);
-    case MGLU_PATH_DECODE: return by_nm<DecodeF>(n_m, x, T, d, W, rows, packed, act, out, ws, s);
-    default: return by_nm<PrefillF>(n_m, x, T, d, W, rows, packed, act, out, ws, s);
+    case MGLU_PATH_F32: return by_nm<SimtF>(n_m, x, T, d, W, rows, packed, act, out, ws, s, mw);
+    case MGLU_PATH_DECODE: return by_nm<DecodeF>(n_m, x, T, d, W, rows, packed, act, out, ws, s, mw);
+    default: return by_nm<PrefillF>(n_m, x, T, d, W, rows, packed, act, out, ws, s, mw);
     }
 }
 
@@ -551,6 +557,55 @@ int mglu_forward(const void *x, int64_t T, int64_t d, const void *W, int64_t h, 
     return run_product(x, T, d, W, h, packed, n_m, act, dtype, out, scratch, reinterpret_cast<cudaStream_t>(stream));
 }
 
+int mglu_forward_weighted(const void *x, int64_t T, int64_t d, const void *W, int64_t h, const uint8_t *packed,
+                          int n_m, int act, int dtype, const float *mask_weights, void *out, void *scratch,
+                          size_t scratch_bytes_, void *stream)
+{
+    int rc = check_forward(x, T, d, W, h, packed, n_m, act, dtype, out);
+    if (rc)
+        return rc;
+    if (T > 0 && !mask_weights)
+        return MGLU_ERR_INVALID;
+    if (T > 0 && !aligned(mask_weights, 4))
+        return MGLU_ERR_ALIGN;
+    if ((rc = check_scratch(T, dtype, h, scratch, scratch_bytes_)))
+        return rc;
+    return run_product(x, T, d, W, h, packed, n_m, act, dtype, out, scratch, reinterpret_cast<cudaStream_t>(stream),
+                       mask_weights);
+}
+
+int mglu_route_topk(const void *x, int64_t T, int64_t d, const void *W_r, int n_m, int k, int mode, int dtype,
+                    float *weights, float *scores, void *stream)
+{
+    if (!sizes_ok(T, d, 1) || (dtype != MGLU_BF16 && dtype != MGLU_F32) || (mode != MGLU_ROUTE_HARD &&
+                                                                             mode != MGLU_ROUTE_SOFTMAX))
+        return MGLU_ERR_INVALID;
+    if (!nm_supported(n_m))
+        return MGLU_ERR_UNSUPPORTED;
+    if (k < 0 || k > n_m)
+        return MGLU_ERR_INVALID;
+    if (T == 0)
+        return MGLU_OK;
+    if (!x || !W_r || !weights)
+        return MGLU_ERR_INVALID;
+    const uintptr_t es = dtype == MGLU_BF16 ? 2 : 4;
+    if (!aligned(x, es) || !aligned(W_r, es) || !aligned(weights, 4) || (scores && !aligned(scores, 4)))
+        return MGLU_ERR_ALIGN;
+    const int64_t blocks = (T + 7) / 8;
+    if (blocks > 0x7FFFFFFF)
+        return MGLU_ERR_INVALID;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (dtype == MGLU_BF16)
+        mglu::route_kernel<__nv_bfloat16><<<(unsigned)blocks, 256, 0, s>>>(
+            reinterpret_cast<const __nv_bfloat16 *>(x), T, d, reinterpret_cast<const __nv_bfloat16 *>(W_r), n_m, k,
+            mode, weights, scores);
+    else
+        mglu::route_kernel<float><<<(unsigned)blocks, 256, 0, s>>>(reinterpret_cast<const float *>(x), T, d,
+                                                                    reinterpret_cast<const float *>(W_r), n_m, k,
+                                                                    mode, weights, scores);
+    return check_launch("route launch");
+}
+
 int mglu_down_proj(const void *hid, int64_t T, int64_t h, const void *W_down, int64_t d, int dtype, void *y,
                    void *scratch, size_t scratch_bytes_, void *stream)
 {
@@ -626,7 +681,7 @@ int mglu_forward_decode_static(const void *x, int64_t T, int64_t d, const void *
         cudaMemsetAsync(reinterpret_cast<uint8_t *>(ws) + mglu::dec::part_bytes(), 0, counters, s);
     if (e != cudaSuccess)
         return cuda_fail(e, "clear built-in decode scratch counters");
-    return by_nm<DecodeF>(n_m, x, T, d, W, h, packed, act, out, ws, s);
+    return by_nm<DecodeF>(n_m, x, T, d, W, h, packed, act, out, ws, s, (const float *)nullptr);
 }
 
 size_t mglu_host_workspace_bytes(int64_t T, int64_t d, int64_t h, int n_m, int dtype, int with_down)

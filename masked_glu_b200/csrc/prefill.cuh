@@ -116,6 +116,8 @@ __device__ __forceinline__ uint2 load_mask_global(const uint8_t *packed, int row
         return make_uint2(__ldg(p), 0u);
 }
 
+// mw: per-token mask weights [T][NM] that scale each mask's term (NULL:
+// every weight 1).
 // mask_direct != 0: the packed rows are not 16-byte strided (d * NM / 8 is
 // not a multiple of 16), so no tensor map can describe them; the builders
 // then read each chunk's mask bits from global memory (issued before they
@@ -127,7 +129,8 @@ __global__ void __launch_bounds__(Cfg<NM>::NTHREADS, 1) prefill_kernel(const __g
                                                               const __grid_constant__ CUtensorMap tm_m, int T,
                                                               int rows, int d, int act,
                                                               __nv_bfloat16 *__restrict__ out,
-                                                              const uint8_t *__restrict__ packed, int mask_direct)
+                                                              const uint8_t *__restrict__ packed, int mask_direct,
+                                                              const float *__restrict__ mw)
 {
     using C = Cfg<NM>;
     extern __shared__ uint8_t smem_raw[];
@@ -331,6 +334,10 @@ __global__ void __launch_bounds__(Cfg<NM>::NTHREADS, 1) prefill_kernel(const __g
             const int m0 = (tile % num_m) * BM;
             const int n0 = (tile / num_m) * C::NJ;
             const int tok = m0 + 32 * q + lane;
+            float wt[NM > 0 ? NM : 1];
+#pragma unroll
+            for (int i = 0; i < (NM > 0 ? NM : 1); ++i)
+                wt[i] = mw && tok < T ? mw[(int64_t)tok * NM + i] : 1.0f;
             const uint32_t tbase = tmem_base + ((uint32_t)(32 * q) << 16) + (uint32_t)(b * ACC_STRIDE);
             __nv_bfloat16 *orow = out + (int64_t)tok * rows;
             for (int jc = 0; jc < C::NJ; jc += C::EC) {
@@ -363,7 +370,7 @@ __global__ void __launch_bounds__(Cfg<NM>::NTHREADS, 1) prefill_kernel(const __g
 #pragma unroll
                             for (int i = 0; i < NM; ++i) {
                                 const float gi = __uint_as_float(gv[i][e]);
-                                acc += act_fn(a, dense_gate ? D : gi) * (D - gi);
+                                acc += wt[i] * (act_fn(a, dense_gate ? D : gi) * (D - gi));
                             }
                             o[e] = acc;
                         }

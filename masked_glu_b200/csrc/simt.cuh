@@ -13,12 +13,13 @@ namespace mglu {
 constexpr int kSimtTokens = 4;
 
 // NM = 0: dense product out[b][j] = sum_k x[b][k] * W[j][k] (the down-projection).
-// NM > 0: out[b][j] = sum_i act(g_i) * (D - g_i) with g_i the gate part of mask i.
+// NM > 0: out[b][j] = sum_i w_i act(g_i) * (D - g_i) with g_i the gate part
+// of mask i and w_i the token's mask weight (mw [T][NM]; NULL: 1).
 template <int NM>
 __global__ void __launch_bounds__(256) simt_f32_kernel(const float *__restrict__ x, int64_t T, int64_t d,
                                                        const float *__restrict__ W, int64_t h,
                                                        const uint8_t *__restrict__ packed, int act,
-                                                       float *__restrict__ out)
+                                                       float *__restrict__ out, const float *__restrict__ mw)
 {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int64_t j = (int64_t)blockIdx.x * 8 + warp;
@@ -80,7 +81,8 @@ __global__ void __launch_bounds__(256) simt_f32_kernel(const float *__restrict__
                 for (int t = 0; t < kSimtTokens; ++t)
                     if (t == lane)
                         g = gate[i][t];
-                o += act_fn(act & ACT_MASK, (act & GATE_DENSE) ? D : g) * (D - g);
+                const float wi = mw ? mw[(t0 + lane) * NM + i] : 1.0f;
+                o += wi * (act_fn(act & ACT_MASK, (act & GATE_DENSE) ? D : g) * (D - g));
             }
         }
         out[(t0 + lane) * h + j] = o;

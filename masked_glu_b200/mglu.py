@@ -59,6 +59,8 @@ def lib() -> ctypes.CDLL:
             "mglu_scratch_bytes": (SZ, [I64]),
             "mglu_forward": (I32, [P, I64, I64, P, I64, P, I32, I32, I32, P, P, SZ, P]),
             "mglu_down_proj": (I32, [P, I64, I64, P, I64, I32, P, P, SZ, P]),
+            "mglu_route_topk": (I32, [P, I64, I64, P, I32, I32, I32, I32, P, P, P]),
+            "mglu_forward_weighted": (I32, [P, I64, I64, P, I64, P, I32, I32, I32, P, P, P, SZ, P]),
             "mglu_workspace_bytes": (SZ, [I64, I64, I64, I32, I32]),
             "mglu_forward_down": (I32, [P, I64, I64, P, I64, P, I32, I32, I32, P, P, SZ, P, P]),
             "mglu_forward_decode_static": (I32, [P, I64, I64, P, I64, P, I32, I32, P, P]),
@@ -194,6 +196,46 @@ def forward(x: torch.Tensor, W: torch.Tensor, packed: torch.Tensor, n_m: int, ac
         scratch = default_scratch(h, x.device)
     _check(lib().mglu_forward(_ptr(x), T, d, _ptr(W), h, _ptr(packed), n_m, _act(act), _dtype(x),
                               _ptr(out), _ptr(scratch), _nbytes(scratch), _stream(stream)), "mglu_forward")
+    return out
+
+
+ROUTE_MODES = {"hard": 0, "softmax": 1}
+
+
+def route_topk(x: torch.Tensor, W_r: torch.Tensor, k: int, mode="hard", weights: Optional[torch.Tensor] = None,
+               scores: Optional[torch.Tensor] = None, stream=None):
+    """Router scores x W_r^T, top-k per token, mask weights [T][n_m] float.
+    Returns (weights, scores)."""
+    T, d = x.shape
+    n_m = W_r.shape[0]
+    if W_r.shape[1] != d or W_r.dtype != x.dtype:
+        raise ValueError("W_r must be [n_m][d] with x's dtype")
+    if weights is None:
+        weights = torch.empty((T, n_m), dtype=torch.float32, device=x.device)
+    if scores is None:
+        scores = torch.empty((T, n_m), dtype=torch.float32, device=x.device)
+    _check(lib().mglu_route_topk(_ptr(x), T, d, _ptr(W_r), n_m, int(k), ROUTE_MODES.get(mode, mode), _dtype(x),
+                                 _ptr(weights), _ptr(scores), _stream(stream)), "mglu_route_topk")
+    return weights, scores
+
+
+def forward_weighted(x: torch.Tensor, W: torch.Tensor, packed: torch.Tensor, n_m: int, mask_weights: torch.Tensor,
+                     act="swish", out: Optional[torch.Tensor] = None, scratch: Optional[torch.Tensor] = None,
+                     stream=None) -> torch.Tensor:
+    """out [T][h] = sum_i w[b, i] act(g_i) v_i with mask_weights [T][n_m] float."""
+    T, d = x.shape
+    h = W.shape[0]
+    if W.shape[1] != d or W.dtype != x.dtype:
+        raise ValueError("W must be [h][d] with x's dtype")
+    if mask_weights.shape != (T, n_m) or mask_weights.dtype != torch.float32:
+        raise ValueError("mask_weights must be [T][n_m] float32")
+    if out is None:
+        out = torch.empty((T, h), dtype=x.dtype, device=x.device)
+    if scratch is None:
+        scratch = default_scratch(h, x.device)
+    _check(lib().mglu_forward_weighted(_ptr(x), T, d, _ptr(W), h, _ptr(packed), n_m, _act(act), _dtype(x),
+                                       _ptr(mask_weights), _ptr(out), _ptr(scratch), _nbytes(scratch),
+                                       _stream(stream)), "mglu_forward_weighted")
     return out
 
 
