@@ -17,7 +17,8 @@
  *
  * Conventions for every call:
  *  - All tensor pointers are DEVICE pointers owned by the caller.  The library
- *    allocates no device memory on any call declared here; the little global
+ *    allocates no device memory on any call declared here except
+ *    mglu_backward's first call (its cuBLAS handle); the little global
  *    scratch the decode kernel needs is a caller-provided buffer (see
  *    mglu_scratch_bytes).
  *  - Calls are asynchronous and ordered on `stream` (a cudaStream_t passed as
@@ -292,6 +293,40 @@ int mglu_forward_host(const void *x_host, int64_t T, int64_t d, const void *W,
                       int64_t h, const uint8_t *packed, int n_m, int act,
                       int dtype, const void *W_down, void *workspace,
                       size_t workspace_bytes, void *result_host, void *stream);
+
+/* Device workspace mglu_backward needs (0 for bad input). */
+size_t mglu_backward_workspace_bytes(int64_t T, int64_t d, int64_t h, int n_m);
+
+/*
+ * The training path's backward through out = MGLU(x) for a given loss
+ * gradient dout = dL/dout ("Masked Gated Linear Unit", "Limitations": the
+ * masks are learned, held as FP16 logits while training; its list of prior
+ * work names the straight-through estimator).  The page gives no formula;
+ * the reading: the gradients of x and W are the exact derivatives of the
+ * forward with the binary masks held fixed (ReLU takes the subgradient 0 at
+ * 0), and a mask logit receives the loss gradient of its binary mask entry
+ * unchanged (straight through):
+ *     a_i = dout act'(g_i) v_i,   c_i = dout act(g_i)
+ *     dx      = sum_i a_i (M_i . W)^T-product + c_i ((1 - M_i) . W)
+ *     dW      = sum_i M_i . (a_i^T x) + (1 - M_i) . (c_i^T x)
+ *     dlogits_i = W . ((a_i - c_i)^T x)
+ *   x [T][d], W [h][d], packed, dout [T][h]: bf16 device (as mglu_forward;
+ *   act without MGLU_GATE_DENSE, else UNSUPPORTED).
+ *   dx [T][d], dW [h][d], dlogits [n_m][h][d]: float device, 16-byte
+ *   aligned, written; dlogits may be NULL (masks held fixed).
+ *   workspace: device, 256-byte aligned, >= mglu_backward_workspace_bytes.
+ * The g_i are recomputed on the tensor cores and the backward's coefficients
+ * formed in that kernel's epilogue (rounded to bf16); the masked operand and
+ * the final masked combination are this library's kernels; the two plain
+ * products over the materialised operands run on cuBLAS, which is loaded on
+ * the first call and, unlike the rest of this library, allocates its own
+ * handle memory then.  Errors: as mglu_forward, plus CUDA if cuBLAS cannot
+ * be loaded.
+ */
+int mglu_backward(const void *x, int64_t T, int64_t d, const void *W,
+                  int64_t h, const uint8_t *packed, int n_m, int act,
+                  const void *dout, float *dx, float *dW, float *dlogits,
+                  void *workspace, size_t workspace_bytes, void *stream);
 
 /* Which kernel family mglu_forward uses for T tokens of `dtype`. */
 int mglu_forward_path(int64_t T, int dtype);

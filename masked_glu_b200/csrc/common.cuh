@@ -29,6 +29,20 @@ __device__ __forceinline__ float act_fn(int act, float z)
         return 0.5f * z * (1.0f + erff(z * 0.70710678118654752440f));
     return fmaxf(z, 0.0f);
 }
+
+// Its derivative, for the training path: Swish sigma(z) + z sigma(z) (1 -
+// sigma(z)); GELU Phi(z) + z phi(z); ReLU 1 for z > 0, else 0 (the subgradient
+// 0 at 0).
+__device__ __forceinline__ float act_grad_fn(int act, float z)
+{
+    if (act == ACT_SWISH) {
+        const float s = __fdividef(1.0f, 1.0f + __expf(-z));
+        return s + z * s * (1.0f - s);
+    }
+    if (act == ACT_GELU)
+        return 0.5f * (1.0f + erff(z * 0.70710678118654752440f)) + z * 0.39894228040143267794f * __expf(-0.5f * z * z);
+    return z > 0.0f ? 1.0f : 0.0f;
+}
 #endif
 
 // prmt in default mode; on the host an emulation of the PTX definition so the

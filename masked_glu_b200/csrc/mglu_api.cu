@@ -1,8 +1,10 @@
 // mglu_api.cu -- the C ABI of libmglu.so (declared in include/mglu.h):
 // argument checks, TMA descriptor encoding, kernel choice and launches.
 // Everything is one translation unit so the device status word is shared.
+#include <cublas_v2.h>
 #include <cuda.h>
 #include <cuda_runtime.h>
+#include <dlfcn.h>
 
 #include <cstdint>
 #include <cstdio>
@@ -18,6 +20,7 @@
 #include "ptx.cuh"
 #include "route.cuh"
 #include "simt.cuh"
+#include "train.cuh"
 
 namespace {
 
@@ -247,9 +250,10 @@ int decode_nt(const void *x, int64_t T, int64_t d, const void *W, int64_t rows, 
 }
 
 // ------------------------------------------------------------------ prefill
-template <int NM>
+template <int NM, bool GRAD = false>
 int launch_prefill(const void *x, int64_t T, int64_t d, const void *W, int64_t rows, const uint8_t *packed, int act,
-                   void *out, void *, cudaStream_t s, const float *mw)
+                   void *out, void *, cudaStream_t s, const float *mw, const void *dout = nullptr,
+                   void *gout = nullptr)
 {
     using C = mglu::pf::Cfg<NM>;
     int dev = 0, rc = current_device(&dev);
@@ -272,15 +276,14 @@ int launch_prefill(const void *x, int64_t T, int64_t d, const void *W, int64_t r
     } else {
         tm = tw;  // not read
     }
-    auto kernel = mglu::pf::prefill_kernel<NM>;
-    if ((rc = ensure_smem<mglu::pf::prefill_kernel<NM>>(C::SMEM, dev)))
+    if ((rc = ensure_smem<mglu::pf::prefill_kernel<NM, GRAD>>(C::SMEM, dev)))
         return rc;
     const int64_t tiles = ((T + mglu::pf::BM - 1) / mglu::pf::BM) * ((rows + C::NJ - 1) / C::NJ);
     const int grid = (int)(tiles < sm_count(dev) ? tiles : sm_count(dev));
-    (void)kernel;
-    return launch_pdl(mglu::pf::prefill_kernel<NM>, dim3((unsigned)grid), dim3(mglu::pf::Cfg<NM>::NTHREADS), C::SMEM, s,
-                      "prefill launch", tx, tw, tm, (int)T, (int)rows, (int)d, act,
-                      reinterpret_cast<__nv_bfloat16 *>(out), packed, mask_direct, mw);
+    return launch_pdl(mglu::pf::prefill_kernel<NM, GRAD>, dim3((unsigned)grid), dim3(mglu::pf::Cfg<NM>::NTHREADS),
+                      C::SMEM, s, "prefill launch", tx, tw, tm, (int)T, (int)rows, (int)d, act,
+                      reinterpret_cast<__nv_bfloat16 *>(out), packed, mask_direct, mw,
+                      reinterpret_cast<const __nv_bfloat16 *>(dout), reinterpret_cast<__nv_bfloat16 *>(gout));
 }
 
 // ------------------------------------------------------------------ fp32
@@ -503,9 +506,166 @@ int static_scratch(int dev, cudaStream_t s, void **ptr)
     return MGLU_OK;
 }
 
+// ------------------------------------------------------------------ training path
+// cuBLAS is loaded on the first backward call (dlopen), so the forward
+// library does not depend on it.  It serves the two plain GEMMs of the
+// backward; the MGLU-specific steps are this library's kernels.
+struct Cublas {
+    using Create = cublasStatus_t (*)(cublasHandle_t *);
+    using SetStream = cublasStatus_t (*)(cublasHandle_t, cudaStream_t);
+    using GemmEx = cublasStatus_t (*)(cublasHandle_t, cublasOperation_t, cublasOperation_t, int, int, int,
+                                      const void *, const void *, cudaDataType, int, const void *, cudaDataType, int,
+                                      const void *, void *, cudaDataType, int, cublasComputeType_t, cublasGemmAlgo_t);
+    using GemmBatched = cublasStatus_t (*)(cublasHandle_t, cublasOperation_t, cublasOperation_t, int, int, int,
+                                           const void *, const void *, cudaDataType, int, long long, const void *,
+                                           cudaDataType, int, long long, const void *, void *, cudaDataType, int,
+                                           long long, int, cublasComputeType_t, cublasGemmAlgo_t);
+    Create create = nullptr;
+    SetStream set_stream = nullptr;
+    GemmEx gemm = nullptr;
+    GemmBatched gemm_batched = nullptr;
+    cublasHandle_t handle[kMaxDevices] = {};
+};
+
+std::mutex g_cublas_mu;
+Cublas g_cublas;
+
+int cublas_for(int dev, cudaStream_t s, Cublas **out)
+{
+    std::lock_guard<std::mutex> lock(g_cublas_mu);
+    Cublas &c = g_cublas;
+    if (!c.create) {
+        void *h = dlopen("libcublas.so.12", RTLD_NOW | RTLD_LOCAL);
+        if (!h)
+            h = dlopen("libcublas.so", RTLD_NOW | RTLD_LOCAL);
+        if (!h) {
+            snprintf(g_last_cuda_error, sizeof(g_last_cuda_error), "libcublas could not be loaded");
+            return MGLU_ERR_CUDA;
+        }
+        c.set_stream = reinterpret_cast<Cublas::SetStream>(dlsym(h, "cublasSetStream_v2"));
+        c.gemm = reinterpret_cast<Cublas::GemmEx>(dlsym(h, "cublasGemmEx"));
+        c.gemm_batched = reinterpret_cast<Cublas::GemmBatched>(dlsym(h, "cublasGemmStridedBatchedEx"));
+        Cublas::Create cr = reinterpret_cast<Cublas::Create>(dlsym(h, "cublasCreate_v2"));
+        if (!cr || !c.set_stream || !c.gemm || !c.gemm_batched) {
+            snprintf(g_last_cuda_error, sizeof(g_last_cuda_error), "libcublas lacks a needed entry point");
+            return MGLU_ERR_CUDA;
+        }
+        c.create = cr;
+    }
+    if (!c.handle[dev] && c.create(&c.handle[dev]) != CUBLAS_STATUS_SUCCESS) {
+        c.handle[dev] = nullptr;
+        snprintf(g_last_cuda_error, sizeof(g_last_cuda_error), "cublasCreate failed");
+        return MGLU_ERR_CUDA;
+    }
+    if (c.set_stream(c.handle[dev], s) != CUBLAS_STATUS_SUCCESS) {
+        snprintf(g_last_cuda_error, sizeof(g_last_cuda_error), "cublasSetStream failed");
+        return MGLU_ERR_CUDA;
+    }
+    *out = &c;
+    return MGLU_OK;
+}
+
+struct BwdLayout {
+    size_t g, b, e, total;  // byte offsets of G, B, E in the workspace and its size
+};
+
+BwdLayout bwd_layout(int64_t T, int64_t d, int64_t h, int n_m)
+{
+    BwdLayout L;
+    const size_t np = (size_t)n_m + 1;
+    L.g = 0;
+    L.b = L.g + round256((size_t)T * np * (size_t)h * 2);
+    L.e = L.b + round256(np * (size_t)h * (size_t)d * 2);
+    L.total = L.e + round256(np * (size_t)h * (size_t)d * 4);
+    return L;
+}
+
+template <int NM>
+int backward_nm(const void *x, int64_t T, int64_t d, const void *W, int64_t h, const uint8_t *packed, int act,
+                const void *dout, float *dx, float *dW, float *dM, uint8_t *ws, cudaStream_t s)
+{
+    const BwdLayout L = bwd_layout(T, d, h, NM);
+    __nv_bfloat16 *G = reinterpret_cast<__nv_bfloat16 *>(ws + L.g);
+    __nv_bfloat16 *B = reinterpret_cast<__nv_bfloat16 *>(ws + L.b);
+    float *E = reinterpret_cast<float *>(ws + L.e);
+    int rc;
+    // 1. a_i - c_i and sum_i c_i from the recomputed products (tcgen05)
+    if ((rc = launch_prefill<NM, true>(x, T, d, W, h, packed, act, nullptr, nullptr, s, nullptr, dout, G)))
+        return rc;
+    // 2. the masked operand [M_1.W; ...; M_n.W; W]
+    const int64_t chunks = h * (d / 8);
+    mglu::tr::masked_weights_kernel<NM><<<(unsigned)((chunks + 255) / 256), 256, 0, s>>>(
+        reinterpret_cast<const __nv_bfloat16 *>(W), packed, h, d, B);
+    if ((rc = check_launch("masked weights launch")))
+        return rc;
+    int dev = 0;
+    if ((rc = current_device(&dev)))
+        return rc;
+    Cublas *cb = nullptr;
+    if ((rc = cublas_for(dev, s, &cb)))
+        return rc;
+    const float one = 1.0f, zero = 0.0f;
+    const int K = (int)((NM + 1) * h);
+    // 3. dx [T][d] = G [T][K] B [K][d]   (column-major: dx^T = B^T-view * G-view)
+    if (cb->gemm(cb->handle[dev], CUBLAS_OP_N, CUBLAS_OP_N, (int)d, (int)T, K, &one, B, CUDA_R_16BF, (int)d, G,
+                 CUDA_R_16BF, K, &zero, dx, CUDA_R_32F, (int)d, CUBLAS_COMPUTE_32F, CUBLAS_GEMM_DEFAULT) !=
+        CUBLAS_STATUS_SUCCESS) {
+        snprintf(g_last_cuda_error, sizeof(g_last_cuda_error), "cublasGemmEx (dx) failed");
+        return MGLU_ERR_CUDA;
+    }
+    // 4. E_i [h][d] = G_i^T x for the NM + 1 column blocks G_i of G
+    if (cb->gemm_batched(cb->handle[dev], CUBLAS_OP_N, CUBLAS_OP_T, (int)d, (int)h, (int)T, &one, x, CUDA_R_16BF,
+                         (int)d, 0, G, CUDA_R_16BF, K, (long long)h, &zero, E, CUDA_R_32F, (int)d,
+                         (long long)(h * d), NM + 1, CUBLAS_COMPUTE_32F, CUBLAS_GEMM_DEFAULT) != CUBLAS_STATUS_SUCCESS) {
+        snprintf(g_last_cuda_error, sizeof(g_last_cuda_error), "cublasGemmStridedBatchedEx (E) failed");
+        return MGLU_ERR_CUDA;
+    }
+    // 5. dW = sum_i M_i . E_i + E_NM, dM_i = W . E_i
+    const int64_t quads = h * d / 4;
+    mglu::tr::combine_kernel<NM><<<(unsigned)((quads + 255) / 256), 256, 0, s>>>(
+        E, reinterpret_cast<const __nv_bfloat16 *>(W), packed, h, d, dW, dM);
+    return check_launch("combine launch");
+}
+
 }  // namespace
 
 extern "C" {
+
+size_t mglu_backward_workspace_bytes(int64_t T, int64_t d, int64_t h, int n_m)
+{
+    if (T <= 0 || d <= 0 || h <= 0 || !nm_supported(n_m))
+        return 0;
+    return bwd_layout(T, d, h, n_m).total;
+}
+
+int mglu_backward(const void *x, int64_t T, int64_t d, const void *W, int64_t h, const uint8_t *packed, int n_m,
+                  int act, const void *dout, float *dx, float *dW, float *dlogits, void *workspace,
+                  size_t workspace_bytes, void *stream)
+{
+    int rc = check_forward(x, T, d, W, h, packed, n_m, act, MGLU_BF16, dout);
+    if (rc)
+        return rc;
+    if (act & MGLU_GATE_DENSE)
+        return MGLU_ERR_UNSUPPORTED;  // the backward covers the method's own gate
+    if (T == 0)
+        return MGLU_OK;
+    if (!dx || !dW || !workspace)
+        return MGLU_ERR_INVALID;
+    if (!aligned(dx, 16) || !aligned(dW, 16) || (dlogits && !aligned(dlogits, 16)) || !aligned(workspace, 256))
+        return MGLU_ERR_ALIGN;
+    if (workspace_bytes < mglu_backward_workspace_bytes(T, d, h, n_m))
+        return MGLU_ERR_INVALID;
+    if (T > INT32_MAX / 8 || (n_m + 1) * h >= INT32_MAX || d >= INT32_MAX)
+        return MGLU_ERR_INVALID;  // cuBLAS takes int dimensions
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    uint8_t *ws = reinterpret_cast<uint8_t *>(workspace);
+    switch (n_m) {
+    case 1: return backward_nm<1>(x, T, d, W, h, packed, act, dout, dx, dW, dlogits, ws, s);
+    case 2: return backward_nm<2>(x, T, d, W, h, packed, act, dout, dx, dW, dlogits, ws, s);
+    case 4: return backward_nm<4>(x, T, d, W, h, packed, act, dout, dx, dW, dlogits, ws, s);
+    default: return backward_nm<8>(x, T, d, W, h, packed, act, dout, dx, dW, dlogits, ws, s);
+    }
+}
 
 size_t mglu_packed_bytes(int n_m, int64_t d, int64_t h)
 {

@@ -98,6 +98,79 @@ __device__ __forceinline__ void build_variants(uint8_t *B, int off, uint4 w, uin
     }
 }
 
+// Store 8 floats as bf16 at p[0..8) (n valid; 16-byte store when all 8 are
+// valid and p is 16-byte aligned).
+__device__ __forceinline__ void store8_bf16(__nv_bfloat16 *p, const float (&v)[8], int n, bool vec)
+{
+    if (vec && n == 8) {
+        uint4 pk;
+        __nv_bfloat162 p0 = __floats2bfloat162_rn(v[0], v[1]);
+        __nv_bfloat162 p1 = __floats2bfloat162_rn(v[2], v[3]);
+        __nv_bfloat162 p2 = __floats2bfloat162_rn(v[4], v[5]);
+        __nv_bfloat162 p3 = __floats2bfloat162_rn(v[6], v[7]);
+        pk.x = *reinterpret_cast<uint32_t *>(&p0);
+        pk.y = *reinterpret_cast<uint32_t *>(&p1);
+        pk.z = *reinterpret_cast<uint32_t *>(&p2);
+        pk.w = *reinterpret_cast<uint32_t *>(&p3);
+        *reinterpret_cast<uint4 *>(p) = pk;
+    } else {
+#pragma unroll
+        for (int e = 0; e < 8; ++e)
+            if (e < n)
+                p[e] = __float2bfloat16_rn(v[e]);
+    }
+}
+
+// The training path's epilogue for one token (one TMEM lane) of a tile: for
+// every column j of the tile, with D = x W and g_i from the accumulators,
+// v_i = D - g_i:
+//   block i < NM of gout:  dout (act'(g_i) v_i - act(g_i))
+//   block NM of gout:      sum_i dout act(g_i)
+// One mask at a time, 8 columns at a time, to keep registers low.
+template <int NM>
+__device__ __forceinline__ void grad_epilogue(uint32_t tbase, int tok, int T, int rows, int n0, int act,
+                                              const __nv_bfloat16 *__restrict__ dout, __nv_bfloat16 *__restrict__ gout)
+{
+    using C = Cfg<NM>;
+    const int a = act & ACT_MASK;
+    const int64_t gstride = (int64_t)(NM + 1) * rows;
+    for (int jc = 0; jc < C::NJ; jc += 8) {
+        const int j = n0 + jc;
+        const int nv = tok < T ? (rows - j < 8 ? (rows - j > 0 ? rows - j : 0) : 8) : 0;
+        const bool vec = (rows & 7) == 0;
+        uint32_t dv[8];
+        tmem_ld_x8(tbase + jc, dv);
+        float go[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e)
+            go[e] = e < nv ? __bfloat162float(dout[(int64_t)tok * rows + j + e]) : 0.0f;
+        tmem_wait_ld();
+        float cs[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e)
+            cs[e] = 0.0f;
+#pragma unroll 1
+        for (int i = 0; i < NM; ++i) {
+            uint32_t gv[8];
+            tmem_ld_x8(tbase + (1 + i) * C::NJ + jc, gv);
+            tmem_wait_ld();
+            float ai[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                const float g = __uint_as_float(gv[e]);
+                const float v = __uint_as_float(dv[e]) - g;
+                const float av = act_fn(a, g);
+                ai[e] = go[e] * (act_grad_fn(a, g) * v - av);
+                cs[e] += go[e] * av;
+            }
+            if (nv > 0)
+                store8_bf16(gout + (int64_t)tok * gstride + (int64_t)i * rows + j, ai, nv, vec);
+        }
+        if (nv > 0)
+            store8_bf16(gout + (int64_t)tok * gstride + (int64_t)NM * rows + j, cs, nv, vec);
+    }
+}
+
 // Mask bits of an 8-weight chunk read straight from global memory (NM bytes
 // at byte offset (row * d + k) * NM / 8; zero outside the matrix).
 template <int NM>
@@ -123,14 +196,23 @@ __device__ __forceinline__ uint2 load_mask_global(const uint8_t *packed, int row
 // then read each chunk's mask bits from global memory (issued before they
 // wait for the W tile, so the two latencies overlap) instead of a staged
 // mask tile.
-template <int NM>
+//
+// GRAD: the epilogue of the training path instead of the forward's.  With
+// the loss gradient dout [T][rows] it writes, for every token b and column
+// j, the n_m + 1 coefficients of the backward's products into
+// gout [T][(NM + 1) * rows]: block i < NM holds dout * (act'(g_i) v_i -
+// act(g_i)) (the gradient of g_i minus that of v_i), block NM holds
+// sum_i dout * act(g_i) (the gradient of every v_i); rounded to bf16.
+template <int NM, bool GRAD = false>
 __global__ void __launch_bounds__(Cfg<NM>::NTHREADS, 1) prefill_kernel(const __grid_constant__ CUtensorMap tm_x,
                                                               const __grid_constant__ CUtensorMap tm_w,
                                                               const __grid_constant__ CUtensorMap tm_m, int T,
                                                               int rows, int d, int act,
                                                               __nv_bfloat16 *__restrict__ out,
                                                               const uint8_t *__restrict__ packed, int mask_direct,
-                                                              const float *__restrict__ mw)
+                                                              const float *__restrict__ mw,
+                                                              const __nv_bfloat16 *__restrict__ dout,
+                                                              __nv_bfloat16 *__restrict__ gout)
 {
     using C = Cfg<NM>;
     extern __shared__ uint8_t smem_raw[];
@@ -339,6 +421,9 @@ __global__ void __launch_bounds__(Cfg<NM>::NTHREADS, 1) prefill_kernel(const __g
             for (int i = 0; i < (NM > 0 ? NM : 1); ++i)
                 wt[i] = mw && tok < T ? mw[(int64_t)tok * NM + i] : 1.0f;
             const uint32_t tbase = tmem_base + ((uint32_t)(32 * q) << 16) + (uint32_t)(b * ACC_STRIDE);
+            if constexpr (GRAD && NM > 0) {
+                grad_epilogue<NM>(tbase, tok, T, rows, n0, act, dout, gout);
+            } else {
             __nv_bfloat16 *orow = out + (int64_t)tok * rows;
             for (int jc = 0; jc < C::NJ; jc += C::EC) {
                 float o[C::EC];
@@ -399,6 +484,7 @@ __global__ void __launch_bounds__(Cfg<NM>::NTHREADS, 1) prefill_kernel(const __g
                                 orow[j + e] = __float2bfloat16_rn(o[e]);
                     }
                 }
+            }
             }
             tc_fence_before();
             __syncwarp();

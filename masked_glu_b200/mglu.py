@@ -65,6 +65,8 @@ def lib() -> ctypes.CDLL:
             "mglu_forward_down": (I32, [P, I64, I64, P, I64, P, I32, I32, I32, P, P, SZ, P, P]),
             "mglu_forward_decode_static": (I32, [P, I64, I64, P, I64, P, I32, I32, P, P]),
             "mglu_host_workspace_bytes": (SZ, [I64, I64, I64, I32, I32, I32]),
+            "mglu_backward_workspace_bytes": (SZ, [I64, I64, I64, I32]),
+            "mglu_backward": (I32, [P, I64, I64, P, I64, P, I32, I32, P, P, P, P, P, SZ, P]),
             "mglu_forward_host": (I32, [P, I64, I64, P, I64, P, I32, I32, I32, P, P, SZ, P, P]),
             "mglu_forward_path": (I32, [I64, I32]),
             "mglu_set_decode_max_tokens": (I32, [I32]),
@@ -313,6 +315,26 @@ def forward_host(x_host: torch.Tensor, W: torch.Tensor, packed: torch.Tensor, n_
                                    _ptr(W_down), _ptr(workspace), _nbytes(workspace), _hptr(out_host),
                                    _stream(stream)), "mglu_forward_host")
     return out_host
+
+
+def backward(x: torch.Tensor, W: torch.Tensor, packed: torch.Tensor, n_m: int, dout: torch.Tensor, act="swish",
+             with_logits: bool = True, workspace: Optional[torch.Tensor] = None, stream=None):
+    """Gradients (dx [T][d], dW [h][d], dlogits [n_m][h][d] or None) of L
+    through out = MGLU(x) for dout = dL/dout [T][h], float32."""
+    T, d = x.shape
+    h = W.shape[0]
+    if dout.shape != (T, h) or dout.dtype != x.dtype:
+        raise ValueError("dout must be [T][h] with x's dtype")
+    dx = torch.empty((T, d), dtype=torch.float32, device=x.device)
+    dW = torch.empty((h, d), dtype=torch.float32, device=x.device)
+    dM = torch.empty((n_m, h, d), dtype=torch.float32, device=x.device) if with_logits else None
+    need = int(lib().mglu_backward_workspace_bytes(T, d, h, n_m))
+    if workspace is None:
+        workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=x.device)
+    _check(lib().mglu_backward(_ptr(x), T, d, _ptr(W), h, _ptr(packed), n_m, _act(act), _ptr(dout), _ptr(dx),
+                               _ptr(dW), _ptr(dM), _ptr(workspace), _nbytes(workspace), _stream(stream)),
+           "mglu_backward")
+    return dx, dW, dM
 
 
 def forward_path(T: int, dtype=torch.bfloat16) -> int:

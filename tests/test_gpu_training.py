@@ -51,3 +51,59 @@ def test_forward_from_logits_equals_forward_from_masks():
     a = mglu.forward(x, W, from_logits, n_m, "swish")
     b = mglu.forward(x, W, packed, n_m, "swish")
     assert torch.equal(a, b)
+
+
+# ------------------------------------------------------------------ backward (straight-through)
+def _grad_bound_check(got, ref, what):
+    """|err| <= 1e-2 rms(ref) elementwise: the backward's coefficients are
+    rounded to bf16 once (relative 2^-9) before fp32 products."""
+    got = np.asarray(got, dtype=np.float64)
+    rms = float(np.sqrt(np.mean(ref * ref)))
+    err = np.abs(got - ref)
+    k = int(np.argmax(err))
+    assert np.all(err <= 1e-2 * rms), f"{what}: |err| {err.flat[k]:.3e} > {1e-2 * rms:.3e} (ref {ref.flat[k]:.3e})"
+
+
+@pytest.mark.parametrize("n_m,T,d,h", [(4, 40, 256, 96), (8, 17, 128, 48), (2, 129, 200, 100), (1, 64, 136, 72)])
+@pytest.mark.parametrize("act", ["swish", "gelu", "relu"])
+def test_backward_matches_oracle(n_m, T, d, h, act):
+    case = inputs.make_case(T, d, h, n_m, seed=2700 + n_m + T + d)
+    x, W, packed, _ = device_case(case)
+    rng = np.random.default_rng(2701 + T)
+    dout = inputs.normal(rng, (T, h), 1.0, "bf16")
+    dx, dW, dM = mglu.backward(x, W, packed, n_m, torch.from_numpy(dout.storage.view(np.int16)).view(torch.bfloat16)
+                               .cuda(), act)
+    assert mglu.last_device_status() == 0
+    a = {"swish": otrain.ACT_SWISH, "gelu": otrain.ACT_GELU, "relu": otrain.ACT_RELU}[act]
+    rdx, rdW, rdM = otrain.backward(case.x.values, case.W.values, case.masks, a, dout.values)
+    _grad_bound_check(dx.cpu().numpy(), rdx, f"dx {act}")
+    _grad_bound_check(dW.cpu().numpy(), rdW, f"dW {act}")
+    _grad_bound_check(dM.cpu().numpy(), rdM, f"dlogits {act}")
+
+
+def test_backward_full_size_sampled():
+    """The prefill-shaped layer (T = 4096, d = 2048, h = 8192, n_m = 4):
+    dx of sampled tokens and dW / dlogits of sampled rows of W."""
+    T, d, h, n_m = 4096, 2048, 8192, 4
+    case = inputs.make_case(T, d, h, n_m, seed=2800)
+    x, W, packed, _ = device_case(case)
+    rng = np.random.default_rng(2801)
+    dout = inputs.normal(rng, (T, h), 1.0, "bf16")
+    dx, dW, dM = mglu.backward(x, W, packed, n_m,
+                               torch.from_numpy(dout.storage.view(np.int16)).view(torch.bfloat16).cuda(), "swish")
+    toks = np.array([0, 1337, T - 1])
+    rows = np.array([0, 4097, h - 1])
+    rdx, rdW, rdM = otrain.backward_sampled(case.x.values, case.W.values, case.masks, otrain.ACT_SWISH, dout.values,
+                                            toks, rows)
+    _grad_bound_check(dx.cpu().numpy()[toks], rdx, "dx sampled")
+    _grad_bound_check(dW.cpu().numpy()[rows], rdW, "dW sampled")
+    _grad_bound_check(dM.cpu().numpy()[:, rows], rdM, "dlogits sampled")
+
+
+def test_backward_without_logit_gradients():
+    case = inputs.make_case(24, 128, 64, 4, seed=2900)
+    x, W, packed, _ = device_case(case)
+    dout = torch.randn(24, 64, device="cuda").to(torch.bfloat16)
+    dx1, dW1, dM1 = mglu.backward(x, W, packed, 4, dout, "gelu")
+    dx2, dW2, dM2 = mglu.backward(x, W, packed, 4, dout, "gelu", with_logits=False)
+    assert dM2 is None and torch.equal(dx1, dx2) and torch.equal(dW1, dW2)
