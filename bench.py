@@ -46,6 +46,7 @@ METRIC = "MGLU fwd HBM GB/s & tok/s (decode), TFLOP/s (prefill) vs B200 roofline
 DEFAULT_WORKLOAD = "decode_d4096_h14336_nm8"
 # the rest of the default run: (workload, tokens, act)
 SUITE = [
+    ("decode_d4096_h14336_nm8", 1, "swish", 2),  # each token routed to 2 of its 8 masks
     ("decode_d2048_h8192_nm4", 1, "swish"),
     ("prefill_T4096_d2048_h8192_nm4", 4096, "swish"),
     ("prefill_T4096_d2048_h8192_nm4", 4096, "gelu"),
@@ -85,7 +86,7 @@ def parse_args(argv=None):
     return args
 
 
-def workload_shape(name, tokens=None, act="swish", p=0.5):
+def workload_shape(name, tokens=None, act="swish", p=0.5, route_k=None):
     from masked_glu_b200 import inputs
     if name not in inputs.WORKLOADS:
         raise SystemExit(f"unknown workload {name}; choose from {list(inputs.WORKLOADS)}")
@@ -97,15 +98,19 @@ def workload_shape(name, tokens=None, act="swish", p=0.5):
                  "tiny" if name.startswith("tiny") else "decode")
     w["seed"] = inputs.WORKLOAD_SEEDS[name] + (w["T"] if tokens is not None else 0)
     w["name"], w["act"], w["p"] = name, act, p
+    w["route_k"] = route_k
     return w
 
 
 def config_of(w, world):
     """The workload's description, identical in the GPU arm and the
     reference arm."""
-    return {"workload": w["name"], "T": w["T"], "d": w["d"], "h": w["h"], "n_m": w["n_m"], "act": w["act"],
-            "p": w["p"] if w["kind"] == "ffn" else 0.5, "l2": L2_POLICY,
-            "parallelism": "replicas" if world > 1 else "single"}
+    c = {"workload": w["name"], "T": w["T"], "d": w["d"], "h": w["h"], "n_m": w["n_m"], "act": w["act"],
+         "p": w["p"] if w["kind"] == "ffn" else 0.5, "l2": L2_POLICY,
+         "parallelism": "replicas" if world > 1 else "single"}
+    if w.get("route_k") is not None:
+        c["route"] = f"top-{w['route_k']} of {w['n_m']} masks per token (hard weights), router in the step"
+    return c
 
 
 def algorithmic(w):
@@ -434,13 +439,23 @@ def measure(args, dist, w, dev, *, sample_clocks):
     out = torch.empty((T, h), dtype=tdt, device=dev)
     y = torch.empty((T, d), dtype=tdt, device=dev) if kind == "ffn" else None
     scratch = torch.zeros(mglu.scratch_bytes(max(d, h)), dtype=torch.uint8, device=dev)
+    routed = w.get("route_k") is not None
+    if routed:
+        g = torch.Generator(device="cpu").manual_seed(w["seed"] + 17)
+        Wr = (torch.randn(nm, d, generator=g) / math.sqrt(d)).to(tdt).to(dev)
+        mw = torch.empty((T, nm), dtype=torch.float32, device=dev)
+        msc = torch.empty((T, nm), dtype=torch.float32, device=dev)
 
     def step(i, ev=None):
         """One step on the current stream; ev = events bracketing its kernels."""
         r = i % R
         if ev is not None:
             ev[0].record()
-        mglu.forward(x, Ws[r], pks[r], nm, w["act"], out=out, scratch=scratch)
+        if routed:
+            mglu.route_topk(x, Wr, w["route_k"], "hard", weights=mw, scores=msc)
+            mglu.forward_weighted(x, Ws[r], pks[r], nm, mw, w["act"], out=out, scratch=scratch)
+        else:
+            mglu.forward(x, Ws[r], pks[r], nm, w["act"], out=out, scratch=scratch)
         if ev is not None:
             ev[1].record()
         if kind == "ffn":
@@ -535,10 +550,14 @@ def measure(args, dist, w, dev, *, sample_clocks):
         mglu.forward_host(x_hs[q], Ws[r], pks[r], nm, w["act"], W_down=Wds[r] if kind == "ffn" else None,
                           out_host=res_hs[q], workspace=ws_hosts[q], stream=e2e_streams[q])
 
-    for i in range(args.warmup):
+    n_host = 50
+    if routed:
+        K_e2e = 0  # the host-buffer entry point has no routed form
+    else:
+        K_e2e = K
+    for i in range(args.warmup if K_e2e else 0):
         e2e_step(i)
     torch.cuda.synchronize(dev)
-    n_host = 50
     h0 = time.perf_counter()
     for i in range(n_host):
         mglu.forward(x, Ws[i % R], pks[i % R], nm, w["act"], out=out, scratch=scratch)
@@ -550,7 +569,7 @@ def measure(args, dist, w, dev, *, sample_clocks):
     e0.record(stream)
     for st in e2e_streams:
         st.wait_event(e0)
-    for i in range(K):
+    for i in range(K_e2e):
         e2e_step(i)
     for st in e2e_streams:
         done = torch.cuda.Event()
@@ -560,7 +579,7 @@ def measure(args, dist, w, dev, *, sample_clocks):
     torch.cuda.synchronize(dev)
     dist.barrier()
     e2e_ms = dist.max(e0.elapsed_time(e1), dev)
-    e2e_value = dist.world * T * K / (e2e_ms / 1000.0)
+    e2e_value = dist.world * T * K_e2e / (e2e_ms / 1000.0) if K_e2e else None
     status = status or mglu.last_device_status()
 
     peaks, peak_src = load_peaks()
@@ -587,9 +606,9 @@ def measure(args, dist, w, dev, *, sample_clocks):
         "value": value, "unit": "tok/s", "ms_per_step": ms_per_step, "dtype": w["dtype"],
         "config": config_of(w, dist.world),
         "roofline": roof,
-        "e2e": {"value": e2e_value, "unit": "tok/s", "h2d_bytes_per_step": x_hs[0].numel() * x_hs[0].element_size(),
-                "d2h_bytes_per_step": res_hs[0].numel() * res_hs[0].element_size()},
-        "gpu_launches": K * (2 if kind == "ffn" else 1),
+        "e2e": ({"value": e2e_value, "unit": "tok/s", "h2d_bytes_per_step": x_hs[0].numel() * x_hs[0].element_size(),
+                 "d2h_bytes_per_step": res_hs[0].numel() * res_hs[0].element_size()} if e2e_value else None),
+        "gpu_launches": K * (2 if kind == "ffn" or routed else 1),
         "host_us_per_forward_call": host_us,
         "device_status": status,
         "rotating_copies": R,
@@ -709,8 +728,10 @@ def run_mglu(args, dist):
 
     if args.suite:
         subs = []
-        for name, T, act in SUITE:
-            ws = workload_shape(name, T if name.startswith("ffn") else None, act, 0.5)
+        for entry in SUITE:
+            name, T, act = entry[:3]
+            ws = workload_shape(name, T if name.startswith("ffn") else None, act, 0.5,
+                                entry[3] if len(entry) > 3 else None)
             r, _ = measure(args, dist, ws, dev, sample_clocks=True)
             subs.append(r)
         line["workloads"] = subs
