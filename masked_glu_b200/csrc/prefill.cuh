@@ -56,6 +56,11 @@ struct Cfg {
     // 384 items, 12 warps, 966 TFLOP/s against 842 with 4 warps); the dense
     // kernel has nothing to build.
     static constexpr int NBW = NM == 0 ? 4 : NM == 8 ? 6 : NM == 4 ? 12 : NM == 2 ? 10 : 8;
+    // builder groups: group b builds the stages with it % BG == b, so each
+    // builder has BG stages' time to hide its loads, stores and fence
+    static constexpr int BG = 1;
+    static constexpr int GW = NBW / BG;  // builder warps per group
+    static_assert(NBW % BG == 0, "builder groups");
     // epilogue columns per TMEM load round (8 where the register budget of the
     // larger block is tight)
     static constexpr int EC = NM >= 4 ? 8 : 16;
@@ -240,7 +245,7 @@ __global__ void __launch_bounds__(Cfg<NM>::NTHREADS, 1) prefill_kernel(const __g
             mbar_init(&xfull[s], 1);
             mbar_init(&full[s], 1);
             mbar_init(&mfull[s], 1);
-            mbar_init(&built[s], C::NBW);
+            mbar_init(&built[s], C::GW);
             mbar_init(&empty[s], 1);
         }
         for (int b = 0; b < 2; ++b) {
@@ -351,21 +356,24 @@ __global__ void __launch_bounds__(Cfg<NM>::NTHREADS, 1) prefill_kernel(const __g
     } else if (warp < 2 + C::NBW) {
         // ---------------------------------------------------------- builders
         if constexpr (NM > 0) {
-            const int bt = threadIdx.x - 64;  // 0 .. 32 * NBW - 1
+            const int grp = (warp - 2) / C::GW;                   // builder group
+            const int bt = threadIdx.x - 64 - grp * 32 * C::GW;   // 0 .. 32 * GW - 1
             constexpr int ITEMS = C::NJ * 8;   // 16-byte pieces of a W tile
-            constexpr int MAXI = (ITEMS + 32 * C::NBW - 1) / (32 * C::NBW);
+            constexpr int MAXI = (ITEMS + 32 * C::GW - 1) / (32 * C::GW);
             int it = 0;
             bool ok = true;
             for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
                 const int n0 = (tile / num_m) * C::NJ;
                 for (int kb = 0; kb < nkb; ++kb, ++it) {
+                    if (C::BG > 1 && it % C::BG != grp)
+                        continue;
                     const int s = it % C::STAGES;
                     const uint32_t ph = (uint32_t)(it / C::STAGES) & 1u;
                     uint2 mg[MAXI];
                     if (mask_direct) {
 #pragma unroll
                         for (int q = 0; q < MAXI; ++q) {
-                            const int item = bt + q * 32 * C::NBW;
+                            const int item = bt + q * 32 * C::GW;
                             mg[q] = item < ITEMS ? load_mask_global<NM>(packed, n0 + (item >> 3), kb * BK + 8 * (item & 7),
                                                                         rows, d)
                                                  : make_uint2(0u, 0u);
@@ -381,7 +389,7 @@ __global__ void __launch_bounds__(Cfg<NM>::NTHREADS, 1) prefill_kernel(const __g
                     const int moff = (kb * BK * NM / 8) % C::MB;  // nonzero only when NM = 1
 #pragma unroll
                     for (int q = 0; q < MAXI; ++q) {
-                        const int item = bt + q * 32 * C::NBW;
+                        const int item = bt + q * 32 * C::GW;
                         if (item < ITEMS) {
                             const int r = item >> 3, c = item & 7;
                             const int off = r * 128 + ((c ^ (r & 7)) << 4);

@@ -121,6 +121,30 @@ __device__ __forceinline__ bool mbar_wait_warp3(uint64_t *a, uint64_t *b, uint64
     return ok != 0;
 }
 
+// ---------------------------------------------------------------- cp.async
+// Per-thread asynchronous copy global -> shared of cp bytes (4, 8 or 16), of
+// which the first src bytes are read and the rest zero-filled (src = 0
+// reads nothing).  .cg (16 bytes) bypasses L1, .ca caches in L1.  The copy's
+// data is visible to the issuing thread once cp.async.wait_group says its
+// group has completed.
+__device__ __forceinline__ void cp_async_cg16(uint32_t dst, const void *src, uint32_t src_bytes)
+{
+    asm volatile("cp.async.cg.shared.global.L2::256B [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes)
+                 : "memory");
+}
+
+template <int CP>
+__device__ __forceinline__ void cp_async_ca(uint32_t dst, const void *src, uint32_t src_bytes)
+{
+    asm volatile("cp.async.ca.shared.global [%0], [%1], %2, %3;" ::"r"(dst), "l"(src), "n"(CP), "r"(src_bytes)
+                 : "memory");
+}
+
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+
 // ---------------------------------------------------------------- dependent launch
 // Kernels are launched with programmatic stream serialization: the next
 // kernel on the stream may be scheduled once every CTA of this one has

@@ -5,15 +5,17 @@ of its warps' steps for small shapes.  The weight stream itself needs no
 model: every lane loads its own operands into its own registers.  What the
 warps share is the row-block hand-off through shared memory:
 
-* a CTA's work has F row-block parts (flushes).  At the end of part f every
-  warp writes its accumulators into slot set f mod 2;
-* from part 2 on, a warp first waits on FREE[f mod 2] (bar.sync) unless it
-  finished part f - 2 itself: that finisher arrived on FREE[f mod 2] once it
-  had read the set, and it does not wait there again;
+* a CTA's work has F row-block parts (flushes).  With S slot sets (1 or 2)
+  every warp writes its accumulators at the end of part f into set f mod S;
+* from part S on, every warp first waits on FREE[f mod S] (bar.sync); the
+  finisher of part f - S gets there only after it has read that set;
 * warp f mod NW finishes part f: after writing its own slot it waits on
-  FULL[f mod 2] (bar.sync), reads every slot of the set and, if part f + 2
-  exists, arrives on FREE[f mod 2]; the other warps arrive on FULL[f mod 2]
-  after writing and carry on.
+  FULL[f mod S] (bar.sync) and reads every slot of the set; the other warps
+  arrive on FULL[f mod S] after writing and carry on.
+
+(An earlier form, in which the finisher arrived on FREE and then skipped its
+own wait there, is kept as a planted mistake: with one slot set it lets a
+warp arrive on the next FREE generation before the current one completes.)
 
 Named barriers are modelled with hardware generations: an arrival counts
 toward the barrier's current generation, whichever part the arriving warp
@@ -29,22 +31,33 @@ Planted protocol mistakes must each be caught.
 import pytest
 
 
-def explore(nw, F, mutation=None):
-    """Depth-first search over all reachable states of nw warps and F parts.
-    Returns (violations found, states visited)."""
+def explore(nw, F, mutation=None, sets=2):
+    """Depth-first search over all reachable states of nw warps and F parts
+    with `sets` slot sets.  Returns (violations found, states visited)."""
+    S = sets
+    # "one_slot_set": the slots of a single set reused while waits assume two
+    reuse = 2 if mutation == "one_slot_set" else S
 
     def finisher(f):
         return f % nw
 
     def waits_free(w, f):
-        if f < 2:
+        if f < reuse:
             return False
         if mutation == "skip_free_wait":
             return False
-        return w != finisher(f - 2)
+        if mutation == "finisher_arrives_and_skips":
+            return w != finisher(f - reuse)
+        return True
 
     def slot_set(f):
-        return 0 if mutation == "one_slot_set" else f & 1
+        return 0 if mutation == "one_slot_set" else f % S
+
+    def gen_free(f):  # generation of FREE[f mod S] that part f waits on
+        return (f - reuse) // reuse if mutation != "one_slot_set" else f - reuse
+
+    def gen_full(f):
+        return f // S if mutation != "one_slot_set" else f
 
     # warp state: (f, pc, gen) with pc in
     #   "FW"  wait on FREE (arrive done), "WR" write slot, "FA" FULL step,
@@ -90,8 +103,7 @@ def explore(nw, F, mutation=None):
 
             s = slot_set(f)
             if pc == "FREE":  # bar.sync FREE[s]: arrive, then wait for the generation
-                nb, g = arrive(bars, 2 + s, (f - 2) // 2 if mutation != "one_slot_set" else f - 2,
-                               f"warp {w} FREE part {f}")
+                nb, g = arrive(bars, 2 + s, gen_free(f), f"warp {w} FREE part {f}")
                 put((f, "FW", g), bars_=nb)
             elif pc == "FW":
                 if bars[2 + s][0] > gen:
@@ -106,12 +118,12 @@ def explore(nw, F, mutation=None):
             elif pc == "FA":
                 fin = finisher(f)
                 if w == fin and mutation != "finisher_does_not_wait":
-                    nb, g = arrive(bars, s, f // 2 if mutation != "one_slot_set" else f, f"finisher {w} FULL {f}")
+                    nb, g = arrive(bars, s, gen_full(f), f"finisher {w} FULL {f}")
                     put((f, "FS", g), bars_=nb)
                 elif w == fin:
                     put((f, "RD", -1))
                 else:
-                    nb, _ = arrive(bars, s, f // 2 if mutation != "one_slot_set" else f, f"warp {w} FULL {f}")
+                    nb, _ = arrive(bars, s, gen_full(f), f"warp {w} FULL {f}")
                     nxt = f + 1
                     put((nxt, start_pc(w, nxt) if nxt < F else "DONE", -1), bars_=nb)
             elif pc == "FS":
@@ -123,9 +135,8 @@ def explore(nw, F, mutation=None):
                         errors.append(f"finisher of part {f} reads warp {ww}'s slot holding part {slots[s][ww]}")
                 nread = read | {f}
                 nb = bars
-                if f + 2 < F and mutation != "finisher_skips_free":
-                    nb, _ = arrive(bars, 2 + s, f // 2 if mutation != "one_slot_set" else f,
-                                   f"finisher {w} FREE after part {f}")
+                if mutation == "finisher_arrives_and_skips" and f + reuse < F:
+                    nb, _ = arrive(bars, 2 + s, f // reuse, f"finisher {w} FREE after part {f}")
                 nxt = f + 1
                 put((nxt, start_pc(w, nxt) if nxt < F else "DONE", -1), bars_=nb, read_=nread)
         if not succ:
@@ -136,16 +147,27 @@ def explore(nw, F, mutation=None):
 
 
 # ---------------------------------------------------------------- the shipped protocol is safe
+@pytest.mark.parametrize("sets", [1, 2])
 @pytest.mark.parametrize("nw,F", [(2, 1), (2, 3), (2, 6), (3, 4), (3, 7), (4, 5), (4, 6)])
-def test_protocol_has_no_race_or_deadlock(nw, F):
-    errors, states = explore(nw, F)
+def test_protocol_has_no_race_or_deadlock(nw, F, sets):
+    errors, states = explore(nw, F, sets=sets)
     assert errors == [], errors[:3]
     assert states > 10
 
 
 # ---------------------------------------------------------------- each planted mistake is caught
-@pytest.mark.parametrize("mutation", ["skip_free_wait", "finisher_skips_free", "finisher_does_not_wait",
-                                      "one_slot_set"])
-def test_planted_protocol_mistakes_are_caught(mutation):
-    errors, _ = explore(3, 5, mutation)
+@pytest.mark.parametrize("sets", [1, 2])
+@pytest.mark.parametrize("mutation", ["skip_free_wait", "finisher_does_not_wait"])
+def test_planted_protocol_mistakes_are_caught(mutation, sets):
+    errors, _ = explore(3, 5, mutation, sets=sets)
     assert errors, f"mutation {mutation} was not caught"
+
+
+def test_one_set_reused_as_if_two_is_caught():
+    errors, _ = explore(3, 5, "one_slot_set")
+    assert errors
+
+
+def test_finisher_that_arrives_and_skips_its_wait_races_with_one_set():
+    errors, _ = explore(2, 3, "finisher_arrives_and_skips", sets=1)
+    assert any("overwrites" in e or "generation" in e for e in errors)
