@@ -751,18 +751,18 @@ int mglu_route_topk(const void *x, int64_t T, int64_t d, const void *W_r, int n_
     const uintptr_t es = dtype == MGLU_BF16 ? 2 : 4;
     if (!aligned(x, es) || !aligned(W_r, es) || !aligned(weights, 4) || (scores && !aligned(scores, 4)))
         return MGLU_ERR_ALIGN;
-    const int64_t blocks = (T + 7) / 8;
-    if (blocks > 0x7FFFFFFF)
+    if (T > 0x7FFFFFFF)
         return MGLU_ERR_INVALID;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    const int vec = d % 8 == 0 && aligned(x, 16) && aligned(W_r, 16);
     if (dtype == MGLU_BF16)
-        mglu::route_kernel<__nv_bfloat16><<<(unsigned)blocks, 256, 0, s>>>(
+        mglu::route_kernel<__nv_bfloat16><<<(unsigned)T, 256, 0, s>>>(
             reinterpret_cast<const __nv_bfloat16 *>(x), T, d, reinterpret_cast<const __nv_bfloat16 *>(W_r), n_m, k,
-            mode, weights, scores);
+            mode, vec, weights, scores);
     else
-        mglu::route_kernel<float><<<(unsigned)blocks, 256, 0, s>>>(reinterpret_cast<const float *>(x), T, d,
-                                                                    reinterpret_cast<const float *>(W_r), n_m, k,
-                                                                    mode, weights, scores);
+        mglu::route_kernel<float><<<(unsigned)T, 256, 0, s>>>(reinterpret_cast<const float *>(x), T, d,
+                                                               reinterpret_cast<const float *>(W_r), n_m, k, mode, 0,
+                                                               weights, scores);
     return check_launch("route launch");
 }
 
