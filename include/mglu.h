@@ -192,6 +192,26 @@ int mglu_forward_weighted(const void *x, int64_t T, int64_t d, const void *W,
                           void *scratch, size_t scratch_bytes, void *stream);
 
 /*
+ * The partial sums behind mglu_forward's output, for checking the
+ * decomposition ("Masked Gated Linear Unit", "Approach": each mask splits W
+ * into a gate part M_i . W and a value part (1 - M_i) . W):
+ *   D[b,j]   = sum_k x[b,k] W[j,k]
+ *   g_i[b,j] = sum_k x[b,k] M_i[j,k] W[j,k]
+ *   v_i[b,j] = sum_k x[b,k] (1 - M_i[j,k]) W[j,k]
+ * computed by the decode kernel (fp32 accumulation, as mglu_forward) and
+ * written unrounded as float32 planes partials[2*n_m + 1][T][h]: plane 0 is
+ * D, plane 1 + 2i is g_i, plane 2 + 2i is v_i.  g_i + v_i equals D up to
+ * float32 rounding.
+ *   Arguments as mglu_forward with dtype MGLU_BF16 (alignment, d % 8);
+ *   partials: device, 16-byte aligned.  T must be in 0..16 (the decode
+ *   kernel), else MGLU_ERR_UNSUPPORTED.  scratch as for mglu_forward.
+ */
+int mglu_forward_partials(const void *x, int64_t T, int64_t d, const void *W,
+                          int64_t h, const uint8_t *packed, int n_m,
+                          float *partials, void *scratch, size_t scratch_bytes,
+                          void *stream);
+
+/*
  * The FFN down-projection alone, a dense product (MGLU replaces only the two
  * GLU projections; "Masked Gated Linear Unit", "Problem"):
  *   y[b,c] = sum_j hid[b,j] * W_down[c,j]

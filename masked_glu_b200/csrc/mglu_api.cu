@@ -209,17 +209,17 @@ int launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, int smem, cudaSt
 }
 
 // ------------------------------------------------------------------ decode
-template <int NM, int NT, bool ROUTED>
+template <int NM, int TT, bool ROUTED>
 int launch_decode(const void *x, int64_t T, int64_t d, const void *W, int64_t rows, const uint8_t *packed, int act,
-                  void *out, void *ws, cudaStream_t s, const float *mw)
+                  void *out, void *ws, cudaStream_t s, const float *mw, float *gv)
 {
-    using L = mglu::dec::Layout<NM, NT>;
+    using L = mglu::dec::Layout<NM, TT>;
     if (d >= ((int64_t)1 << 22) || rows >= ((int64_t)1 << 27))
         return MGLU_ERR_INVALID;  // the kernel's 32-bit schedule arithmetic
     int dev = 0, rc = current_device(&dev);
     if (rc)
         return rc;
-    if ((rc = ensure_smem<mglu::dec::decode_kernel<NM, NT, ROUTED>>(L::SMEM, dev)))
+    if ((rc = ensure_smem<mglu::dec::decode_kernel<NM, TT, ROUTED>>(L::SMEM, dev)))
         return rc;
     const int64_t rb = (rows + mglu::dec::ROWS - 1) / mglu::dec::ROWS;
     const int64_t units = rb * ((d + L::KS - 1) / L::KS);
@@ -230,23 +230,34 @@ int launch_decode(const void *x, int64_t T, int64_t d, const void *W, int64_t ro
         grid = units;
     float *ws_part = reinterpret_cast<float *>(ws);
     int *ws_count = reinterpret_cast<int *>(reinterpret_cast<uint8_t *>(ws) + mglu::dec::part_bytes());
-    return launch_pdl(mglu::dec::decode_kernel<NM, NT, ROUTED>, dim3((unsigned)grid), dim3(L::NTHREADS), L::SMEM, s,
+    return launch_pdl(mglu::dec::decode_kernel<NM, TT, ROUTED>, dim3((unsigned)grid), dim3(L::NTHREADS), L::SMEM, s,
                       "decode launch", reinterpret_cast<const __nv_bfloat16 *>(x),
                       reinterpret_cast<const __nv_bfloat16 *>(W), packed, (int)T, (int)rows, (int)d, act, ws_part,
-                      ws_count, reinterpret_cast<__nv_bfloat16 *>(out), mw);
+                      ws_count, reinterpret_cast<__nv_bfloat16 *>(out), mw, gv);
+}
+
+// Token capacity by T: 2, 8 or 16 (the slots and the finisher's work follow
+// the call's T; the capacity fixes the MMA column blocks and shared memory).
+template <int NM, bool ROUTED>
+int decode_tt(const void *x, int64_t T, int64_t d, const void *W, int64_t rows, const uint8_t *packed, int act,
+              void *out, void *ws, cudaStream_t s, const float *mw, float *gv)
+{
+    if (T <= 2)
+        return launch_decode<NM, 2, ROUTED>(x, T, d, W, rows, packed, act, out, ws, s, mw, gv);
+    if (T <= 8)
+        return launch_decode<NM, 8, ROUTED>(x, T, d, W, rows, packed, act, out, ws, s, mw, gv);
+    return launch_decode<NM, 16, ROUTED>(x, T, d, W, rows, packed, act, out, ws, s, mw, gv);
 }
 
 template <int NM>
 int decode_nt(const void *x, int64_t T, int64_t d, const void *W, int64_t rows, const uint8_t *packed, int act,
-              void *out, void *ws, cudaStream_t s, const float *mw)
+              void *out, void *ws, cudaStream_t s, const float *mw, float *gv = nullptr)
 {
     if constexpr (NM > 0) {
         if (mw)
-            return T <= 8 ? launch_decode<NM, 1, true>(x, T, d, W, rows, packed, act, out, ws, s, mw)
-                          : launch_decode<NM, 2, true>(x, T, d, W, rows, packed, act, out, ws, s, mw);
+            return decode_tt<NM, true>(x, T, d, W, rows, packed, act, out, ws, s, mw, gv);
     }
-    return T <= 8 ? launch_decode<NM, 1, false>(x, T, d, W, rows, packed, act, out, ws, s, nullptr)
-                  : launch_decode<NM, 2, false>(x, T, d, W, rows, packed, act, out, ws, s, nullptr);
+    return decode_tt<NM, false>(x, T, d, W, rows, packed, act, out, ws, s, nullptr, gv);
 }
 
 // ------------------------------------------------------------------ prefill
@@ -715,6 +726,32 @@ int mglu_forward(const void *x, int64_t T, int64_t d, const void *W, int64_t h, 
     if ((rc = check_scratch(T, dtype, h, scratch, scratch_bytes_)))
         return rc;
     return run_product(x, T, d, W, h, packed, n_m, act, dtype, out, scratch, reinterpret_cast<cudaStream_t>(stream));
+}
+
+int mglu_forward_partials(const void *x, int64_t T, int64_t d, const void *W, int64_t h, const uint8_t *packed,
+                          int n_m, float *partials, void *scratch, size_t scratch_bytes_, void *stream)
+{
+    // n_m = 0 (the dense product alone) is allowed here; packed is then not read
+    int rc = check_forward(x, T, d, W, h, packed, n_m == 0 ? 1 : n_m, MGLU_ACT_SWISH, MGLU_BF16, partials);
+    if (rc)
+        return rc;
+    if (T > 16)
+        return MGLU_ERR_UNSUPPORTED;
+    if (T == 0)
+        return MGLU_OK;
+    if (!scratch || scratch_bytes_ < scratch_bytes(h))
+        return MGLU_ERR_INVALID;
+    if (!aligned(scratch, 16))
+        return MGLU_ERR_ALIGN;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    switch (n_m) {
+    case 0: return decode_nt<0>(x, T, d, W, h, packed, 0, nullptr, scratch, s, nullptr, partials);
+    case 1: return decode_nt<1>(x, T, d, W, h, packed, 0, nullptr, scratch, s, nullptr, partials);
+    case 2: return decode_nt<2>(x, T, d, W, h, packed, 0, nullptr, scratch, s, nullptr, partials);
+    case 4: return decode_nt<4>(x, T, d, W, h, packed, 0, nullptr, scratch, s, nullptr, partials);
+    case 8: return decode_nt<8>(x, T, d, W, h, packed, 0, nullptr, scratch, s, nullptr, partials);
+    default: return MGLU_ERR_UNSUPPORTED;
+    }
 }
 
 int mglu_forward_weighted(const void *x, int64_t T, int64_t d, const void *W, int64_t h, const uint8_t *packed,

@@ -140,6 +140,18 @@ __device__ __forceinline__ void cp_async_ca(uint32_t dst, const void *src, uint3
                  : "memory");
 }
 
+// The same copies with every byte read.
+__device__ __forceinline__ void cp_async_cg16(uint32_t dst, const void *src)
+{
+    asm volatile("cp.async.cg.shared.global.L2::256B [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+
+template <int CP>
+__device__ __forceinline__ void cp_async_ca(uint32_t dst, const void *src)
+{
+    asm volatile("cp.async.ca.shared.global [%0], [%1], %2;" ::"r"(dst), "l"(src), "n"(CP) : "memory");
+}
+
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 
 template <int N>

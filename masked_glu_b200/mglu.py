@@ -61,6 +61,7 @@ def lib() -> ctypes.CDLL:
             "mglu_down_proj": (I32, [P, I64, I64, P, I64, I32, P, P, SZ, P]),
             "mglu_route_topk": (I32, [P, I64, I64, P, I32, I32, I32, I32, P, P, P]),
             "mglu_forward_weighted": (I32, [P, I64, I64, P, I64, P, I32, I32, I32, P, P, P, SZ, P]),
+            "mglu_forward_partials": (I32, [P, I64, I64, P, I64, P, I32, P, P, SZ, P]),
             "mglu_workspace_bytes": (SZ, [I64, I64, I64, I32, I32]),
             "mglu_forward_down": (I32, [P, I64, I64, P, I64, P, I32, I32, I32, P, P, SZ, P, P]),
             "mglu_forward_decode_static": (I32, [P, I64, I64, P, I64, P, I32, I32, P, P]),
@@ -238,6 +239,22 @@ def forward_weighted(x: torch.Tensor, W: torch.Tensor, packed: torch.Tensor, n_m
     _check(lib().mglu_forward_weighted(_ptr(x), T, d, _ptr(W), h, _ptr(packed), n_m, _act(act), _dtype(x),
                                        _ptr(mask_weights), _ptr(out), _ptr(scratch), _nbytes(scratch),
                                        _stream(stream)), "mglu_forward_weighted")
+    return out
+
+
+def forward_partials(x: torch.Tensor, W: torch.Tensor, packed: torch.Tensor, n_m: int,
+                     scratch: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """The decode kernel's unrounded partial sums, float32 [2 n_m + 1][T][h]:
+    plane 0 = D = x W^T, plane 1 + 2i = g_i, plane 2 + 2i = v_i (bf16, T <= 16)."""
+    T, d = x.shape
+    h = W.shape[0]
+    if W.shape[1] != d or W.dtype != x.dtype:
+        raise ValueError("W must be [h][d] with x's dtype")
+    out = torch.empty((2 * n_m + 1, T, h), dtype=torch.float32, device=x.device)
+    if scratch is None:
+        scratch = default_scratch(h, x.device)
+    _check(lib().mglu_forward_partials(_ptr(x), T, d, _ptr(W), h, _ptr(packed), n_m, _ptr(out), _ptr(scratch),
+                                       _nbytes(scratch), _stream(stream)), "mglu_forward_partials")
     return out
 
 
