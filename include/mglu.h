@@ -123,12 +123,12 @@ int mglu_unpack_masks(const uint8_t *packed, int n_m, int64_t d, int64_t h,
 
 /*
  * Bytes of scratch the decode kernel needs for a product with `rows` output
- * rows (h for mglu_forward, d for mglu_down_proj): partial sums of the row
- * blocks that two CTAs share, plus one arrival counter per 16 rows (about
- * 6 MB).  The scratch must be 16-byte aligned and ZERO-FILLED before its
- * first use (e.g. one cudaMemset); every call that returns leaves it zeroed
- * again.  Calls that may run concurrently (other streams) need separate
- * scratch buffers.  Only the decode path touches it: when
+ * rows (h for mglu_forward, d for mglu_down_proj): the partial sums of the
+ * row blocks that several CTAs share, two slots per CTA of the grid (about
+ * 6 MB, the same for every `rows`).  The scratch must be 16-byte aligned; its
+ * contents need no initialization (every slot is written before it is read
+ * within a call).  Calls that may run concurrently (other streams) need
+ * separate scratch buffers.  Only the decode path touches it: when
  * mglu_forward_path(T, dtype) is not MGLU_PATH_DECODE it may be NULL.
  */
 size_t mglu_scratch_bytes(int64_t rows);
@@ -226,9 +226,7 @@ int mglu_down_proj(const void *hid, int64_t T, int64_t h, const void *W_down,
  * max(d, h) rows (mglu_scratch_bytes) at the START of the workspace, then the
  * hidden activation [T][h] in the path's dtype (rounded up to 256 bytes).
  * The scratch's place does not depend on T, so one workspace serves calls of
- * any token count on the same layer shape.  Zero-fill it before its first
- * use, as for scratch; zero-fill it again before using it for a layer with a
- * larger max(d, h), whose scratch reaches into bytes that held activations. */
+ * any token count; like the scratch, it needs no initialization. */
 size_t mglu_workspace_bytes(int64_t T, int64_t d, int64_t h, int n_m, int dtype);
 
 /*
@@ -245,8 +243,7 @@ int mglu_forward_down(const void *x, int64_t T, int64_t d, const void *W,
                       int dtype, const void *W_down, void *workspace,
                       size_t workspace_bytes, void *y, void *stream);
 
-/* Most output rows mglu_forward_decode_static accepts (its built-in scratch
- * holds one counter per 16 of them). */
+/* Most output rows mglu_forward_decode_static accepts. */
 #define MGLU_STATIC_SCRATCH_MAX_ROWS 262144
 
 /*
@@ -273,8 +270,6 @@ int mglu_forward_down(const void *x, int64_t T, int64_t d, const void *W,
  * The first call on each device does the set-up: it looks up the array's
  * device address (cudaGetSymbolAddress, return code checked) and clears the
  * scratch on `stream`.  Make that first call before any stream capture.
- * Every call also clears the arrival counters of its row blocks on `stream`
- * before the kernel starts, since those must start at zero.
  *
  * There is one such scratch per device, so calls that may overlap in time
  * (other streams, other host threads) race on it and give wrong results.
@@ -304,8 +299,8 @@ size_t mglu_host_workspace_bytes(int64_t T, int64_t d, int64_t h, int n_m,
  * reaches the end of the call (synchronize before reading it).  Pinned host
  * memory (cudaHostAlloc) makes both copies asynchronous; pageable memory
  * works but the copies then block the calling thread.
- *   workspace: device, 256-byte aligned, >= mglu_host_workspace_bytes(...),
- *   zero-filled before its first use (it holds the decode scratch).
+ *   workspace: device, 256-byte aligned, >= mglu_host_workspace_bytes(...)
+ *   (it holds the decode scratch; no initialization needed).
  * Nothing is allocated.  Errors: as mglu_forward / mglu_forward_down, plus
  * INVALID for a missing or small workspace or a NULL host pointer.
  */

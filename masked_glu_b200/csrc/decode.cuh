@@ -5,43 +5,37 @@
 // decoding is bound by reading the weights, so each weight and its mask bits
 // are read exactly once and the masks are unpacked inside the kernel):
 //
-//  * Work is made of stages (row block of ROWS = 16 rows of W, k-stage of
-//    KS = 64 * NW k: two 32-k units per warp).  A persistent grid of
-//    one CTA per SM splits the stages evenly: every CTA gets the same number
-//    of whole row blocks (data-parallel part) plus an equal contiguous share
-//    of the stages of the remaining row blocks (stream-K part), so all SMs
-//    stream the same number of bytes.  Each CTA does its stream-K share
-//    first, so the combining of row blocks split between CTAs overlaps the
-//    data-parallel part instead of trailing the kernel.
-//  * Each warp streams its own units of every stage through a private ring of
-//    P stages in shared memory: lane (g, c) copies (cp.async) 16 bytes of W
-//    rows g and g + 8 per unit (eight weights each) and their mask bits,
-//    P - 1 stages ahead of the one it multiplies, and reads back only what
-//    it copied itself; x (small, read by every CTA) comes from L1 one stage
-//    ahead.  The copies are tracked by
-//    cp.async groups, not registers, so the ring can be deep (about 100 KB in
-//    flight per SM); no staged operand passes from one thread to another, so
-//    the weight stream needs no barrier.
+//  * Work is made of units (row block of ROWS = 16 rows of W, step of
+//    STEP_K = 64 k: two 32-k MMA units).  A persistent grid of one CTA per
+//    SM gives every warp of the grid an equal contiguous range of units
+//    (warp-level stream-K, see sched.cuh), so all warps stream the same
+//    number of bytes and none ever waits for another while it streams.
+//  * Each warp streams its units through a private ring of P stages in
+//    shared memory: lane (g, c) copies (cp.async) 16 bytes of W rows g and
+//    g + 8 per MMA unit (eight weights each) and their mask bits, P - 1 units
+//    ahead of the one it multiplies, and reads back only what it copied
+//    itself; x (small, read by every CTA) comes from L1 at the top of each
+//    unit.  The copies are tracked by cp.async groups, not registers, so the
+//    ring can be deep; no staged operand passes from one thread to another,
+//    so the weight stream needs no barrier.
 //  * Masks are applied by sign flips (see group_bits / flip_pair): the warp
 //    accumulates the dense product D = x W and h_i = x (S_i . W) with
 //    S_i = +1 where mask i is set and -1 where it is clear, on mma.sync
 //    m16n8k16 with the 16 rows as M and the tokens as N; one LOP3 and one
 //    shift per bf16 pair and mask build the operand.  Then g_i = (D + h_i)/2
 //    and v_i = (D - h_i)/2 = D - g_i.
-//  * At the end of a row block's part in this CTA each warp drops its
-//    accumulators into a shared-memory slot (one or two slot sets, used in
-//    turn)
-//    and carries on, except the part's finisher: the warps take that role in
-//    turn (part f: warp f mod NW), wait for every slot of the part, add them
-//    in a fixed order and finish the part.  It releases the set as soon as
-//    it has read it.  A row block whose k range lies
-//    inside one CTA is finished there:
-//    out = sum_i act(g_i) v_i, rounded once to bf16.  A row block split
-//    between CTAs (only at the two ends of a stream-K share) is finished by
-//    whichever of its CTAs arrives last: the others' partial sums come from
-//    a small global scratch, added in CTA order, so the result does not
-//    depend on arrival order.  The arrival counter is reset by the finishing
-//    CTA, leaving the scratch zeroed.
+//  * A warp's range meets each row block in one segment.  A segment that
+//    covers the whole row block is finished by the warp at once: each lane
+//    holds every sum of its (row, token) pairs, so out = sum_i act(g_i) v_i,
+//    rounded once to bf16, needs no exchange.  The range's first and last
+//    segments may be partial: the first is dropped into a shared-memory head
+//    slot, the last stays in registers.  After the stream (one __syncthreads,
+//    no fences while copies are in flight) the CTA adds the partial segments
+//    of each of its row blocks in warp order.  The first and last row block
+//    of a CTA's range may also have units in other CTAs: their CTA sums go to
+//    a small global scratch, and split_kernel, launched right after on the
+//    same stream, adds them in CTA order.  Every sum is therefore formed in
+//    a fixed order: results do not depend on timing.
 #pragma once
 #include <cstdint>
 #include <cuda_bf16.h>
@@ -57,14 +51,6 @@ constexpr int MAX_CTAS = 320;  // grid cap; sizes the split-row-block scratch
 // floats of one CTA's partial of a split row block: the largest slot (n_m = 8,
 // 16 tokens)
 constexpr int PART_FLOATS = 9 * ROWS * 16;
-// named barriers: slot set b is full (writers arrive, the part's finisher
-// waits); a set is free again for part f (the finisher of part f - SETS
-// arrives once it has read it, the other warps wait) on FREE0 + f % 2
-constexpr int BAR_FULL0 = 1;
-constexpr int BAR_FREE0 = 3;
-// cooperative finishing (token capacity 8 or 16): the reducer warps' own
-// barrier
-constexpr int BAR_READ = 5;
 
 // Token capacity TT of an instance (2, 8 or 16 tokens) and its 8-token
 // MMA column blocks.
@@ -84,9 +70,11 @@ struct DefaultShape {
 };
 
 // A warp's slot holds its sums of a part compactly: float (v, row, tok) at
-// (v * ROWS + row) * T + tok for the call's T tokens (v = 0 the dense
-// product, 1 + i mask i), so writing, adding and finishing a part cost in
-// proportion to the tokens the call has, not to the MMA's 8 columns.
+// (v * ROWS + row) * TT + tok for the instance's token capacity TT (v = 0 the
+// dense product, 1 + i mask i).  Only the call's T tokens are written and
+// added, so writing, adding and finishing a part cost in proportion to the
+// tokens the call has, not to the MMA's 8 columns; the constant stride keeps
+// every slot address a fixed offset from the lane's base.
 template <int NM, int TT>
 constexpr int slot_floats()
 {
@@ -96,16 +84,14 @@ constexpr int slot_floats()
 template <int NM, int TT, int NW_ = DefaultShape<NM, TT>::NW>
 struct Layout {
     static constexpr int NT = token_blocks<TT>();
-    static constexpr int NW = NW_;                     // warps, each a consumer and in turn a finisher
-    static constexpr int UPW = 2;                      // 32-k units per warp and stage
+    static constexpr int NW = NW_;                     // warps, each streaming its own unit range
+    static constexpr int UPW = STEP_K / 32;            // 32-k MMA units per unit of work
     static constexpr int NTHREADS = NW * 32;
-    static constexpr int BAR_COUNT = NW * 32;
-    static constexpr int KS = NW * 32 * UPW;           // k per stage
     static constexpr int ACC = slot_floats<NM, TT>();  // floats of one warp's slot
-    static constexpr int SLOT_SET = NW * ACC;          // floats of one slot set
-    // one stage of a warp's ring, per unit u and lane: W rows g and g + 8
-    // (16 bytes each) and their mask bytes (n_m >= 4; narrower masks go
-    // through registers), laid out lane-contiguous per row so that each
+    static constexpr int HEADS = NW * ACC;             // the warps' head slots
+    // one stage of a warp's ring, per 32-k MMA unit u and lane: W rows g and
+    // g + 8 (16 bytes each) and their mask bytes (n_m >= 4; narrower masks
+    // go through registers), laid out lane-contiguous per row so that each
     // 16-byte read of a warp is conflict-free; x comes from L1 (its rows are
     // small and every warp of every CTA reads them)
     static constexpr int MB = NM >= 4 ? NM : 0;         // mask bytes per lane and row in the ring
@@ -116,17 +102,14 @@ struct Layout {
     static __host__ __device__ constexpr int m_b(int u) { return UPW * W_BYTES + u * M_BYTES + 32 * MB; }
     static constexpr int STG = (UPW * (W_BYTES + M_BYTES) + 127) / 128 * 128;
     static constexpr int BUDGET = 227 * 1024;
-    static constexpr int ring_depth(int sets) { return (BUDGET - sets * SLOT_SET * 4) / (NW * STG); }
-    // two slot sets when a set is small (an eighth of shared memory at
-    // most), so a part's finisher never holds up the next part; else one,
-    // leaving the room to the ring
-    static constexpr int SETS = TT <= 2 && SLOT_SET * 4 <= BUDGET / 8 ? 2 : 1;
-    static constexpr int P = ring_depth(SETS) > 8 ? 8 : ring_depth(SETS);
-    static constexpr int RING_OFF = SETS * SLOT_SET * 4;
+    static constexpr int DEPTH = (BUDGET - HEADS * 4) / (NW * STG);
+    static constexpr int P = DEPTH > 8 ? 8 : DEPTH;    // ring stages per warp
+    static constexpr int RING_OFF = HEADS * 4;
     static constexpr int SMEM = RING_OFF + NW * P * STG;
     static_assert(NW % 4 == 0, "warps are allocated registers in groups of four");
     static_assert(P >= 3, "ring too shallow");
     static_assert(SMEM <= BUDGET, "shared memory");
+    static_assert(HEADS <= NW * P * STG / 4, "the tail slots reuse the rings after the stream");
 };
 
 // ---------------------------------------------------------------- loads
@@ -304,207 +287,151 @@ __device__ __forceinline__ void write_partials(float *__restrict__ gv, int64_t p
     }
 }
 
-// Finish row-block part f (the calling warp is its finisher) from the NW
-// slots of its set (compact, see slot_floats): add them element by element
-// in warp order into the warp's own slot, arrive on FREE barrier free_bar (if
-// not 0: a later part reuses the set; the own slot is written again only by
-// this warp), then either write the outputs or, for a row block split
-// between CTAs, publish this CTA's partial sums and let the last CTA to
-// arrive add all partials in CTA order and write them.  Not inlined: it runs
-// once per part, and keeping its registers out of the streaming loop leaves
-// that loop without spills.
-template <int NM, bool ROUTED, int NW>
-__device__ __noinline__ void finish_part(float *__restrict__ set_base, int slot_cap, int rb, bool stream_k,
-                                         int free_bar, const Sched sc, int act, int T, int rows,
-                                         float *__restrict__ ws_part, int *__restrict__ ws_count,
-                                         __nv_bfloat16 *__restrict__ out, const float *__restrict__ mw,
-                                         float *__restrict__ gv)
+// The output of one (row, token) of row block rb from its NM + 1 sums (or,
+// for the checking entry point, its partial sums).
+template <int NM, bool ROUTED>
+__device__ __forceinline__ void write_output(const float (&sums)[NM + 1], int rb, int row, int tok, int act, int T,
+                                             int rows, __nv_bfloat16 *__restrict__ out,
+                                             const float *__restrict__ mw, float *__restrict__ gv)
 {
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int E = (NM + 1) * ROWS * T;  // sums of the part
-    float *own = set_base + warp * slot_cap;
+    const int r = rb * ROWS + row;
+    if (r >= rows)
+        return;
+    const int64_t at = (int64_t)tok * rows + r;
+    if (gv)
+        write_partials<NM>(gv, (int64_t)T * rows, at, sums);
+    else
+        out[at] = __float2bfloat16_rn(out_value<NM>(act, sums, ROUTED ? mw + (int64_t)tok * NM : nullptr));
+}
+
+// After the stream, one warp per row block of its CTA's range: add the
+// partial segments this CTA's warps hold of row block rb, in warp order (a
+// warp's first segment sits in its head slot, its last in its tail slot),
+// then write the outputs, or, if other CTAs also hold units of rb, store
+// this CTA's sums for split_kernel.  A row block that one warp covered whole
+// was finished by that warp already.
+template <int NM, int TT, bool ROUTED>
+__device__ __noinline__ void combine_cta(int rb, const Plan pl, const float *__restrict__ heads,
+                                         const float *__restrict__ tails, int act, int T, int rows,
+                                         float *__restrict__ ws_part, __nv_bfloat16 *__restrict__ out,
+                                         const float *__restrict__ mw, float *__restrict__ gv)
+{
+    constexpr int ACC = slot_floats<NM, TT>();
+    const int lane = threadIdx.x & 31;
+    const int cta = blockIdx.x, w0 = cta * pl.NW;
+    const uint32_t ub = (uint32_t)rb * (uint32_t)pl.nsw, ue = ub + (uint32_t)pl.nsw;
+    int w_lo = pl.owner(ub), w_hi = pl.owner(ue - 1u);
+    if (w_lo == w_hi)
+        return;  // one warp covered it whole
+    w_lo = w_lo > w0 ? w_lo : w0;
+    w_hi = w_hi < w0 + pl.NW - 1 ? w_hi : w0 + pl.NW - 1;
+    int c_first, c_last;
+    pl.ctas_of(rb, c_first, c_last);
+    float *mine = c_first != c_last ? ws_part + (int64_t)pl.slot(cta, rb) * PART_FLOATS : nullptr;
 #pragma unroll 1
-    for (int e = lane; e < E; e += 32) {
-        float v[NW];
+    for (int p = lane; p < ROWS * T; p += 32) {
+        const int row = p / T, tok = p - row * T;
+        float sums[NM + 1];
 #pragma unroll
-        for (int w = 0; w < NW; ++w)
-            v[w] = set_base[w * slot_cap + e];
-        float s = v[0];
-#pragma unroll
-        for (int w = 1; w < NW; ++w)
-            s += v[w];
-        own[e] = s;  // element e of the own slot was read above, by this lane
-    }
-    if (free_bar) {
-        __threadfence_block();  // the slot reads above come before the set is written again
-        named_bar_arrive(free_bar, NW * 32);  // the other warps may write this set again
-    }
-    bool finish = true;
-    if (stream_k) {
-        int c_first, c_last;
-        const int nparts = sc.contributors(rb, c_first, c_last);
-        if (c_first != c_last) {
-            float *mine = ws_part + (int64_t)sc.slot(sc.cta, rb) * PART_FLOATS;
+        for (int v = 0; v <= NM; ++v)
+            sums[v] = 0.f;
 #pragma unroll 1
-            for (int e = lane; e < E; e += 32)
-                __stcg(mine + e, own[e]);
-            __threadfence();
-            __syncwarp();
-            int prev = 0;
-            if (lane == 0)
-                prev = atomicAdd(ws_count + rb, 1);
-            prev = __shfl_sync(0xffffffffu, prev, 0);
-            finish = prev == nparts - 1;
-            if (finish) {
-                // every partial, this CTA's included, read back in CTA order
-                __threadfence();
-#pragma unroll 1
-                for (int e = lane; e < E; e += 32) {
-                    float s = 0.f;
-#pragma unroll 1
-                    for (int cc = c_first; cc <= c_last; ++cc)
-                        if (sc.contributes(cc))
-                            s += __ldcg(ws_part + (int64_t)sc.slot(cc, rb) * PART_FLOATS + e);
-                    own[e] = s;
-                }
-                if (lane == 0)
-                    ws_count[rb] = 0;  // leave the scratch zeroed for the next call
-            }
-        }
-    }
-    if (finish) {
-        __syncwarp();  // every lane's sums are in the own slot
-        const int row0 = rb * ROWS;
-        const int64_t plane = (int64_t)T * rows;
-#pragma unroll 1
-        for (int p = lane; p < ROWS * T; p += 32) {
-            const int row = p / T, tok = p - row * T;
-            if (row0 + row >= rows)
-                continue;
-            float sums[NM + 1];
+        for (int w = w_lo; w <= w_hi; ++w) {
+            const uint32_t b = pl.begin(w), e = pl.begin(w + 1);
+            if (b == e)
+                continue;  // an empty range (more warps than units) holds nothing
+            // warp w's first row block is its head segment unless it is also its last
+            const int first = (int)(b / (uint32_t)pl.nsw), last = (int)((e - 1u) / (uint32_t)pl.nsw);
+            const float *src = (rb == first && first != last ? heads : tails) + (w - w0) * ACC;
 #pragma unroll
             for (int v = 0; v <= NM; ++v)
-                sums[v] = own[(v * ROWS + row) * T + tok];
-            const int64_t at = (int64_t)tok * rows + row0 + row;
-            if (gv)
-                write_partials<NM>(gv, plane, at, sums);
-            else
-                out[at] = __float2bfloat16_rn(out_value<NM>(act, sums, ROUTED ? mw + (int64_t)tok * NM : nullptr));
+                sums[v] += src[(v * ROWS + row) * TT + tok];
+        }
+        if (mine) {
+#pragma unroll
+            for (int v = 0; v <= NM; ++v)
+                mine[(v * ROWS + row) * TT + tok] = sums[v];
+        } else {
+            write_output<NM, ROUTED>(sums, rb, row, tok, act, T, rows, out, mw, gv);
         }
     }
 }
 
-// Cooperative finishing of part f for token capacities 8 and 16, run by the
-// reducer warps (the first R = ceil(16 T / 32) warps), one thread per
-// (row, token) of the row block: it adds that output's NM + 1 sums over the
-// NW slots in warp order, the reducers meet on BAR_READ (every slot is read)
-// and, if a later part exists and some warps are not reducers, arrive on
-// FREE so those warps may write the set again.  A row block split between
-// CTAs is finished as in finish_part, by whichever CTA arrives last.
-template <int NM, bool ROUTED, int NW>
-__device__ __noinline__ void finish_coop(const float *__restrict__ set_base, int slot_cap, int rb, bool stream_k,
-                                         int R, bool free_arrive, const Sched sc, int act, int T, int rows,
-                                         float *__restrict__ ws_part, int *__restrict__ ws_count,
-                                         __nv_bfloat16 *__restrict__ out, const float *__restrict__ mw,
-                                         float *__restrict__ gv)
+// Row blocks whose units several CTAs hold: the first CTA of each (for which
+// it is the last row block of its range) adds every CTA's stored sums in CTA
+// order and writes the outputs.  Launched after the decode kernel on the same
+// stream (its stores are visible once it has completed); one warp per CTA of
+// that grid, most of which have nothing to do.
+template <int NM, int TT, bool ROUTED>
+__global__ void __launch_bounds__(32) split_kernel(int rows, int d, int grid, int nw, int T, int act,
+                                                   const float *__restrict__ ws_part,
+                                                   __nv_bfloat16 *__restrict__ out, const float *__restrict__ mw,
+                                                   float *__restrict__ gv)
 {
-    __shared__ int s_last;
-    const int p = threadIdx.x;  // (row, token) of this thread
-    const bool has = p < ROWS * T;
-    const int row = has ? p / T : 0, tok = has ? p - row * T : 0;
-    float sums[NM + 1];
-#pragma unroll
-    for (int v = 0; v <= NM; ++v) {
-        float acc = 0.f;
-        if (has) {
-            const float *q = set_base + (v * ROWS + row) * T + tok;
-            acc = q[0];
-#pragma unroll
-            for (int w = 1; w < NW; ++w)
-                acc += q[w * slot_cap];
-        }
-        sums[v] = acc;
-    }
-    named_bar_sync(BAR_READ, R * 32);  // every reducer has read the set
-    if (free_arrive) {
-        __threadfence_block();
-        named_bar_arrive(BAR_FREE0, NW * 32);
-    }
-    bool finish = true;
-    if (stream_k) {
-        int c_first, c_last;
-        const int nparts = sc.contributors(rb, c_first, c_last);
-        if (c_first != c_last) {
-            float *mine = ws_part + (int64_t)sc.slot(sc.cta, rb) * PART_FLOATS;
-            if (has) {
-#pragma unroll
-                for (int v = 0; v <= NM; ++v)
-                    __stcg(mine + (v * ROWS + row) * T + tok, sums[v]);
-            }
-            __threadfence();
-            named_bar_sync(BAR_READ, R * 32);  // this CTA's partial is published
-            if (p == 0)
-                s_last = atomicAdd(ws_count + rb, 1) == nparts - 1;
-            named_bar_sync(BAR_READ, R * 32);
-            finish = s_last != 0;
-            if (finish) {
-                // every partial, this CTA's included, read back in CTA order
-                __threadfence();
-                if (has) {
-#pragma unroll
-                    for (int v = 0; v <= NM; ++v) {
-                        float acc = 0.f;
+    pdl_launch_dependents();
+    Plan pl;
+    pl.init(rows, d, grid, nw);
+    const int c = blockIdx.x;
+    if (!pl.cta_has_units(c))
+        return;
+    const int rb = pl.last_rb(c);
+    int c_first, c_last;
+    pl.ctas_of(rb, c_first, c_last);
+    if (c_first == c_last || c_first != c)
+        return;
+    pdl_wait();  // the decode kernel has completed
+    const int lane = threadIdx.x;
 #pragma unroll 1
-                        for (int cc = c_first; cc <= c_last; ++cc)
-                            if (sc.contributes(cc))
-                                acc += __ldcg(ws_part + (int64_t)sc.slot(cc, rb) * PART_FLOATS +
-                                              (v * ROWS + row) * T + tok);
-                        sums[v] = acc;
-                    }
-                }
-                if (p == 0)
-                    ws_count[rb] = 0;  // leave the scratch zeroed for the next call
-            }
+    for (int p = lane; p < ROWS * T; p += 32) {
+        const int row = p / T, tok = p - row * T;
+        float sums[NM + 1];
+#pragma unroll
+        for (int v = 0; v <= NM; ++v)
+            sums[v] = 0.f;
+#pragma unroll 1
+        for (int cc = c_first; cc <= c_last; ++cc) {
+            if (!pl.cta_has_units(cc))
+                continue;
+            const float *src = ws_part + (int64_t)pl.slot(cc, rb) * PART_FLOATS;
+#pragma unroll
+            for (int v = 0; v <= NM; ++v)
+                sums[v] += src[(v * ROWS + row) * TT + tok];
         }
-    }
-    const int row0 = rb * ROWS;
-    if (finish && has && row0 + row < rows) {
-        const int64_t at = (int64_t)tok * rows + row0 + row;
-        if (gv)
-            write_partials<NM>(gv, (int64_t)T * rows, at, sums);
-        else
-            out[at] = __float2bfloat16_rn(out_value<NM>(act, sums, ROUTED ? mw + (int64_t)tok * NM : nullptr));
+        write_output<NM, ROUTED>(sums, rb, row, tok, act, T, rows, out, mw, gv);
     }
 }
 
-// Scratch (global, caller-provided): partial sums of split row blocks, two
-// slots per CTA (first and last row block of its stream-K share), then one
-// arrival counter per row block.  Counters must be zero on entry and are
-// zero again when the kernel completes.
+// The decode kernel.  Scratch (global, caller-provided): this CTA's sums of
+// the first and the last row block of its range when other CTAs also hold
+// units of them (read by split_kernel); it needs no initialization.
 //
 // ROUTED: per-token mask weights mw [T][NM] scale each mask's term, and a
 // mask that no token of the call weights (all its weights zero) skips its
 // products (the weight stream is read in full either way).
+// gv (not NULL): write the partial sums D, g_i, v_i instead of outputs.
 template <int NM, int TT, bool ROUTED = false, int NW_ = DefaultShape<NM, TT>::NW>
 __global__ void __launch_bounds__(Layout<NM, TT, NW_>::NTHREADS, 1)
     decode_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__restrict__ W,
                   const uint8_t *__restrict__ packed, int T, int rows, int d, int act, float *__restrict__ ws_part,
-                  int *__restrict__ ws_count, __nv_bfloat16 *__restrict__ out, const float *__restrict__ mw,
-                  float *__restrict__ gv)
+                  __nv_bfloat16 *__restrict__ out, const float *__restrict__ mw, float *__restrict__ gv)
 {
     using L = Layout<NM, TT, NW_>;
     constexpr int NT = L::NT;
-    extern __shared__ __align__(128) float slots[];  // L::SETS sets of NW slots, then the warps' rings
+    extern __shared__ __align__(128) float slots[];  // the warps' head slots, then their rings
 
     // The next kernel in the stream may start its prologue now; every access
     // to global memory below waits for the previous kernel to finish.
     pdl_launch_dependents();
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int g = lane >> 2, c = lane & 3;
-    Sched sc;
-    sc.init(rows, d, L::KS, gridDim.x, blockIdx.x);
-    if (sc.n == 0)
+    Plan pl;
+    pl.init(rows, d, gridDim.x, L::NW);
+    if (!pl.cta_has_units(blockIdx.x))
         return;
+    const int gw = blockIdx.x * L::NW + warp;
+    const uint32_t u0 = pl.begin(gw), u1 = pl.begin(gw + 1);
+    const int n = (int)(u1 - u0);  // this warp's units
+    const int nsw = pl.nsw;
     pdl_wait();
 
     // masks some token of the call weights
@@ -516,10 +443,10 @@ __global__ void __launch_bounds__(Layout<NM, TT, NW_>::NTHREADS, 1)
         used = __reduce_or_sync(0xffffffffu, u);
     }
 
-    // ----------------------------------------------------------------- consumers
-    // This warp's units of stage ks start at k = ks * KS + 32 * (UPW * warp + u);
-    // this lane's 8 weights of unit u at k = that + 8 * c.
-    const int kl = 32 * L::UPW * warp + 8 * c;
+    // Unit (rb, s) covers k = s * STEP_K + 32 u + [0, 32) for MMA units u of
+    // rows rb * ROWS + [0, 16); this lane's 8 weights of MMA unit u start at
+    // k = s * STEP_K + 32 u + 8 c.
+    const int kl = 8 * c;
     const int64_t mrow = (int64_t)d * NM / 8;  // mask bytes per row of W
     int xrow[NT];
 #pragma unroll
@@ -528,42 +455,42 @@ __global__ void __launch_bounds__(Layout<NM, TT, NW_>::NTHREADS, 1)
     uint8_t *ring = reinterpret_cast<uint8_t *>(slots) + L::RING_OFF + warp * L::P * L::STG;
     const uint32_t ring_s = smem_u32(ring);
 
-    // The copy cursor: the stage it copies next and this lane's source
-    // pointers for it (rows g and g + 8 of the row block, k of the lane's
-    // piece of the warp's first unit).  Inside a row block the pointers
-    // advance by one stage; a new row block recomputes them.
+    // The copy cursor: the unit it copies next and this lane's source
+    // pointers for it (rows g and g + 8 of the row block).  Inside a row
+    // block the pointers advance by one unit; a new row block recomputes them.
     struct Cursor {
-        int rb, ks;
+        int rb, s;
         bool rows_in;  // all 16 rows of the row block exist
         const __nv_bfloat16 *wa, *wb;
         const uint8_t *ma, *mb;
     };
-    const int kfull = d / L::KS;  // k-stages that lie wholly inside the row
+    const int kfull = d / STEP_K;  // units that lie wholly inside the row
     auto place = [&](Cursor &cu) {
         const int ra = cu.rb * ROWS + g;
-        const int k = cu.ks * L::KS + kl;
+        const int k = cu.s * STEP_K + kl;
         cu.rows_in = cu.rb * ROWS + ROWS <= rows;
         cu.wa = W + (int64_t)ra * d + k;
         cu.wb = cu.wa + 8 * (int64_t)d;
         cu.ma = packed + (int64_t)ra * mrow + (int64_t)k * NM / 8;
         cu.mb = cu.ma + 8 * mrow;
     };
-    auto advance = [&](int i, Cursor &cu) {  // past unit i of this CTA
-        sc.next(i, cu.rb, cu.ks);
-        if (cu.ks != 0) {
-            cu.wa += L::KS, cu.wb += L::KS;
-            cu.ma += L::KS * NM / 8, cu.mb += L::KS * NM / 8;
+    auto advance = [&](Cursor &cu) {
+        if (++cu.s < nsw) {
+            cu.wa += STEP_K, cu.wb += STEP_K;
+            cu.ma += STEP_K * NM / 8, cu.mb += STEP_K * NM / 8;
         } else {
+            cu.s = 0;
+            ++cu.rb;
             place(cu);
         }
     };
-    // Copies of the cursor's stage into ring stage ss.  A stage wholly inside
+    // Copies of the cursor's unit into ring stage ss.  A unit wholly inside
     // the matrix copies without checks; otherwise lanes outside it copy
     // zeros (a d % 8 == 0 row keeps a lane's 8 weights all in or out).
     auto issue = [&](int ss, const Cursor &cu) {
         const uint32_t st = ring_s + (uint32_t)(ss * L::STG) + lane * 16;
         const uint32_t sm = ring_s + (uint32_t)(ss * L::STG) + lane * L::MB;
-        if (cu.rows_in && cu.ks < kfull) {
+        if (cu.rows_in && cu.s < kfull) {
 #pragma unroll
             for (int u = 0; u < L::UPW; ++u) {
                 cp_async_cg16(st + L::w_a(u), cu.wa + 32 * u);
@@ -577,7 +504,7 @@ __global__ void __launch_bounds__(Layout<NM, TT, NW_>::NTHREADS, 1)
             const int ra = cu.rb * ROWS + g;
 #pragma unroll
             for (int u = 0; u < L::UPW; ++u) {
-                const bool kin = cu.ks * L::KS + kl + 32 * u < d;
+                const bool kin = cu.s * STEP_K + kl + 32 * u < d;
                 const bool va = kin && ra < rows, vb = kin && ra + 8 < rows;
                 cp_async_cg16(st + L::w_a(u), va ? cu.wa + 32 * u : W, va ? 16u : 0u);
                 cp_async_cg16(st + L::w_b(u), vb ? cu.wb + 32 * u : W, vb ? 16u : 0u);
@@ -590,17 +517,17 @@ __global__ void __launch_bounds__(Layout<NM, TT, NW_>::NTHREADS, 1)
             }
         }
     };
-    // x of a stage comes from L1 (its rows are small and every warp reads
-    // them), loaded at the top of the stage's iteration; for n_m <= 2 the
+    // x of a unit comes from L1 (its rows are small and every warp reads
+    // them), loaded at the top of the unit's iteration; for n_m <= 2 the
     // narrow mask bits (one or two bytes a lane and row) stream from memory
-    // into registers one stage ahead.
+    // into registers one unit ahead.
     const __nv_bfloat16 *xl[NT];  // this lane's x rows at its k offset
 #pragma unroll
     for (int t = 0; t < NT; ++t)
         xl[t] = x + (int64_t)xrow[t] * d + kl;
-    auto load_x = [&](uint4 (&xv)[L::UPW][NT], int ks) {
-        const int k0 = ks * L::KS;
-        if (ks < kfull) {
+    auto load_x = [&](uint4 (&xv)[L::UPW][NT], int s) {
+        const int k0 = s * STEP_K;
+        if (s < kfull) {
 #pragma unroll
             for (int u = 0; u < L::UPW; ++u)
 #pragma unroll
@@ -617,11 +544,11 @@ __global__ void __launch_bounds__(Layout<NM, TT, NW_>::NTHREADS, 1)
     struct NarrowMasks {
         uint2 a[L::UPW], b[L::UPW];
     };
-    auto load_narrow = [&](NarrowMasks &nm, int rb, int ks) {
+    auto load_narrow = [&](NarrowMasks &nm, int rb, int s) {
         const int ra = rb * ROWS + g, rbb = ra + 8;
 #pragma unroll
         for (int u = 0; u < L::UPW; ++u) {
-            const int k = ks * L::KS + kl + 32 * u;
+            const int k = s * STEP_K + kl + 32 * u;
             const bool kin = k < d;
             nm.a[u] = nm.b[u] = make_uint2(0u, 0u);
             if (kin && ra < rows)
@@ -632,11 +559,10 @@ __global__ void __launch_bounds__(Layout<NM, TT, NW_>::NTHREADS, 1)
     };
     constexpr bool NARROW = NM > 0 && L::MB == 0;
 
-    const int nflushes = sc.flushes();
     float acc[NM + 1][NT][4];
     zero_acc<NM, NT>(acc);
-    // a warp's sums of a part into its slot, compactly (see slot_floats)
-    auto write_slot = [&](float *slot, const float (&a)[NM + 1][NT][4]) {
+    // a warp's sums of a segment into a slot, compactly (see slot_floats)
+    auto write_slot = [&](float *slot) {
 #pragma unroll
         for (int v = 0; v <= NM; ++v)
 #pragma unroll
@@ -645,52 +571,72 @@ __global__ void __launch_bounds__(Layout<NM, TT, NW_>::NTHREADS, 1)
                 for (int r = 0; r < 4; ++r) {
                     const int tok = 8 * t + 2 * c + (r & 1), row = g + 8 * (r >> 1);
                     if (tok < T)
-                        slot[(v * ROWS + row) * T + tok] = a[v][t][r];
+                        slot[(v * ROWS + row) * TT + tok] = acc[v][t][r];
                 }
     };
+    // a row block this warp covered whole: every lane holds all NM + 1 sums
+    // of its (row, token) pairs, so it writes their outputs directly
+    auto finish_whole = [&](int rb) {
+#pragma unroll
+        for (int t = 0; t < NT; ++t)
+#pragma unroll
+            for (int r = 0; r < 4; ++r) {
+                const int tok = 8 * t + 2 * c + (r & 1), row = g + 8 * (r >> 1);
+                if (tok < T) {
+                    float sums[NM + 1];
+#pragma unroll
+                    for (int v = 0; v <= NM; ++v)
+                        sums[v] = acc[v][t][r];
+                    write_output<NM, ROUTED>(sums, rb, row, tok, act, T, rows, out, mw, gv);
+                }
+            }
+    };
 
-    // the copy cursor runs P - 1 stages ahead of the compute cursor
-    int rb_c, ks_c;
-    sc.start(rb_c, ks_c);
+    // the copy cursor runs P - 1 units ahead of the compute cursor
+    int rb_c = (int)(u0 / (uint32_t)nsw), s_c = (int)(u0 % (uint32_t)nsw);
+    int seg_start = s_c;  // first unit of the current segment
     Cursor cl;
-    cl.rb = rb_c, cl.ks = ks_c;
+    cl.rb = rb_c, cl.s = s_c;
     place(cl);
     for (int b = 0; b < L::P - 1; ++b) {
-        if (b < sc.n)
+        if (b < n)
             issue(b, cl);
-        cp_async_commit();  // one group per stage, empty past the end
-        if (b + 1 < sc.n)
-            advance(b, cl);
+        cp_async_commit();  // one group per unit, empty past the end
+        if (b + 1 < n)
+            advance(cl);
     }
     NarrowMasks nmask;
-    if constexpr (NARROW)
-        load_narrow(nmask, rb_c, ks_c);
+    if constexpr (NARROW) {
+        if (n > 0)
+            load_narrow(nmask, rb_c, s_c);
+    }
 
-    int nflush = 0;
-    for (int i = 0; i < sc.n; ++i) {
+    bool tail = false;  // the last segment is partial: its sums stay in acc
+    for (int i = 0; i < n; ++i) {
         uint4 xv[L::UPW][NT];
-        load_x(xv, ks_c);
+        load_x(xv, s_c);
         const int il = i + L::P - 1;
-        if (il < sc.n)
+        if (il < n)
             issue(il % L::P, cl);
         cp_async_commit();
-        if (il + 1 < sc.n)
-            advance(il, cl);
-        int rb_n = rb_c, ks_n = ks_c;
-        sc.next(i, rb_n, ks_n);
+        if (il + 1 < n)
+            advance(cl);
+        int rb_n = rb_c, s_n = s_c + 1;
+        if (s_n == nsw)
+            s_n = 0, ++rb_n;
         NarrowMasks cur;
         if constexpr (NARROW) {
             cur = nmask;
-            if (i + 1 < sc.n)
-                load_narrow(nmask, rb_n, ks_n);
+            if (i + 1 < n)
+                load_narrow(nmask, rb_n, s_n);
         }
-        cp_async_wait<L::P - 1>();  // this lane's copies of stage i have landed
+        cp_async_wait<L::P - 1>();  // this lane's copies of unit i have landed
 
+        // Units past the end of the row (a ragged last unit) hold zeros in
+        // the ring and in x, so they add nothing.
         const uint8_t *st = ring + (i % L::P) * L::STG;
 #pragma unroll
         for (int u = 0; u < L::UPW; ++u) {
-            if (ks_c * L::KS + 32 * (L::UPW * warp + u) >= d)
-                continue;  // the whole unit lies past the end of the row
             Operands<NM, NT> o;
             o.wa = *reinterpret_cast<const uint4 *>(st + L::w_a(u) + lane * 16);
             o.wb = *reinterpret_cast<const uint4 *>(st + L::w_b(u) + lane * 16);
@@ -712,56 +658,38 @@ __global__ void __launch_bounds__(Layout<NM, TT, NW_>::NTHREADS, 1)
             unit_step<NM, NT, ROUTED, 0>(acc, o, used);
             unit_step<NM, NT, ROUTED, 1>(acc, o, used);
         }
-        if (sc.flush_at(i, ks_c)) {
-            // ---------------------------------------------- row-block part done here
-            const int f = nflush++;
-            if constexpr (TT <= 2) {
-                const int set = f % L::SETS;
-                // this set was last used by part f - SETS: wait until its
-                // finisher has read it (that finisher arrived as soon as it
-                // had, and does not wait here); the FREE barrier alternates by
-                // part
-                if (f >= L::SETS && warp != (f - L::SETS) % L::NW)
-                    named_bar_sync(BAR_FREE0 + (f & 1), L::BAR_COUNT);
-                write_slot(slots + set * L::SLOT_SET + warp * L::ACC, acc);
+        if (s_c == nsw - 1 || i == n - 1) {
+            // ---------------------------------------------- a segment ends here
+            if (seg_start == 0 && s_c == nsw - 1) {
+                finish_whole(rb_c);
                 zero_acc<NM, NT>(acc);
-                if (warp == f % L::NW) {
-                    named_bar_sync(BAR_FULL0 + set, L::BAR_COUNT);  // every slot of part f is written
-                    finish_part<NM, ROUTED, L::NW>(slots + set * L::SLOT_SET, L::ACC, rb_c, i < sc.n_sk,
-                                                   f + L::SETS < nflushes ? BAR_FREE0 + ((f + L::SETS) & 1) : 0,
-                                                   sc, act, T, rows, ws_part, ws_count, out, mw, gv);
-                } else {
-                    __threadfence_block();  // the slot writes are visible before the finisher reads them
-                    named_bar_arrive(BAR_FULL0 + set, L::BAR_COUNT);
-                }
+            } else if (i < n - 1) {
+                write_slot(slots + warp * L::ACC);  // the head: the range's first segment
+                zero_acc<NM, NT>(acc);
             } else {
-                // one slot set; the reducers read part f - 1 before anyone
-                // writes part f (the reducers met on BAR_READ after reading,
-                // the others wait on FREE, on which the reducers arrived)
-                const int R = (ROWS * T + 31) / 32;
-                if (f >= 1 && warp >= R)
-                    named_bar_sync(BAR_FREE0, L::BAR_COUNT);
-                write_slot(slots + warp * L::ACC, acc);
-                zero_acc<NM, NT>(acc);
-                named_bar_sync(BAR_FULL0, L::BAR_COUNT);  // every slot of part f is written
-                if (warp < R)
-                    finish_coop<NM, ROUTED, L::NW>(slots, L::ACC, rb_c, i < sc.n_sk, R,
-                                                   f + 1 < nflushes && R < L::NW, sc, act, T, rows, ws_part,
-                                                   ws_count, out, mw, gv);
+                tail = true;
             }
+            seg_start = 0;
         }
-        rb_c = rb_n, ks_c = ks_n;
+        rb_c = rb_n, s_c = s_n;
     }
-    cp_async_wait<0>();  // no copy outlives the kernel
+    cp_async_wait<0>();  // no copy outlives the stream
+
+    // After the stream: the partial segments of the CTA's row blocks.
+    float *tails = slots + L::HEADS;  // the rings are free once every warp is here
+    __syncthreads();
+    if (tail)
+        write_slot(tails + warp * L::ACC);
+    __syncthreads();
+    const int rb_last = pl.last_rb(blockIdx.x);
+#pragma unroll 1
+    for (int rb = pl.first_rb(blockIdx.x) + warp; rb <= rb_last; rb += L::NW)
+        combine_cta<NM, TT, ROUTED>(rb, pl, slots, tails, act, T, rows, ws_part, out, mw, gv);
 }
 
-// Scratch bytes of the decode kernel: partial slots for the largest grid,
-// then one counter per row block of `rows` (256-byte aligned pieces).
+// Scratch bytes of the decode kernel: two partial slots per CTA.
 __host__ __device__ constexpr int64_t part_bytes() { return (int64_t)2 * MAX_CTAS * PART_FLOATS * 4; }
-__host__ __device__ constexpr int64_t workspace_bytes(int64_t rows)
-{
-    return part_bytes() + ((rows + ROWS - 1) / ROWS * 4 + 255) / 256 * 256;
-}
+__host__ __device__ constexpr int64_t workspace_bytes(int64_t) { return part_bytes(); }
 
 }  // namespace dec
 }  // namespace mglu

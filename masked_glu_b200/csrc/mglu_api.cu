@@ -214,26 +214,42 @@ int launch_decode(const void *x, int64_t T, int64_t d, const void *W, int64_t ro
                   void *out, void *ws, cudaStream_t s, const float *mw, float *gv)
 {
     using L = mglu::dec::Layout<NM, TT>;
-    if (d >= ((int64_t)1 << 22) || rows >= ((int64_t)1 << 27))
-        return MGLU_ERR_INVALID;  // the kernel's 32-bit schedule arithmetic
+    const int64_t rb = (rows + mglu::dec::ROWS - 1) / mglu::dec::ROWS;
+    const int64_t units = rb * ((d + mglu::dec::STEP_K - 1) / mglu::dec::STEP_K);
+    if (units >= ((int64_t)1 << 31))
+        return MGLU_ERR_INVALID;  // the kernel's 32-bit unit numbering
     int dev = 0, rc = current_device(&dev);
     if (rc)
         return rc;
     if ((rc = ensure_smem<mglu::dec::decode_kernel<NM, TT, ROUTED>>(L::SMEM, dev)))
         return rc;
-    const int64_t rb = (rows + mglu::dec::ROWS - 1) / mglu::dec::ROWS;
-    const int64_t units = rb * ((d + L::KS - 1) / L::KS);
     int64_t grid = (int64_t)sm_count(dev);
     if (grid > mglu::dec::MAX_CTAS)
         grid = mglu::dec::MAX_CTAS;
     if (grid > units)
         grid = units;
     float *ws_part = reinterpret_cast<float *>(ws);
-    int *ws_count = reinterpret_cast<int *>(reinterpret_cast<uint8_t *>(ws) + mglu::dec::part_bytes());
-    return launch_pdl(mglu::dec::decode_kernel<NM, TT, ROUTED>, dim3((unsigned)grid), dim3(L::NTHREADS), L::SMEM, s,
-                      "decode launch", reinterpret_cast<const __nv_bfloat16 *>(x),
-                      reinterpret_cast<const __nv_bfloat16 *>(W), packed, (int)T, (int)rows, (int)d, act, ws_part,
-                      ws_count, reinterpret_cast<__nv_bfloat16 *>(out), mw, gv);
+    __nv_bfloat16 *o = reinterpret_cast<__nv_bfloat16 *>(out);
+    if ((rc = launch_pdl(mglu::dec::decode_kernel<NM, TT, ROUTED>, dim3((unsigned)grid), dim3(L::NTHREADS), L::SMEM, s,
+                         "decode launch", reinterpret_cast<const __nv_bfloat16 *>(x),
+                         reinterpret_cast<const __nv_bfloat16 *>(W), packed, (int)T, (int)rows, (int)d, act, ws_part, o,
+                         mw, gv)))
+        return rc;
+    // row blocks whose units several CTAs hold are finished by split_kernel
+    mglu::dec::Plan pl;
+    pl.init((int)rows, (int)d, (int)grid, L::NW);
+    bool shared = false;
+    for (int c = 0; c < (int)grid && !shared; ++c) {
+        if (!pl.cta_has_units(c))
+            continue;
+        int cf, cl;
+        pl.ctas_of(pl.last_rb(c), cf, cl);
+        shared = cf != cl;
+    }
+    if (!shared)
+        return MGLU_OK;
+    return launch_pdl(mglu::dec::split_kernel<NM, TT, ROUTED>, dim3((unsigned)grid), dim3(32), 0, s, "split launch",
+                      (int)rows, (int)d, (int)grid, L::NW, (int)T, act, (const float *)ws_part, o, mw, gv);
 }
 
 // Token capacity by T: 2, 8 or 16 (the slots and the finisher's work follow
@@ -872,12 +888,6 @@ int mglu_forward_decode_static(const void *x, int64_t T, int64_t d, const void *
     void *ws = nullptr;
     if ((rc = static_scratch(dev, s, &ws)))
         return rc;
-    // the arrival counters of this call's row blocks must start at zero
-    const size_t counters = (size_t)((h + mglu::dec::ROWS - 1) / mglu::dec::ROWS) * sizeof(int);
-    const cudaError_t e =
-        cudaMemsetAsync(reinterpret_cast<uint8_t *>(ws) + mglu::dec::part_bytes(), 0, counters, s);
-    if (e != cudaSuccess)
-        return cuda_fail(e, "clear built-in decode scratch counters");
     return by_nm<DecodeF>(n_m, x, T, d, W, h, packed, act, out, ws, s, (const float *)nullptr);
 }
 

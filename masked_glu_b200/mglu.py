@@ -170,7 +170,7 @@ _scratch = {}
 def default_scratch(rows: int, device) -> torch.Tensor:
     """A zero-filled scratch buffer per device, grown on demand and shared by
     calls that pass none.  Calls on several streams at once must pass their
-    own buffers (the decode kernel's counters are not safe to share)."""
+    own buffers (the decode kernel's partial slots are not safe to share)."""
     dev = torch.device(device)
     key = dev.index if dev.index is not None else torch.cuda.current_device()
     need = scratch_bytes(rows)

@@ -1,10 +1,14 @@
 // Host check of the decode kernel's work split (masked_glu_b200/csrc/sched.cuh)
-// over many shapes and grid sizes: every (row block, k-stage) unit is done by
-// exactly one CTA; a row block is either finished inside one CTA or is a
-// stream-K row block whose contributors (counted by Sched::contributors) are
-// exactly the CTAs that flush a part of it; their scratch slots are distinct
-// and each CTA uses each of its two slots for at most one row block; and
-// Sched::flushes() counts a CTA's flushes exactly.
+// over many shapes and grid sizes, following the kernel's own steps:
+//  - every (row block, unit) is streamed by exactly one warp;
+//  - a warp's range meets each row block in one segment; only its first
+//    segment can go to the head slot and only its last stays as the tail;
+//  - after the stream, the CTA's combine for a row block adds exactly the
+//    partial segments its warps hold of it (head or tail as the kernel picks
+//    them), and publishes to a scratch slot that no other row block uses;
+//  - split_kernel's chosen CTA adds exactly the CTAs that published that
+//    row block;
+//  - every row block's outputs are written exactly once.
 // Prints "ok" and exits 0 on success.
 #include <cstdio>
 #include <map>
@@ -13,117 +17,141 @@
 
 #include "sched.cuh"
 
-using mglu::dec::ROWS;
-using mglu::dec::Sched;
+using mglu::dec::Plan;
 
-static int check(int rows, int d, int ks_width, int G)
+static int fail(const char *what, int rows, int d, int G, int NW, int a, int b)
 {
-    Sched ref;
-    ref.init(rows, d, ks_width, G, 0);
-    const int RB = ref.RB, nst = ref.nst;
-    std::vector<int> seen((size_t)RB * nst, 0);
-    std::map<int, std::set<int>> flushers;        // stream-K row block -> CTAs flushing it
-    std::map<int, int> slot_owner;                // slot -> row block
-    std::set<int> complete;                       // row blocks finished inside one CTA
-    for (int c = 0; c < G; ++c) {
-        Sched sc;
-        sc.init(rows, d, ks_width, G, c);
-        int rb, ks, cur_rb = -1, seg_start = 0, nflush = 0;
-        sc.start(rb, ks);
-        for (int i = 0; i < sc.n; sc.next(i, rb, ks), ++i) {
-            nflush += sc.flush_at(i, ks) ? 1 : 0;
-            if (rb < 0 || rb >= RB || ks < 0 || ks >= nst) {
-                std::printf("unit out of range rows=%d d=%d G=%d c=%d rb=%d ks=%d\n", rows, d, G, c, rb, ks);
-                return 1;
-            }
-            seen[(size_t)rb * nst + ks]++;
-            if (rb != cur_rb) {  // a new row-block segment of this CTA
-                cur_rb = rb;
-                seg_start = ks;
-            }
-            if (!sc.flush_at(i, ks))
-                continue;
-            const bool whole = seg_start == 0 && ks == nst - 1;
-            if (i < sc.n_sk) {
-                int cf, cl;
-                const int np = sc.contributors(rb, cf, cl);
-                if (cf == cl) {
-                    if (!whole || cf != c) {
-                        std::printf("stream-K row block %d owned by one CTA but not whole (c=%d)\n", rb, c);
-                        return 1;
-                    }
-                    complete.insert(rb);
+    std::printf("%s (rows=%d d=%d grid=%d nw=%d: %d %d)\n", what, rows, d, G, NW, a, b);
+    return 1;
+}
+
+static int check(int rows, int d, int G, int NW)
+{
+    Plan pl;
+    pl.init(rows, d, G, NW);
+    const int RB = pl.RB, nsw = pl.nsw;
+    std::vector<int> seen((size_t)pl.U, 0), written(RB, 0);
+    // partial segments: row block -> warps holding one, and which slot kind
+    std::map<int, std::map<int, char>> partial;  // rb -> (warp -> 'h' or 't')
+    for (int gw = 0; gw < pl.GW; ++gw) {
+        const uint32_t u0 = pl.begin(gw), u1 = pl.begin(gw + 1);
+        const int n = (int)(u1 - u0);
+        int rb = (int)(u0 / nsw), s = (int)(u0 % nsw), seg_start = s;
+        for (int i = 0; i < n; ++i) {
+            const uint32_t u = u0 + (uint32_t)i;
+            if (u != (uint32_t)rb * nsw + (uint32_t)s || rb >= RB)
+                return fail("unit numbering", rows, d, G, NW, gw, i);
+            if (pl.owner(u) != gw)
+                return fail("owner() disagrees with begin()", rows, d, G, NW, gw, (int)u);
+            seen[u]++;
+            if (s == nsw - 1 || i == n - 1) {
+                if (seg_start == 0 && s == nsw - 1) {
+                    if (!pl.covers(gw, rb))
+                        return fail("whole segment not covered", rows, d, G, NW, gw, rb);
+                    written[rb]++;
+                } else if (i < n - 1) {
+                    if (rb != (int)(u0 / nsw))
+                        return fail("head slot used by a later segment", rows, d, G, NW, gw, rb);
+                    partial[rb][gw] = 'h';
                 } else {
-                    flushers[rb].insert(c);
-                    const int sl = sc.slot(c, rb);
-                    if (sl != 2 * c && sl != 2 * c + 1) {
-                        std::printf("slot %d not owned by CTA %d\n", sl, c);
-                        return 1;
-                    }
-                    if (slot_owner.count(sl) && slot_owner[sl] != rb) {
-                        std::printf("slot %d used for row blocks %d and %d\n", sl, slot_owner[sl], rb);
-                        return 1;
-                    }
-                    slot_owner[sl] = rb;
-                    (void)np;
+                    partial[rb][gw] = 't';
                 }
-            } else {
-                if (!whole) {
-                    std::printf("data-parallel row block %d not whole in CTA %d\n", rb, c);
-                    return 1;
-                }
-                complete.insert(rb);
+                seg_start = 0;
             }
-            cur_rb = -1;  // the next unit starts a new segment
-        }
-        if (nflush != sc.flushes()) {
-            std::printf("CTA %d flushes %d times, flushes() says %d (rows=%d d=%d ks=%d G=%d)\n", c, nflush,
-                        sc.flushes(), rows, d, ks_width, G);
-            return 1;
+            if (++s == nsw)
+                s = 0, ++rb;
         }
     }
-    for (size_t u = 0; u < seen.size(); ++u)
-        if (seen[u] != 1) {
-            std::printf("unit %zu done %d times (rows=%d d=%d ks=%d G=%d)\n", u, seen[u], rows, d, ks_width, G);
-            return 1;
+    for (uint32_t u = 0; u < pl.U; ++u)
+        if (seen[u] != 1)
+            return fail("unit not streamed exactly once", rows, d, G, NW, (int)u, seen[u]);
+    std::map<int, int> slot_rb;                 // scratch slot -> row block
+    std::map<int, std::set<int>> published;     // row block -> CTAs that stored sums
+    for (int c = 0; c < G; ++c) {
+        if (!pl.cta_has_units(c))
+            continue;
+        const int w0 = c * NW;
+        for (int rb = pl.first_rb(c); rb <= pl.last_rb(c); ++rb) {
+            const uint32_t ub = (uint32_t)rb * nsw, ue = ub + nsw;
+            int w_lo = pl.owner(ub), w_hi = pl.owner(ue - 1u);
+            if (w_lo == w_hi) {
+                if (partial.count(rb))
+                    return fail("row block skipped but has partial segments", rows, d, G, NW, c, rb);
+                continue;
+            }
+            w_lo = w_lo > w0 ? w_lo : w0;
+            w_hi = w_hi < w0 + NW - 1 ? w_hi : w0 + NW - 1;
+            std::set<int> used;
+            for (int w = w_lo; w <= w_hi; ++w) {
+                if (pl.begin(w + 1) == pl.begin(w))
+                    continue;  // an empty range holds nothing (its slots are never read)
+                const int first = (int)(pl.begin(w) / nsw), last = (int)((pl.begin(w + 1) - 1u) / nsw);
+                const char kind = (rb == first && first != last) ? 'h' : 't';
+                auto it = partial.find(rb);
+                if (it == partial.end() || !it->second.count(w) || it->second.at(w) != kind)
+                    return fail("combine reads a slot that does not hold this row block", rows, d, G, NW, w, rb);
+                used.insert(w);
+            }
+            for (auto &kv : partial[rb])
+                if (kv.first / NW == c && !used.count(kv.first))
+                    return fail("combine misses a partial segment", rows, d, G, NW, kv.first, rb);
+            int cf, cl;
+            pl.ctas_of(rb, cf, cl);
+            if (cf == cl) {
+                written[rb]++;
+            } else {
+                const int sl = pl.slot(c, rb);
+                if (sl != 2 * c && sl != 2 * c + 1)
+                    return fail("slot outside the CTA's pair", rows, d, G, NW, c, sl);
+                if (slot_rb.count(sl) && slot_rb[sl] != rb)
+                    return fail("slot reused for two row blocks", rows, d, G, NW, sl, rb);
+                slot_rb[sl] = rb;
+                published[rb].insert(c);
+            }
         }
-    for (auto &kv : flushers) {
+    }
+    for (int c = 0; c < G; ++c) {  // split_kernel
+        if (!pl.cta_has_units(c))
+            continue;
+        const int rb = pl.last_rb(c);
         int cf, cl;
-        const int np = ref.contributors(kv.first, cf, cl);
-        std::set<int> want;
+        pl.ctas_of(rb, cf, cl);
+        if (cf == cl || cf != c)
+            continue;
+        std::set<int> adds;
         for (int cc = cf; cc <= cl; ++cc)
-            if (ref.contributes(cc))
-                want.insert(cc);
-        if ((int)kv.second.size() != np || kv.second != want) {
-            std::printf("row block %d: %zu CTAs flush it, contributors says %d (rows=%d d=%d G=%d)\n", kv.first,
-                        kv.second.size(), np, rows, d, G);
-            return 1;
-        }
-        if (complete.count(kv.first)) {
-            std::printf("row block %d both split and complete\n", kv.first);
-            return 1;
-        }
+            if (pl.cta_has_units(cc)) {
+                adds.insert(cc);
+                if (slot_rb.count(pl.slot(cc, rb)) == 0 || slot_rb[pl.slot(cc, rb)] != rb)
+                    return fail("split adds a slot that holds another row block", rows, d, G, NW, cc, rb);
+            }
+        if (adds != published[rb])
+            return fail("split adds a different set of CTAs than published", rows, d, G, NW, c, rb);
+        written[rb]++;
     }
-    if ((int)(complete.size() + flushers.size()) != RB) {
-        std::printf("row blocks accounted %zu of %d (rows=%d d=%d G=%d)\n", complete.size() + flushers.size(), RB,
-                    rows, d, G);
-        return 1;
-    }
+    for (int rb = 0; rb < RB; ++rb)
+        if (written[rb] != 1)
+            return fail("row block not written exactly once", rows, d, G, NW, rb, written[rb]);
     return 0;
 }
 
 int main()
 {
-    const int rows_list[] = {1, 16, 40, 200, 1024, 4096, 8192, 14336, 2000};
-    const int d_list[] = {8, 128, 200, 640, 2048, 4096, 14336};
-    const int ks_list[] = {256, 384, 512, 768, 1024};
-    const int g_list[] = {1, 7, 64, 148, 296, 320};
+    const int rows_list[] = {1, 7, 16, 17, 33, 100, 256, 1000, 2048, 8192, 14336};
+    const int d_list[] = {8, 64, 72, 200, 512, 1000, 2048, 4096};
+    const int grids[] = {1, 2, 3, 7, 148, 320};
+    const int nws[] = {8, 12, 16};
     for (int rows : rows_list)
         for (int d : d_list)
-            for (int ks : ks_list)
-                for (int G : g_list)
-                    if (check(rows, d, ks, G))
+            for (int G : grids)
+                for (int NW : nws) {
+                    Plan pl;
+                    pl.init(rows, d, G, NW);
+                    if ((uint32_t)G > pl.U)
+                        continue;  // the host caps the grid at the number of units
+                    if (check(rows, d, G, NW))
                         return 1;
+                }
     std::printf("ok\n");
     return 0;
 }

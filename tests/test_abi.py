@@ -96,7 +96,8 @@ def test_forward_rejects_bad_arguments(L):
     assert fwd(L, ws=None) == mglu.ERR_INVALID
     assert fwd(L, wsb=need - 1) == mglu.ERR_INVALID
     assert fwd(L, ws=A + 8, wsb=need) == mglu.ERR_ALIGN
-    assert L.mglu_scratch_bytes(14336) > L.mglu_scratch_bytes(16)
+    # two partial slots per CTA of the grid, whatever the number of rows
+    assert L.mglu_scratch_bytes(14336) == L.mglu_scratch_bytes(16)
 
 
 def test_forward_zero_tokens_is_a_noop(L):

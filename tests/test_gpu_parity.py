@@ -210,19 +210,21 @@ def test_forward_down_block(T):
 
 
 @pytest.mark.parametrize("T", [1, 9])
-def test_decode_scratch_is_left_zeroed(T):
-    """Row blocks split between CTAs go through the scratch counters; every
-    call must leave them at zero for the next one."""
+def test_decode_scratch_needs_no_initialization(T):
+    """Row blocks split between CTAs pass their partial sums through the
+    scratch; every slot is written before it is read, so a scratch full of
+    NaN bit patterns gives the same result as a zeroed one, call after call."""
     case = inputs.make_case(T, 2048, 256, 8, seed=700 + T)
     x, W, packed, _ = device_case(case)
-    scratch = torch.zeros(mglu.scratch_bytes(256), dtype=torch.uint8, device="cuda")
-    outs = []
+    clean = torch.zeros(mglu.scratch_bytes(256), dtype=torch.uint8, device="cuda")
+    want = to_f64(mglu.forward(x, W, packed, 8, "swish", scratch=clean))
+    dirty = torch.full((mglu.scratch_bytes(256),), 0xFF, dtype=torch.uint8, device="cuda")
     for _ in range(3):
-        outs.append(to_f64(mglu.forward(x, W, packed, 8, "swish", scratch=scratch)))
+        got = to_f64(mglu.forward(x, W, packed, 8, "swish", scratch=dirty))
         torch.cuda.synchronize()
-        counters = scratch[mglu.scratch_bytes(256) - 256:].cpu().numpy()
-        assert not counters.any(), "scratch counters not reset"
-    assert np.array_equal(outs[0], outs[1]) and np.array_equal(outs[1], outs[2]), "run-to-run difference"
+        assert np.array_equal(got, want), "result depends on the scratch's prior contents"
+    ref, _ = oracle.forward(case.x.values, case.W.values, oracle_packed(case), 8, ACT["swish"])
+    assert_close(want, ref, "bf16", f"decode T={T}")
 
 
 # Repeat tests: every repeat must match the oracle and be bit-identical to
@@ -286,10 +288,8 @@ def test_forward_host_matches_device_calls(n_m, T, d, h, down):
 def test_workspace_reused_across_token_counts_and_block_modes():
     """One workspace reused by FFN-block calls of different token counts
     (tensor-core hidden write, then decode), and by host-buffer calls with and
-    without the down-projection: the decode scratch sits at the start of the
-    workspace, so activations written by one call never land on the arrival
-    counters a later call reads.  Every result must equal the same call made
-    on a fresh zero-filled workspace."""
+    without the down-projection: whatever an earlier call left in it, every
+    result must equal the same call made on a fresh workspace."""
     d, h, n_m = 256, 1024, 8
     case = inputs.make_case(512, d, h, n_m, seed=1300, with_down=True)
     x, W, packed, Wd = device_case(case)
