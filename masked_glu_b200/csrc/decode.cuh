@@ -175,18 +175,27 @@ struct Operands {
     uint4 xv[NT];
 };
 
-// v << S for a constant S >= 0, as an integer multiply so that it issues to
-// the FMA pipe (the ALU pipe takes the LOP3s of the sign flips).
-template <int S>
-__device__ __forceinline__ uint32_t shl_fma(uint32_t v)
-{
-    if constexpr (S == 0) {
-        return v;
-    } else {
-        uint32_t r;
-        asm("mul.lo.u32 %0, %1, %2;" : "=r"(r) : "r"(v), "n"(1u << S));
-        return r;
+// The shifts of the sign flips, v << (15 - I) for mask I, as integer
+// multiplies by powers of two held in registers.  The value 1 they are made
+// from is not known to the compiler, which would otherwise turn a constant
+// shift into an ALU instruction: the ALU pipe already takes one LOP3 per
+// flipped bf16 pair, so the shifts go to the FMA pipe instead.
+template <int NM>
+struct Shifts {
+    uint32_t m[NM > 0 ? NM : 1];
+    __device__ __forceinline__ void init(uint32_t one)
+    {
+#pragma unroll
+        for (int i = 0; i < NM; ++i)
+            m[i] = one << (15 - i);
     }
+};
+
+__device__ __forceinline__ uint32_t mul_u32(uint32_t v, uint32_t m)
+{
+    uint32_t r;
+    asm("mul.lo.u32 %0, %1, %2;" : "=r"(r) : "r"(v), "r"(m));
+    return r;
 }
 
 __device__ __forceinline__ uint32_t u4(const uint4 &v, int q)
@@ -199,20 +208,25 @@ __device__ __forceinline__ uint32_t u4(const uint4 &v, int q)
 // gives them a nonzero weight) skip their products.
 template <int NM, int NT, bool ROUTED, int S, int I>
 struct FlipLoop {
+    // ra, rb: the group bits of rows g and g + 8 (mask I of the pair (4S, 4S+1)
+    // at bits I and 16 + I); ra8, rb8 the same words shifted right by 8 (mask
+    // I of the pair (4S+2, 4S+3) at those bits).  Shifting left by 15 - I puts
+    // the bits at 15 and 31, the pairs' sign bits.
     static __device__ __forceinline__ void run(float (&acc)[NM + 1][NT][4], const Operands<NM, NT> &o, uint32_t ra,
-                                               uint32_t rb, uint32_t used)
+                                               uint32_t rb, uint32_t ra8, uint32_t rb8, uint32_t used,
+                                               const Shifts<NM> &sh)
     {
         if constexpr (I < NM) {
             if (!ROUTED || ((used >> I) & 1u)) {
-                const uint32_t a0 = flip_pair(u4(o.wa, 2 * S), shl_fma<15 - I>(ra));
-                const uint32_t a1 = flip_pair(u4(o.wb, 2 * S), shl_fma<15 - I>(rb));
-                const uint32_t a2 = flip_pair(u4(o.wa, 2 * S + 1), shl_fma<7 - I>(ra));
-                const uint32_t a3 = flip_pair(u4(o.wb, 2 * S + 1), shl_fma<7 - I>(rb));
+                const uint32_t a0 = flip_pair(u4(o.wa, 2 * S), mul_u32(ra, sh.m[I]));
+                const uint32_t a1 = flip_pair(u4(o.wb, 2 * S), mul_u32(rb, sh.m[I]));
+                const uint32_t a2 = flip_pair(u4(o.wa, 2 * S + 1), mul_u32(ra8, sh.m[I]));
+                const uint32_t a3 = flip_pair(u4(o.wb, 2 * S + 1), mul_u32(rb8, sh.m[I]));
 #pragma unroll
                 for (int t = 0; t < NT; ++t)
                     mma_bf16_16816(acc[1 + I][t], a0, a1, a2, a3, u4(o.xv[t], 2 * S), u4(o.xv[t], 2 * S + 1));
             }
-            FlipLoop<NM, NT, ROUTED, S, I + 1>::run(acc, o, ra, rb, used);
+            FlipLoop<NM, NT, ROUTED, S, I + 1>::run(acc, o, ra, rb, ra8, rb8, used, sh);
         }
     }
 };
@@ -223,7 +237,8 @@ struct FlipLoop {
 // and S; x (operand B) is loaded with the same permutation, so every sum is
 // unchanged.
 template <int NM, int NT, bool ROUTED, int S>
-__device__ __forceinline__ void unit_step(float (&acc)[NM + 1][NT][4], const Operands<NM, NT> &o, uint32_t used)
+__device__ __forceinline__ void unit_step(float (&acc)[NM + 1][NT][4], const Operands<NM, NT> &o, uint32_t used,
+                                          const Shifts<NM> &sh)
 {
 #pragma unroll
     for (int t = 0; t < NT; ++t)
@@ -232,7 +247,7 @@ __device__ __forceinline__ void unit_step(float (&acc)[NM + 1][NT][4], const Ope
     if constexpr (NM > 0) {
         const uint32_t ra = group_bits<NM, S>(o.ma.x, o.ma.y);
         const uint32_t rb = group_bits<NM, S>(o.mb.x, o.mb.y);
-        FlipLoop<NM, NT, ROUTED, S, 0>::run(acc, o, ra, rb, used);
+        FlipLoop<NM, NT, ROUTED, S, 0>::run(acc, o, ra, rb, ra >> 8, rb >> 8, used, sh);
     }
 }
 
@@ -433,6 +448,9 @@ __global__ void __launch_bounds__(Layout<NM, TT, NW_>::NTHREADS, 1)
     const int n = (int)(u1 - u0);  // this warp's units
     const int nsw = pl.nsw;
     pdl_wait();
+
+    Shifts<NM> sh;
+    sh.init(1u + ((uint32_t)act >> 16));  // act < 2^16: the value is 1
 
     // masks some token of the call weights
     uint32_t used = (1u << NM) - 1u;
@@ -655,8 +673,8 @@ __global__ void __launch_bounds__(Layout<NM, TT, NW_>::NTHREADS, 1)
             } else {
                 o.ma = o.mb = make_uint2(0u, 0u);
             }
-            unit_step<NM, NT, ROUTED, 0>(acc, o, used);
-            unit_step<NM, NT, ROUTED, 1>(acc, o, used);
+            unit_step<NM, NT, ROUTED, 0>(acc, o, used, sh);
+            unit_step<NM, NT, ROUTED, 1>(acc, o, used, sh);
         }
         if (s_c == nsw - 1 || i == n - 1) {
             // ---------------------------------------------- a segment ends here

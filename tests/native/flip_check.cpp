@@ -1,8 +1,8 @@
 // Host check of the sign-flip operand construction used by the decode kernel
 // (masked_glu_b200/csrc/common.cuh: group_bits, flip_pair).  For every n_m,
 // k16 group S, weight pair p and mask I, it shifts group_bits as the kernel
-// does (left by 15 - I for the pair (4S, 4S+1), by 7 - I for (4S+2, 4S+3))
-// and checks that bits 15 and 31 are mask I of the pair's two weights as the
+// does (left by 15 - I for the pair (4S, 4S+1); right by 8, then left by
+// 15 - I, for (4S+2, 4S+3)) and checks that bits 15 and 31 are mask I of the pair's two weights as the
 // packed format defines them (bit w*n_m + i of an 8-weight chunk is mask i
 // of weight w), and that flip_pair negates exactly the weights whose bit is
 // clear.  Prints "ok" and exits 0 on success.
@@ -20,8 +20,7 @@ static int check_group(uint32_t lo, uint32_t hi, uint32_t w)
     int bad = 0;
     for (int p = 0; p < 2; ++p)
         for (int I = 0; I < NM; ++I) {
-            const int shift = p == 0 ? 15 - I : 7 - I;
-            const uint32_t m = r << shift;
+            const uint32_t m = (p == 0 ? r : r >> 8) << (15 - I);
             const int w0 = 4 * S + 2 * p, w1 = w0 + 1;
             const uint32_t b0 = (uint32_t)(bits >> (w0 * NM + I)) & 1u;
             const uint32_t b1 = (uint32_t)(bits >> (w1 * NM + I)) & 1u;
