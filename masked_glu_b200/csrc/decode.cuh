@@ -505,17 +505,56 @@ __global__ void __launch_bounds__(Layout<NM, TT, NW_>::NTHREADS, 1)
     // Copies of the cursor's unit into ring stage ss.  A unit wholly inside
     // the matrix copies without checks; otherwise lanes outside it copy
     // zeros (a d % 8 == 0 row keeps a lane's 8 weights all in or out).
+    // Mask bytes (n_m >= 4): the four lanes of a group g hold 4 * MB
+    // contiguous bytes per row and MMA unit, so when the packed rows are
+    // 16-byte strided the group copies them in 16-byte pieces (lane c takes
+    // pieces c, c + 4, ...), a quarter (n_m = 4) or half (n_m = 8) as many
+    // copies as one per lane; the lanes then read each other's bytes after a
+    // __syncwarp.  Otherwise every lane copies its own MB bytes.
+    constexpr int MH = L::MB / 4 > 0 ? L::MB / 4 : 1;  // 16-byte pieces per row and MMA unit
+    constexpr int MPL = 2 * L::UPW * MH / 4;           // pieces per lane
+    const bool mask16 = L::MB > 0 && mrow % 16 == 0;
+    auto issue_masks16 = [&](uint32_t stage, const Cursor &cu, bool checked) {
+        const uint8_t *ma0 = cu.ma - c * L::MB, *mb0 = cu.mb - c * L::MB;  // the group's first bytes
+        const int ra = cu.rb * ROWS + g;
+#pragma unroll
+        for (int j = 0; j < MPL; ++j) {
+            const int q = c + 4 * j;
+            const int row = q / (L::UPW * MH), u = (q / MH) % L::UPW, half = q % MH;
+            const uint8_t *src = (row ? mb0 : ma0) + u * (32 * NM / 8) + half * 16;
+            const uint32_t dst = stage + (row ? L::m_b(u) : L::m_a(u)) + g * 4 * L::MB + half * 16;
+            if (!checked) {
+                cp_async_cg16(dst, src);
+            } else {
+                const int kp = cu.s * STEP_K + 32 * u + half * (128 / NM);  // first weight of the piece
+                const int wts = d - kp < 128 / NM ? d - kp : 128 / NM;
+                const bool ok = wts > 0 && ra + 8 * row < rows;
+                cp_async_cg16(dst, ok ? src : packed, ok ? (uint32_t)(wts * NM / 8) : 0u);
+            }
+        }
+    };
+    // Copies of the cursor's unit into ring stage ss.  A unit wholly inside
+    // the matrix copies without checks; otherwise lanes outside it copy
+    // zeros (a d % 8 == 0 row keeps a lane's 8 weights all in or out).
     auto issue = [&](int ss, const Cursor &cu) {
-        const uint32_t st = ring_s + (uint32_t)(ss * L::STG) + lane * 16;
-        const uint32_t sm = ring_s + (uint32_t)(ss * L::STG) + lane * L::MB;
+        const uint32_t stage = ring_s + (uint32_t)(ss * L::STG);
+        const uint32_t st = stage + lane * 16;
+        const uint32_t sm = stage + lane * L::MB;
         if (cu.rows_in && cu.s < kfull) {
 #pragma unroll
             for (int u = 0; u < L::UPW; ++u) {
                 cp_async_cg16(st + L::w_a(u), cu.wa + 32 * u);
                 cp_async_cg16(st + L::w_b(u), cu.wb + 32 * u);
-                if constexpr (L::MB > 0) {
-                    cp_async_ca<L::MB>(sm + L::m_a(u), cu.ma + 32 * u * NM / 8);
-                    cp_async_ca<L::MB>(sm + L::m_b(u), cu.mb + 32 * u * NM / 8);
+            }
+            if constexpr (L::MB > 0) {
+                if (mask16) {
+                    issue_masks16(stage, cu, false);
+                } else {
+#pragma unroll
+                    for (int u = 0; u < L::UPW; ++u) {
+                        cp_async_ca<L::MB>(sm + L::m_a(u), cu.ma + 32 * u * NM / 8);
+                        cp_async_ca<L::MB>(sm + L::m_b(u), cu.mb + 32 * u * NM / 8);
+                    }
                 }
             }
         } else {
@@ -527,11 +566,17 @@ __global__ void __launch_bounds__(Layout<NM, TT, NW_>::NTHREADS, 1)
                 cp_async_cg16(st + L::w_a(u), va ? cu.wa + 32 * u : W, va ? 16u : 0u);
                 cp_async_cg16(st + L::w_b(u), vb ? cu.wb + 32 * u : W, vb ? 16u : 0u);
                 if constexpr (L::MB > 0) {
-                    cp_async_ca<L::MB>(sm + L::m_a(u), va ? cu.ma + 32 * u * NM / 8 : packed,
-                                       va ? (uint32_t)L::MB : 0u);
-                    cp_async_ca<L::MB>(sm + L::m_b(u), vb ? cu.mb + 32 * u * NM / 8 : packed,
-                                       vb ? (uint32_t)L::MB : 0u);
+                    if (!mask16) {
+                        cp_async_ca<L::MB>(sm + L::m_a(u), va ? cu.ma + 32 * u * NM / 8 : packed,
+                                           va ? (uint32_t)L::MB : 0u);
+                        cp_async_ca<L::MB>(sm + L::m_b(u), vb ? cu.mb + 32 * u * NM / 8 : packed,
+                                           vb ? (uint32_t)L::MB : 0u);
+                    }
                 }
+            }
+            if constexpr (L::MB > 0) {
+                if (mask16)
+                    issue_masks16(stage, cu, true);
             }
         }
     };
@@ -649,6 +694,8 @@ __global__ void __launch_bounds__(Layout<NM, TT, NW_>::NTHREADS, 1)
                 load_narrow(nmask, rb_n, s_n);
         }
         cp_async_wait<L::P - 1>();  // this lane's copies of unit i have landed
+        if constexpr (L::MB > 0)
+            __syncwarp();  // and, for the shared mask pieces, every lane's
 
         // Units past the end of the row (a ragged last unit) hold zeros in
         // the ring and in x, so they add nothing.
