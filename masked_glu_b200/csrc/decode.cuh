@@ -6,7 +6,7 @@
 // are read exactly once and the masks are unpacked inside the kernel):
 //
 //  * Work is made of units (row block of ROWS = 16 rows of W, step of
-//    STEP_K = 64 k: two 32-k MMA units).  A persistent grid of one CTA per
+//    STEP = 64 k: two 32-k MMA units).  A persistent grid of one CTA per
 //    SM gives every warp of the grid an equal contiguous range of units
 //    (warp-level stream-K, see sched.cuh), so all warps stream the same
 //    number of bytes and none ever waits for another while it streams.
@@ -66,7 +66,10 @@ constexpr int token_blocks()
 // thread, 12 get 168, 8 get 255.
 template <int NM, int TT>
 struct DefaultShape {
-    static constexpr int NW = token_blocks<TT>() == 1 ? 16 : NM == 8 ? 8 : NM == 4 ? 12 : 16;
+    // n_m = 8 with 3 to 8 tokens: 8 warps of 255 registers, four MMA units
+    // per unit of work (measured faster there; not at 1 or 2 tokens)
+    static constexpr int NW = token_blocks<TT>() == 1 ? (NM == 8 && TT == 8 ? 8 : 16) : NM == 8 ? 8 : NM == 4 ? 12 : 16;
+    static constexpr int UPW = NM == 8 && TT == 8 ? 4 : 2;  // 32-k MMA units a warp takes per unit of work
 };
 
 // A warp's slot holds its sums of a part compactly: float (v, row, tok) at
@@ -85,7 +88,8 @@ template <int NM, int TT, int NW_ = DefaultShape<NM, TT>::NW>
 struct Layout {
     static constexpr int NT = token_blocks<TT>();
     static constexpr int NW = NW_;                     // warps, each streaming its own unit range
-    static constexpr int UPW = STEP_K / 32;            // 32-k MMA units per unit of work
+    static constexpr int UPW = DefaultShape<NM, TT>::UPW;  // 32-k MMA units per unit of work
+    static constexpr int STEP = 32 * UPW;              // k per unit of work
     static constexpr int NTHREADS = NW * 32;
     static constexpr int ACC = slot_floats<NM, TT>();  // floats of one warp's slot
     static constexpr int HEADS = NW * ACC;             // the warps' head slots
@@ -378,14 +382,14 @@ __device__ __noinline__ void combine_cta(int rb, const Plan pl, const float *__r
 // stream (its stores are visible once it has completed); one warp per CTA of
 // that grid, most of which have nothing to do.
 template <int NM, int TT, bool ROUTED>
-__global__ void __launch_bounds__(32) split_kernel(int rows, int d, int grid, int nw, int T, int act,
+__global__ void __launch_bounds__(32) split_kernel(int rows, int d, int step, int grid, int nw, int T, int act,
                                                    const float *__restrict__ ws_part,
                                                    __nv_bfloat16 *__restrict__ out, const float *__restrict__ mw,
                                                    float *__restrict__ gv)
 {
     pdl_launch_dependents();
     Plan pl;
-    pl.init(rows, d, grid, nw);
+    pl.init(rows, d, step, grid, nw);
     const int c = blockIdx.x;
     if (!pl.cta_has_units(c))
         return;
@@ -440,7 +444,7 @@ __global__ void __launch_bounds__(Layout<NM, TT, NW_>::NTHREADS, 1)
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int g = lane >> 2, c = lane & 3;
     Plan pl;
-    pl.init(rows, d, gridDim.x, L::NW);
+    pl.init(rows, d, L::STEP, gridDim.x, L::NW);
     if (!pl.cta_has_units(blockIdx.x))
         return;
     const int gw = blockIdx.x * L::NW + warp;
@@ -461,9 +465,9 @@ __global__ void __launch_bounds__(Layout<NM, TT, NW_>::NTHREADS, 1)
         used = __reduce_or_sync(0xffffffffu, u);
     }
 
-    // Unit (rb, s) covers k = s * STEP_K + 32 u + [0, 32) for MMA units u of
+    // Unit (rb, s) covers k = s * STEP + 32 u + [0, 32) for MMA units u of
     // rows rb * ROWS + [0, 16); this lane's 8 weights of MMA unit u start at
-    // k = s * STEP_K + 32 u + 8 c.
+    // k = s * STEP + 32 u + 8 c.
     const int kl = 8 * c;
     const int64_t mrow = (int64_t)d * NM / 8;  // mask bytes per row of W
     int xrow[NT];
@@ -482,10 +486,10 @@ __global__ void __launch_bounds__(Layout<NM, TT, NW_>::NTHREADS, 1)
         const __nv_bfloat16 *wa, *wb;
         const uint8_t *ma, *mb;
     };
-    const int kfull = d / STEP_K;  // units that lie wholly inside the row
+    const int kfull = d / L::STEP;  // units that lie wholly inside the row
     auto place = [&](Cursor &cu) {
         const int ra = cu.rb * ROWS + g;
-        const int k = cu.s * STEP_K + kl;
+        const int k = cu.s * L::STEP + kl;
         cu.rows_in = cu.rb * ROWS + ROWS <= rows;
         cu.wa = W + (int64_t)ra * d + k;
         cu.wb = cu.wa + 8 * (int64_t)d;
@@ -494,8 +498,8 @@ __global__ void __launch_bounds__(Layout<NM, TT, NW_>::NTHREADS, 1)
     };
     auto advance = [&](Cursor &cu) {
         if (++cu.s < nsw) {
-            cu.wa += STEP_K, cu.wb += STEP_K;
-            cu.ma += STEP_K * NM / 8, cu.mb += STEP_K * NM / 8;
+            cu.wa += L::STEP, cu.wb += L::STEP;
+            cu.ma += L::STEP * NM / 8, cu.mb += L::STEP * NM / 8;
         } else {
             cu.s = 0;
             ++cu.rb;
@@ -526,8 +530,9 @@ __global__ void __launch_bounds__(Layout<NM, TT, NW_>::NTHREADS, 1)
             if (!checked) {
                 cp_async_cg16(dst, src);
             } else {
-                const int kp = cu.s * STEP_K + 32 * u + half * (128 / NM);  // first weight of the piece
-                const int wts = d - kp < 128 / NM ? d - kp : 128 / NM;
+                constexpr int PW = 128 / (NM > 0 ? NM : 1);  // weights per 16-byte piece
+                const int kp = cu.s * L::STEP + 32 * u + half * PW;  // first weight of the piece
+                const int wts = d - kp < PW ? d - kp : PW;
                 const bool ok = wts > 0 && ra + 8 * row < rows;
                 cp_async_cg16(dst, ok ? src : packed, ok ? (uint32_t)(wts * NM / 8) : 0u);
             }
@@ -561,7 +566,7 @@ __global__ void __launch_bounds__(Layout<NM, TT, NW_>::NTHREADS, 1)
             const int ra = cu.rb * ROWS + g;
 #pragma unroll
             for (int u = 0; u < L::UPW; ++u) {
-                const bool kin = cu.s * STEP_K + kl + 32 * u < d;
+                const bool kin = cu.s * L::STEP + kl + 32 * u < d;
                 const bool va = kin && ra < rows, vb = kin && ra + 8 < rows;
                 cp_async_cg16(st + L::w_a(u), va ? cu.wa + 32 * u : W, va ? 16u : 0u);
                 cp_async_cg16(st + L::w_b(u), vb ? cu.wb + 32 * u : W, vb ? 16u : 0u);
@@ -589,7 +594,7 @@ __global__ void __launch_bounds__(Layout<NM, TT, NW_>::NTHREADS, 1)
     for (int t = 0; t < NT; ++t)
         xl[t] = x + (int64_t)xrow[t] * d + kl;
     auto load_x = [&](uint4 (&xv)[L::UPW][NT], int s) {
-        const int k0 = s * STEP_K;
+        const int k0 = s * L::STEP;
         if (s < kfull) {
 #pragma unroll
             for (int u = 0; u < L::UPW; ++u)
@@ -611,7 +616,7 @@ __global__ void __launch_bounds__(Layout<NM, TT, NW_>::NTHREADS, 1)
         const int ra = rb * ROWS + g, rbb = ra + 8;
 #pragma unroll
         for (int u = 0; u < L::UPW; ++u) {
-            const int k = s * STEP_K + kl + 32 * u;
+            const int k = s * L::STEP + kl + 32 * u;
             const bool kin = k < d;
             nm.a[u] = nm.b[u] = make_uint2(0u, 0u);
             if (kin && ra < rows)

@@ -215,7 +215,7 @@ int launch_decode(const void *x, int64_t T, int64_t d, const void *W, int64_t ro
 {
     using L = mglu::dec::Layout<NM, TT>;
     const int64_t rb = (rows + mglu::dec::ROWS - 1) / mglu::dec::ROWS;
-    const int64_t units = rb * ((d + mglu::dec::STEP_K - 1) / mglu::dec::STEP_K);
+    const int64_t units = rb * ((d + L::STEP - 1) / L::STEP);
     if (units >= ((int64_t)1 << 31))
         return MGLU_ERR_INVALID;  // the kernel's 32-bit unit numbering
     int dev = 0, rc = current_device(&dev);
@@ -237,7 +237,7 @@ int launch_decode(const void *x, int64_t T, int64_t d, const void *W, int64_t ro
         return rc;
     // row blocks whose units several CTAs hold are finished by split_kernel
     mglu::dec::Plan pl;
-    pl.init((int)rows, (int)d, (int)grid, L::NW);
+    pl.init((int)rows, (int)d, L::STEP, (int)grid, L::NW);
     bool shared = false;
     for (int c = 0; c < (int)grid && !shared; ++c) {
         if (!pl.cta_has_units(c))
@@ -249,7 +249,7 @@ int launch_decode(const void *x, int64_t T, int64_t d, const void *W, int64_t ro
     if (!shared)
         return MGLU_OK;
     return launch_pdl(mglu::dec::split_kernel<NM, TT, ROUTED>, dim3((unsigned)grid), dim3(32), 0, s, "split launch",
-                      (int)rows, (int)d, (int)grid, L::NW, (int)T, act, (const float *)ws_part, o, mw, gv);
+                      (int)rows, (int)d, L::STEP, (int)grid, L::NW, (int)T, act, (const float *)ws_part, o, mw, gv);
 }
 
 // Token capacity by T: 2, 8 or 16 (the slots and the finisher's work follow

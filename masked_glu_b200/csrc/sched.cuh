@@ -1,6 +1,7 @@
 // sched.cuh -- how the decode kernel splits its work over a persistent grid.
 //
-// A unit is (row block of ROWS rows of W, step of STEP_K = 64 k).  The units
+// A unit is (row block of ROWS rows of W, step of k: 32 k per MMA unit
+// times the MMA units a warp takes at once).  The units
 // are numbered row block by row block, u = rb * nsw + s, and every warp of the
 // grid gets an equal contiguous range of them (warp-level stream-K): warp gw
 // of GW does [begin(gw), begin(gw + 1)).  A warp never waits for another while
@@ -19,18 +20,17 @@ namespace mglu {
 namespace dec {
 
 constexpr int ROWS = 16;
-constexpr int STEP_K = 64;  // k per unit: two 32-k MMA units of one warp
 
 struct Plan {
-    int nsw;     // units per row block (ceil(d / STEP_K))
+    int nsw;     // units per row block (ceil(d / step))
     int RB;      // row blocks
     uint32_t U;  // units, RB * nsw (the host keeps it below 2^31)
     int GW;      // warps of the grid
     int NW;      // warps per CTA
 
-    MGLU_HD void init(int rows, int d, int grid, int nw)
+    MGLU_HD void init(int rows, int d, int step, int grid, int nw)
     {
-        nsw = (d + STEP_K - 1) / STEP_K;
+        nsw = (d + step - 1) / step;
         RB = (rows + ROWS - 1) / ROWS;
         U = (uint32_t)RB * (uint32_t)nsw;
         NW = nw;

@@ -25,10 +25,10 @@ static int fail(const char *what, int rows, int d, int G, int NW, int a, int b)
     return 1;
 }
 
-static int check(int rows, int d, int G, int NW)
+static int check(int rows, int d, int step, int G, int NW)
 {
     Plan pl;
-    pl.init(rows, d, G, NW);
+    pl.init(rows, d, step, G, NW);
     const int RB = pl.RB, nsw = pl.nsw;
     std::vector<int> seen((size_t)pl.U, 0), written(RB, 0);
     // partial segments: row block -> warps holding one, and which slot kind
@@ -141,17 +141,19 @@ int main()
     const int d_list[] = {8, 64, 72, 200, 512, 1000, 2048, 4096};
     const int grids[] = {1, 2, 3, 7, 148, 320};
     const int nws[] = {8, 12, 16};
+    const int steps[] = {64, 128};
     for (int rows : rows_list)
         for (int d : d_list)
-            for (int G : grids)
-                for (int NW : nws) {
-                    Plan pl;
-                    pl.init(rows, d, G, NW);
-                    if ((uint32_t)G > pl.U)
-                        continue;  // the host caps the grid at the number of units
-                    if (check(rows, d, G, NW))
-                        return 1;
-                }
+            for (int step : steps)
+                for (int G : grids)
+                    for (int NW : nws) {
+                        Plan pl;
+                        pl.init(rows, d, step, G, NW);
+                        if ((uint32_t)G > pl.U)
+                            continue;  // the host caps the grid at the number of units
+                        if (check(rows, d, step, G, NW))
+                            return 1;
+                    }
     std::printf("ok\n");
     return 0;
 }
