@@ -17,6 +17,7 @@
 #include "decode.cuh"
 #include "pack.cuh"
 #include "prefill.cuh"
+#include "prefill_pair.cuh"
 #include "ptx.cuh"
 #include "route.cuh"
 #include "simt.cuh"
@@ -277,6 +278,62 @@ int decode_nt(const void *x, int64_t T, int64_t d, const void *W, int64_t rows, 
 }
 
 // ------------------------------------------------------------------ prefill
+// The forward on CTA pairs (clusters of two, one 256-token MMA per k16 step
+// issued by the first CTA of each pair); the grid is as many pairs as fit at
+// once, each looping over tiles.
+template <int NM>
+int launch_prefill_pair(const void *x, int64_t T, int64_t d, const void *W, int64_t rows, const uint8_t *packed,
+                        int act, void *out, cudaStream_t s, const float *mw, int dev)
+{
+    using C = mglu::pf::PairCfg<NM>;
+    CUtensorMap tx, tw, tm;
+    int rc;
+    if ((rc = make_map(&tx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, x, d, T, d * 2, mglu::pf::BK, mglu::pf::BM,
+                       CU_TENSOR_MAP_SWIZZLE_128B)))
+        return rc;
+    if ((rc = make_map(&tw, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, W, d, rows, d * 2, mglu::pf::BK, C::NJH,
+                       CU_TENSOR_MAP_SWIZZLE_128B)))
+        return rc;
+    if ((rc = make_map(&tm, CU_TENSOR_MAP_DATA_TYPE_UINT8, packed, d * NM / 8, rows, d * NM / 8, C::MB, C::NJH,
+                       CU_TENSOR_MAP_SWIZZLE_NONE)))
+        return rc;
+    if ((rc = ensure_smem<mglu::pf::prefill_pair_kernel<NM>>(C::SMEM, dev)))
+        return rc;
+    static std::atomic<int> max_pairs[kMaxDevices];
+    int pairs = max_pairs[dev].load(std::memory_order_relaxed);
+    cudaLaunchConfig_t cfg = {};
+    cfg.blockDim = dim3(C::NTHREADS);
+    cfg.dynamicSmemBytes = (size_t)C::SMEM;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    if (pairs == 0) {
+        cfg.gridDim = dim3((unsigned)(2 * sm_count(dev)));
+        cfg.numAttrs = 1;
+        const cudaError_t e = cudaOccupancyMaxActiveClusters(&pairs, mglu::pf::prefill_pair_kernel<NM>, &cfg);
+        if (e != cudaSuccess)
+            return cuda_fail(e, "cudaOccupancyMaxActiveClusters");
+        if (pairs < 1)
+            return MGLU_ERR_UNSUPPORTED;
+        max_pairs[dev].store(pairs, std::memory_order_relaxed);
+    }
+    const int64_t tiles = ((T + 2 * mglu::pf::BM - 1) / (2 * mglu::pf::BM)) * ((rows + C::NJ - 1) / C::NJ);
+    const int64_t grid_pairs = tiles < pairs ? tiles : pairs;
+    cfg.gridDim = dim3((unsigned)(2 * grid_pairs));
+    cfg.numAttrs = 2;
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, mglu::pf::prefill_pair_kernel<NM>, tx, tw, tm, (int)T, (int)rows,
+                                             (int)d, act, reinterpret_cast<__nv_bfloat16 *>(out), mw);
+    if (e != cudaSuccess)
+        return cuda_fail(e, "prefill pair launch");
+    return check_launch("prefill pair launch");
+}
+
 template <int NM, bool GRAD = false>
 int launch_prefill(const void *x, int64_t T, int64_t d, const void *W, int64_t rows, const uint8_t *packed, int act,
                    void *out, void *, cudaStream_t s, const float *mw, const void *dout = nullptr,
@@ -296,6 +353,10 @@ int launch_prefill(const void *x, int64_t T, int64_t d, const void *W, int64_t r
     // a tensor map needs 16-byte row strides; other packed rows are read by
     // the builder warps directly
     const int mask_direct = NM > 0 && (d * NM / 8) % 16 != 0;
+    if constexpr (NM > 0 && !GRAD) {
+        if (!mask_direct && T > mglu::pf::BM)
+            return launch_prefill_pair<NM>(x, T, d, W, rows, packed, act, out, s, mw, dev);
+    }
     if (NM > 0 && !mask_direct) {
         if ((rc = make_map(&tm, CU_TENSOR_MAP_DATA_TYPE_UINT8, packed, d * NM / 8, rows, d * NM / 8, C::MB, C::NJ,
                            CU_TENSOR_MAP_SWIZZLE_NONE)))

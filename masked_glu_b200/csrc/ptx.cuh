@@ -220,9 +220,12 @@ __device__ __forceinline__ uint32_t cluster_ctarank()
     return r;
 }
 
+// Every thread of every CTA of the cluster arrives; returns once all have
+// (release / acquire at cluster scope).  Not the .aligned form: callers may
+// reach it from divergent code.
 __device__ __forceinline__ void cluster_sync()
 {
-    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+    asm volatile("barrier.cluster.arrive.release;\n\tbarrier.cluster.wait.acquire;" ::: "memory");
 }
 
 // Address of the same shared-memory location in CTA `rank` of this cluster.
@@ -231,16 +234,6 @@ __device__ __forceinline__ uint32_t mapa_shared(uint32_t addr, uint32_t rank)
     uint32_t r;
     asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(rank));
     return r;
-}
-
-__device__ __forceinline__ float4 ld_shared_cluster_f4(uint32_t addr)
-{
-    float4 v;
-    asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
-                 : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
-                 : "r"(addr)
-                 : "memory");
-    return v;
 }
 
 // ---------------------------------------------------------------- bit tricks
@@ -331,6 +324,86 @@ __device__ __forceinline__ uint64_t sw128_kmajor_desc(uint32_t smem_addr)
     desc |= (uint64_t)1 << 46;                        // descriptor version (sm_100)
     desc |= (uint64_t)2 << 61;                        // layout: 128-byte swizzle
     return desc;
+}
+
+// ---------------------------------------------------------------- CTA pairs (cta_group::2)
+// A pair of CTAs in a cluster of two: one MMA issued by the first (rank 0)
+// computes a 256-row tile whose A rows and B columns are split between the two
+// CTAs' shared memories and whose accumulator rows live in both CTAs' TMEM.
+
+// The address of this CTA's shared-memory location `p` in CTA `rank` of the
+// cluster (same offset), for remote mbarrier arrivals and TMA barriers.
+__device__ __forceinline__ uint32_t cluster_addr(const void *p, uint32_t rank)
+{
+    return mapa_shared(smem_u32(p), rank);
+}
+
+// Arrive on an mbarrier of a CTA of the cluster (default semantics: release
+// at CTA scope).  Used to hand over data the arriving thread wrote into its
+// OWN CTA's shared memory (made visible to the async proxy by a proxy fence
+// first) to the peer CTA's MMA issuer, whose tensor-core reads go to that
+// same shared memory; and to return an accumulator after its tcgen05.ld's
+// completed.  A release at cluster scope would add a memory barrier per
+// arrival that waits for the SM's TMA traffic (the builders of the CTA-pair
+// kernel stalled on it: 1.09 ms instead of 0.60 ms for 4096 tokens, d = 2048,
+// h = 8192, n_m = 4 on B200).
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_bar)
+{
+    asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(cluster_bar) : "memory");
+}
+
+// 2-D tile load into this CTA's shared memory that completes its bytes on
+// `leader_bar` (a cluster address, normally the pair's first CTA's barrier).
+__device__ __forceinline__ void tma_load_2d_pair(void *smem_dst, const CUtensorMap *map, uint32_t leader_bar,
+                                                 int c0, int c1)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, "
+        "%4}], [%2];" ::"r"(smem_u32(smem_dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(leader_bar), "r"(c0), "r"(c1)
+        : "memory");
+}
+
+__device__ __forceinline__ void tmem_alloc_pair(uint32_t *dst_smem, uint32_t ncols)
+{
+    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(dst_smem)),
+                 "r"(ncols)
+                 : "memory");
+}
+
+__device__ __forceinline__ void tmem_relinquish_pair()
+{
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ void tmem_dealloc_pair(uint32_t taddr, uint32_t ncols)
+{
+    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+
+// The pair's MMA, issued by the first CTA: D (both CTAs' TMEM, their own A
+// rows) (+)= A (each CTA's shared memory, same offset) * B (columns split
+// between the two CTAs' shared memories, same offset).
+__device__ __forceinline__ void umma_f16_ss_pair(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                                 uint32_t accumulate)
+{
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+// Arrive on the mbarrier at `bar`'s offset in every CTA of `cta_mask` once all
+// previously issued pair MMAs of this thread have completed.
+__device__ __forceinline__ void umma_commit_pair(uint64_t *bar, uint16_t cta_mask)
+{
+    asm volatile(
+        "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(
+            smem_u32(bar)),
+        "h"(cta_mask)
+        : "memory");
 }
 
 // Instruction descriptor, kind::f16: bf16 A and B, f32 accumulator, both

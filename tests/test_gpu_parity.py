@@ -128,6 +128,28 @@ def test_prefill_parity(n_m, T, d, h):
     assert_close(got, ref, "bf16", f"prefill n_m={n_m} T={T} d={d} h={h}")
 
 
+# More than 128 tokens with 16-byte strided packed rows run on CTA pairs (256
+# tokens per tile; each CTA of a pair holds half of every weight block).
+# Cases where the second CTA of the last token tile has no valid token, where
+# the last weight tile ends inside the first CTA's half, and several pair tiles
+# per CTA pair.
+PAIR_CASES = [
+    (8, 257, 256, 50),
+    (4, 385, 192, 121),
+    (2, 700, 128, 97),
+    (1, 640, 320, 200),
+    (4, 2100, 128, 1000),
+]
+
+
+@pytest.mark.parametrize("n_m,T,d,h", PAIR_CASES)
+def test_prefill_pair_parity(n_m, T, d, h):
+    case = inputs.make_case(T, d, h, n_m, seed=330 + n_m + T + d + h)
+    got = run_forward(case, "swish")
+    ref, _ = oracle.forward(case.x.values, case.W.values, oracle_packed(case), n_m, ACT["swish"])
+    assert_close(got, ref, "bf16", f"prefill pair n_m={n_m} T={T} d={d} h={h}")
+
+
 @pytest.mark.parametrize("act", ACT_NAMES)
 def test_prefill_acts(act):
     case = inputs.make_case(160, 256, 96, 4, seed=401)

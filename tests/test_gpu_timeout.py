@@ -1,7 +1,8 @@
 """The bounded-wait failure path of the tensor-core kernel, driven on purpose
 in a test-only build of the library (libmglu_testhooks.so): there, every
 mbarrier wait gives up after 20 ms, and mglu_test_set_stall(1) makes the
-kernel's producer stop after the loads of its first stage.  Every load it did
+kernel's producer stop after the loads of its first stage (T = 300: the kernel
+on CTA pairs, both producers stop; T = 40: the one-CTA kernel).  Every load it did
 issue still lands and is waited for, every MMA issued is drained before TMEM
 is released, and every other wait of the CTA runs out, records
 MGLU_ERR_TIMEOUT in the device status word and returns.  No trap, no fault,
