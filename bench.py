@@ -13,9 +13,12 @@ is outside the timed region.
 The headline workload is the n_m = 8 decode layer (d = 4096, h = 14336, one
 token).  With no --workload given, the run then times the other workloads of
 the suite the same way and adds them to the same JSON line as sub-records
-(``workloads``): the n_m = 4 decode layer, the 4096-token prefill with Swish
-and with GELU, and the FFN block at 1 and 2048 tokens.  One JSON line is
-printed by rank 0.
+(``workloads``): the routed n_m = 8 decode step, the n_m = 4 decode layer,
+the 4096-token prefill with Swish, with GELU and with the dense gate, and the
+FFN block at 1 and 2048 tokens; then the training path's backward on the
+prefill layer (``training_backward``).  One JSON line is printed by rank 0.
+``gpu_launches`` counts this library's kernel launches per step with the
+library's own counter (``mglu_kernel_launches``).
 
 Inputs are seeded synthetic tensors with the workload's shapes.  To keep every
 timed launch reading HBM, each step uses the next of R device copies of
@@ -50,6 +53,7 @@ SUITE = [
     ("decode_d2048_h8192_nm4", 1, "swish"),
     ("prefill_T4096_d2048_h8192_nm4", 4096, "swish"),
     ("prefill_T4096_d2048_h8192_nm4", 4096, "gelu"),
+    ("prefill_T4096_d2048_h8192_nm4", 4096, "swish+dense_gate"),  # the dense-gate ablation
     ("ffn_d4096_h14336_nm8", 1, "swish"),
     ("ffn_d4096_h14336_nm8", 2048, "swish"),
 ]
@@ -469,6 +473,11 @@ def measure(args, dist, w, dev, *, sample_clocks):
     torch.cuda.synchronize(dev)
     if mglu.last_device_status() != 0:
         raise SystemExit(f"device status error during warm-up of {w['name']}")
+    # this library's kernel launches per step, counted by the library itself
+    n_before = mglu.kernel_launches()
+    step(0)
+    launches_per_step = mglu.kernel_launches() - n_before
+    torch.cuda.synchronize(dev)
 
     # The K timed steps are captured once as a CUDA graph and replayed: the
     # kernels run back to back (each may start its prologue while the
@@ -608,7 +617,7 @@ def measure(args, dist, w, dev, *, sample_clocks):
         "roofline": roof,
         "e2e": ({"value": e2e_value, "unit": "tok/s", "h2d_bytes_per_step": x_hs[0].numel() * x_hs[0].element_size(),
                  "d2h_bytes_per_step": res_hs[0].numel() * res_hs[0].element_size()} if e2e_value else None),
-        "gpu_launches": K * (2 if kind == "ffn" or routed else 1),
+        "gpu_launches": K * launches_per_step,
         "host_us_per_forward_call": host_us,
         "device_status": status,
         "rotating_copies": R,
@@ -629,6 +638,77 @@ def measure(args, dist, w, dev, *, sample_clocks):
     gc.collect()
     torch.cuda.empty_cache()
     return rec, extra
+
+
+def measure_backward(args, dist, dev):
+    """The training path's backward (straight-through gradients dx, dW and the
+    mask-logit gradients) on the prefill layer: K calls timed with CUDA events
+    around them on the launching stream, after the warm-up calls."""
+    import numpy as np
+    import torch
+
+    from masked_glu_b200 import inputs, mglu
+
+    w = workload_shape("prefill_T4096_d2048_h8192_nm4")
+    T, d, h, nm = w["T"], w["d"], w["h"], w["n_m"]
+    case = inputs.make_case(T, d, h, nm, seed=w["seed"] + 31 + 7919 * dist.rank)
+
+    def up(t):
+        return torch.from_numpy(t.storage.view(np.int16)).view(torch.bfloat16).to(dev)
+
+    x, W = up(case.x), up(case.W)
+    packed = mglu.pack_masks(torch.from_numpy(case.masks).to(dev))
+    del case
+    g = torch.Generator(device="cpu").manual_seed(w["seed"] + 37)
+    dout = torch.randn((T, h), generator=g).to(torch.bfloat16).to(dev)
+    ws = torch.empty(max(256, int(mglu.lib().mglu_backward_workspace_bytes(T, d, h, nm))), dtype=torch.uint8,
+                     device=dev)
+    for _ in range(args.warmup):
+        mglu.backward(x, W, packed, nm, dout, "swish", workspace=ws)
+    torch.cuda.synchronize(dev)
+    n_before = mglu.kernel_launches()
+    mglu.backward(x, W, packed, nm, dout, "swish", workspace=ws)
+    launches_per_step = mglu.kernel_launches() - n_before
+    torch.cuda.synchronize(dev)
+    if mglu.last_device_status() != 0:
+        raise SystemExit("device status error during the backward's warm-up")
+    K = args.steps
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    sampler = ClockSampler(dist.local)
+    sampler.start()
+    dist.barrier()
+    torch.cuda.synchronize(dev)
+    t0.record()
+    for _ in range(K):
+        mglu.backward(x, W, packed, nm, dout, "swish", workspace=ws)
+    t1.record()
+    torch.cuda.synchronize(dev)
+    dist.barrier()
+    clocks = sampler.stop()
+    ms = dist.max(t0.elapsed_time(t1), dev) / K
+    # the recomputed products, dx = G B over K = (n_m + 1) h, and the n_m + 1
+    # products E_i = G_i^T x: three contractions of 2 T d h (n_m + 1) each
+    flops = 3 * 2 * T * d * h * (nm + 1)
+    peaks, peak_src = load_peaks()
+    achieved = flops / (ms / 1000.0) / 1e12
+    rec = {
+        "value": dist.world * T / (ms / 1000.0), "unit": "tok/s", "ms_per_step": ms, "dtype": "bf16",
+        "config": {"workload": w["name"], "pass": "backward (dx, dW, mask-logit gradients)", "T": T, "d": d, "h": h,
+                   "n_m": nm, "act": "swish"},
+        "roofline": {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                     "frac": achieved / peaks["bf16_tflops"],
+                     "peak_source": f"{peak_src} bf16_tflops (burst)", "algorithmic_flops": flops,
+                     "note": "whole backward: the tensor-core recompute with the gradient epilogue, the masked "
+                             "operand, two cuBLAS GEMMs and the combine"},
+        "gpu_launches": K * launches_per_step,
+        "timing": "K eager calls between CUDA events on the launching stream",
+        "clocks": clocks,
+        "device_status": mglu.last_device_status(),
+    }
+    del x, W, packed, dout, ws
+    gc.collect()
+    torch.cuda.empty_cache()
+    return rec
 
 
 def tstar_sweep(args, dist, dev):
@@ -735,7 +815,9 @@ def run_mglu(args, dist):
             r, _ = measure(args, dist, ws, dev, sample_clocks=True)
             subs.append(r)
         line["workloads"] = subs
-        line["gpu_launches_all_workloads"] = line["gpu_launches"] + sum(r["gpu_launches"] for r in subs)
+        line["training_backward"] = measure_backward(args, dist, dev)
+        line["gpu_launches_all_workloads"] = (line["gpu_launches"] + sum(r["gpu_launches"] for r in subs) +
+                                              line["training_backward"]["gpu_launches"])
     if args.tstar_sweep:
         line["tstar_sweep"] = tstar_sweep(args, dist, dev)
 

@@ -362,6 +362,12 @@ int mglu_last_device_status(void *stream);
 /* Text of the last CUDA error seen by the library on this thread ("" if none). */
 const char *mglu_last_cuda_error(void);
 
+/* Number of kernels this library has launched in this process, over all
+ * threads and devices (a kernel recorded into a CUDA graph counts once, when
+ * it is recorded).  For counting the launches of a call: read it before and
+ * after.  Never fails. */
+uint64_t mglu_kernel_launches(void);
+
 /* Static text for an mglu_status value. */
 const char *mglu_status_string(int status);
 

@@ -35,10 +35,17 @@ int cuda_fail(cudaError_t e, const char *what)
     return MGLU_ERR_CUDA;
 }
 
+// Kernels this library has launched in this process (every launch ends in
+// check_launch); read with mglu_kernel_launches().
+std::atomic<uint64_t> g_kernel_launches{0};
+
 int check_launch(const char *what)
 {
     const cudaError_t e = cudaGetLastError();
-    return e == cudaSuccess ? MGLU_OK : cuda_fail(e, what);
+    if (e != cudaSuccess)
+        return cuda_fail(e, what);
+    g_kernel_launches.fetch_add(1, std::memory_order_relaxed);
+    return MGLU_OK;
 }
 
 bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
@@ -1033,6 +1040,8 @@ int mglu_last_device_status(void *stream)
 }
 
 const char *mglu_last_cuda_error(void) { return g_last_cuda_error; }
+
+uint64_t mglu_kernel_launches(void) { return g_kernel_launches.load(std::memory_order_relaxed); }
 
 #ifdef MGLU_TEST_HOOKS
 // Test-hook build only (not part of the product ABI): nonzero stops the

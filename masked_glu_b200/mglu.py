@@ -74,6 +74,7 @@ def lib() -> ctypes.CDLL:
             "mglu_last_device_status": (I32, [P]),
             "mglu_last_cuda_error": (ctypes.c_char_p, []),
             "mglu_status_string": (ctypes.c_char_p, [I32]),
+            "mglu_kernel_launches": (ctypes.c_uint64, []),
         }
         for name, (res, args) in sig.items():
             f = getattr(L, name)
@@ -367,3 +368,8 @@ def set_decode_max_tokens(t: int) -> int:
 
 def last_device_status(stream=None) -> int:
     return int(lib().mglu_last_device_status(_stream(stream)))
+
+
+def kernel_launches() -> int:
+    """Kernels the library has launched in this process so far."""
+    return int(lib().mglu_kernel_launches())

@@ -29,6 +29,15 @@ def test_exports_every_declared_symbol(L):
         assert f" T {n}" in out, n
 
 
+def test_kernel_launch_counter_counts_only_launches(L):
+    """The counter moves only when a kernel was launched: calls rejected on
+    the host (here: bad arguments, or no device at all) leave it as it was."""
+    before = mglu.kernel_launches()
+    assert before >= 0
+    assert L.mglu_forward(None, 1, 64, None, 64, None, 4, 0, 0, None, None, 0, None) != 0
+    assert mglu.kernel_launches() == before
+
+
 def test_status_strings(L):
     for s in (0, -1, -2, -3, -4, -5):
         assert mglu.status_string(s) and mglu.status_string(s) != "unknown status"

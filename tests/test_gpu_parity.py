@@ -150,6 +150,21 @@ def test_prefill_pair_parity(n_m, T, d, h):
     assert_close(got, ref, "bf16", f"prefill pair n_m={n_m} T={T} d={d} h={h}")
 
 
+@pytest.mark.parametrize("T,want", [(40, {1}), (200, {1}), (1, {1, 2})])
+def test_kernel_launch_counter(T, want):
+    """One tensor-core launch per forward (one CTA or a CTA pair); the decode
+    forward is its kernel plus, when CTAs share a row block, the split kernel."""
+    case = inputs.make_case(T, 512, 1000, 4, seed=350 + T)
+    x, W, packed, _ = device_case(case)
+    out = torch.empty((T, 1000), dtype=torch.bfloat16, device="cuda")
+    mglu.forward(x, W, packed, 4, "swish", out=out)
+    torch.cuda.synchronize()
+    before = mglu.kernel_launches()
+    mglu.forward(x, W, packed, 4, "swish", out=out)
+    torch.cuda.synchronize()
+    assert mglu.kernel_launches() - before in want
+
+
 @pytest.mark.parametrize("act", ACT_NAMES)
 def test_prefill_acts(act):
     case = inputs.make_case(160, 256, 96, 4, seed=401)
