@@ -288,9 +288,9 @@ int decode_nt(const void *x, int64_t T, int64_t d, const void *W, int64_t rows, 
 // The forward on CTA pairs (clusters of two, one 256-token MMA per k16 step
 // issued by the first CTA of each pair); the grid is as many pairs as fit at
 // once, each looping over tiles.
-template <int NM>
+template <int NM, bool GRAD>
 int launch_prefill_pair(const void *x, int64_t T, int64_t d, const void *W, int64_t rows, const uint8_t *packed,
-                        int act, void *out, cudaStream_t s, const float *mw, int dev)
+                        int act, void *out, cudaStream_t s, const float *mw, int dev, const void *dout, void *gout)
 {
     using C = mglu::pf::PairCfg<NM>;
     CUtensorMap tx, tw, tm;
@@ -304,7 +304,7 @@ int launch_prefill_pair(const void *x, int64_t T, int64_t d, const void *W, int6
     if ((rc = make_map(&tm, CU_TENSOR_MAP_DATA_TYPE_UINT8, packed, d * NM / 8, rows, d * NM / 8, C::MB, C::NJH,
                        CU_TENSOR_MAP_SWIZZLE_NONE)))
         return rc;
-    if ((rc = ensure_smem<mglu::pf::prefill_pair_kernel<NM>>(C::SMEM, dev)))
+    if ((rc = ensure_smem<mglu::pf::prefill_pair_kernel<NM, GRAD>>(C::SMEM, dev)))
         return rc;
     static std::atomic<int> max_pairs[kMaxDevices];
     int pairs = max_pairs[dev].load(std::memory_order_relaxed);
@@ -323,7 +323,7 @@ int launch_prefill_pair(const void *x, int64_t T, int64_t d, const void *W, int6
     if (pairs == 0) {
         cfg.gridDim = dim3((unsigned)(2 * sm_count(dev)));
         cfg.numAttrs = 1;
-        const cudaError_t e = cudaOccupancyMaxActiveClusters(&pairs, mglu::pf::prefill_pair_kernel<NM>, &cfg);
+        const cudaError_t e = cudaOccupancyMaxActiveClusters(&pairs, mglu::pf::prefill_pair_kernel<NM, GRAD>, &cfg);
         if (e != cudaSuccess)
             return cuda_fail(e, "cudaOccupancyMaxActiveClusters");
         if (pairs < 1)
@@ -334,8 +334,10 @@ int launch_prefill_pair(const void *x, int64_t T, int64_t d, const void *W, int6
     const int64_t grid_pairs = tiles < pairs ? tiles : pairs;
     cfg.gridDim = dim3((unsigned)(2 * grid_pairs));
     cfg.numAttrs = 2;
-    const cudaError_t e = cudaLaunchKernelEx(&cfg, mglu::pf::prefill_pair_kernel<NM>, tx, tw, tm, (int)T, (int)rows,
-                                             (int)d, act, reinterpret_cast<__nv_bfloat16 *>(out), mw);
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, mglu::pf::prefill_pair_kernel<NM, GRAD>, tx, tw, tm, (int)T,
+                                             (int)rows, (int)d, act, reinterpret_cast<__nv_bfloat16 *>(out), mw,
+                                             reinterpret_cast<const __nv_bfloat16 *>(dout),
+                                             reinterpret_cast<__nv_bfloat16 *>(gout));
     if (e != cudaSuccess)
         return cuda_fail(e, "prefill pair launch");
     return check_launch("prefill pair launch");
@@ -360,9 +362,9 @@ int launch_prefill(const void *x, int64_t T, int64_t d, const void *W, int64_t r
     // a tensor map needs 16-byte row strides; other packed rows are read by
     // the builder warps directly
     const int mask_direct = NM > 0 && (d * NM / 8) % 16 != 0;
-    if constexpr (NM > 0 && !GRAD) {
+    if constexpr (NM > 0) {
         if (!mask_direct && T > mglu::pf::BM)
-            return launch_prefill_pair<NM>(x, T, d, W, rows, packed, act, out, s, mw, dev);
+            return launch_prefill_pair<NM, GRAD>(x, T, d, W, rows, packed, act, out, s, mw, dev, dout, gout);
     }
     if (NM > 0 && !mask_direct) {
         if ((rc = make_map(&tm, CU_TENSOR_MAP_DATA_TYPE_UINT8, packed, d * NM / 8, rows, d * NM / 8, C::MB, C::NJ,

@@ -131,15 +131,17 @@ __device__ __forceinline__ void store8_bf16(__nv_bfloat16 *p, const float (&v)[8
 // v_i = D - g_i:
 //   block i < NM of gout:  dout (act'(g_i) v_i - act(g_i))
 //   block NM of gout:      sum_i dout act(g_i)
-// One mask at a time, 8 columns at a time, to keep registers low.
-template <int NM>
+// One mask at a time, 8 columns at a time, to keep registers low.  The tile's
+// NC columns start at weight row n0; block i of the accumulator starts BS
+// TMEM columns after block i - 1.
+template <int NM, int BS = Cfg<NM>::NJ, int NC = Cfg<NM>::NJ>
 __device__ __forceinline__ void grad_epilogue(uint32_t tbase, int tok, int T, int rows, int n0, int act,
                                               const __nv_bfloat16 *__restrict__ dout, __nv_bfloat16 *__restrict__ gout)
 {
-    using C = Cfg<NM>;
+    static_assert(NC % 8 == 0, "eight columns at a time");
     const int a = act & ACT_MASK;
     const int64_t gstride = (int64_t)(NM + 1) * rows;
-    for (int jc = 0; jc < C::NJ; jc += 8) {
+    for (int jc = 0; jc < NC; jc += 8) {
         const int j = n0 + jc;
         const int nv = tok < T ? (rows - j < 8 ? (rows - j > 0 ? rows - j : 0) : 8) : 0;
         const bool vec = (rows & 7) == 0;
@@ -157,7 +159,7 @@ __device__ __forceinline__ void grad_epilogue(uint32_t tbase, int tok, int T, in
 #pragma unroll 1
         for (int i = 0; i < NM; ++i) {
             uint32_t gv[8];
-            tmem_ld_x8(tbase + (1 + i) * C::NJ + jc, gv);
+            tmem_ld_x8(tbase + (1 + i) * BS + jc, gv);
             tmem_wait_ld();
             float ai[8];
 #pragma unroll

@@ -82,11 +82,14 @@ __device__ __forceinline__ void build_variants_pair(uint8_t *B, int off, uint4 w
 
 // mw: per-token mask weights [T][NM] (NULL: every weight 1).  The packed
 // rows must be 16-byte strided (a tensor map describes the mask tiles).
-template <int NM>
+// GRAD: the training path's epilogue (see grad_epilogue) into gout from the
+// loss gradient dout, instead of the forward's output.
+template <int NM, bool GRAD = false>
 __global__ void __launch_bounds__(PairCfg<NM>::NTHREADS, 1)
     prefill_pair_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_w,
                         const __grid_constant__ CUtensorMap tm_m, int T, int rows, int d, int act,
-                        __nv_bfloat16 *__restrict__ out, const float *__restrict__ mw)
+                        __nv_bfloat16 *__restrict__ out, const float *__restrict__ mw,
+                        const __nv_bfloat16 *__restrict__ dout, __nv_bfloat16 *__restrict__ gout)
 {
     using C = PairCfg<NM>;
     extern __shared__ uint8_t smem_raw[];
@@ -270,11 +273,17 @@ __global__ void __launch_bounds__(PairCfg<NM>::NTHREADS, 1)
             const int m0 = (tile % num_m) * C::BM2 + (int)rank * BM;
             const int n0 = (tile / num_m) * C::NJ;
             const int tok = m0 + 32 * q + lane;
+            const uint32_t tbase = tmem_base + ((uint32_t)(32 * q) << 16) + (uint32_t)(b * ACC_STRIDE);
+            if constexpr (GRAD) {
+                // both halves of the tile: CTA 0's weight rows, then CTA 1's
+                grad_epilogue<NM, C::NJH, C::NJH>(tbase, tok, T, rows, n0, act, dout, gout);
+                grad_epilogue<NM, C::NJH, C::NJH>(tbase + (uint32_t)C::NH, tok, T, rows, n0 + C::NJH, act, dout,
+                                                  gout);
+            } else {
             float wt[NM];
 #pragma unroll
             for (int i = 0; i < NM; ++i)
                 wt[i] = mw && tok < T ? mw[(int64_t)tok * NM + i] : 1.0f;
-            const uint32_t tbase = tmem_base + ((uint32_t)(32 * q) << 16) + (uint32_t)(b * ACC_STRIDE);
             __nv_bfloat16 *orow = out + (int64_t)tok * rows;
             const bool dense_gate = (act & GATE_DENSE) != 0;
             const int a = act & ACT_MASK;
@@ -326,6 +335,7 @@ __global__ void __launch_bounds__(PairCfg<NM>::NTHREADS, 1)
                         }
                     }
                 }
+            }
             }
             tc_fence_before();
             __syncwarp();
