@@ -301,9 +301,13 @@ int launch_prefill_pair(const void *x, int64_t T, int64_t d, const void *W, int6
     if ((rc = make_map(&tw, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, W, d, rows, d * 2, mglu::pf::BK, C::NJH,
                        CU_TENSOR_MAP_SWIZZLE_128B)))
         return rc;
-    if ((rc = make_map(&tm, CU_TENSOR_MAP_DATA_TYPE_UINT8, packed, d * NM / 8, rows, d * NM / 8, C::MB, C::NJH,
-                       CU_TENSOR_MAP_SWIZZLE_NONE)))
-        return rc;
+    if constexpr (NM > 0) {
+        if ((rc = make_map(&tm, CU_TENSOR_MAP_DATA_TYPE_UINT8, packed, d * NM / 8, rows, d * NM / 8, C::MB, C::NJH,
+                           CU_TENSOR_MAP_SWIZZLE_NONE)))
+            return rc;
+    } else {
+        tm = tw;  // not read
+    }
     if ((rc = ensure_smem<mglu::pf::prefill_pair_kernel<NM, GRAD>>(C::SMEM, dev)))
         return rc;
     static std::atomic<int> max_pairs[kMaxDevices];
@@ -362,7 +366,7 @@ int launch_prefill(const void *x, int64_t T, int64_t d, const void *W, int64_t r
     // a tensor map needs 16-byte row strides; other packed rows are read by
     // the builder warps directly
     const int mask_direct = NM > 0 && (d * NM / 8) % 16 != 0;
-    if constexpr (NM > 0) {
+    if constexpr (NM > 0 || !GRAD) {
         if (!mask_direct && T > mglu::pf::BM)
             return launch_prefill_pair<NM, GRAD>(x, T, d, W, rows, packed, act, out, s, mw, dev, dout, gout);
     }

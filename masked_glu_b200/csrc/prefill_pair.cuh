@@ -1,6 +1,7 @@
-// prefill_pair.cuh -- the many-token MGLU up-projection on CTA pairs
-// (tcgen05 cta_group::2): one MMA of 256 tokens x N columns per k16 step,
-// issued by the pair's first CTA.
+// prefill_pair.cuh -- the many-token MGLU up-projection (and the dense
+// product of the down-projection, NM = 0) on CTA pairs (tcgen05
+// cta_group::2): one MMA of 256 tokens x N columns per k16 step, issued by
+// the pair's first CTA.
 //
 // The 1-CTA kernel (prefill.cuh) is bound by shared-memory bandwidth: per
 // k-stage every CTA writes the x tile and the W tile by TMA, its builder warps
@@ -37,7 +38,6 @@ namespace pf {
 
 template <int NM>
 struct PairCfg {
-    static_assert(NM > 0, "the pair kernel builds masked operands");
     static constexpr int NJ = Cfg<NM>::NJ;       // weight rows of a column tile (both CTAs)
     static constexpr int NJH = NJ / 2;           // this CTA's half
     static constexpr int N = (NM + 1) * NJ;      // MMA columns
@@ -45,15 +45,16 @@ struct PairCfg {
     static constexpr int BM2 = 2 * BM;           // tokens of a pair tile
     static constexpr int A_BYTES = BM * BK * 2;  // 16 KB
     static constexpr int B_BYTES = NH * BK * 2;
-    static constexpr int MB = Cfg<NM>::MB;       // mask bytes per row per stage
+    static constexpr int MB = Cfg<NM>::MB;       // mask bytes per row per stage (0: the dense product)
     static constexpr int M_BYTES = NJH * MB;
     static constexpr int STAGE = (A_BYTES + B_BYTES + M_BYTES + 1023) / 1024 * 1024;
     static constexpr int STAGES = (227 * 1024 - 2048) / STAGE > 8 ? 8 : (227 * 1024 - 2048) / STAGE;
     static constexpr uint32_t W_TX = NJH * BK * 2;
     static constexpr int BAR_OFF = STAGES * STAGE;
     static constexpr int SMEM = BAR_OFF + 1024 + 1024;
-    // builders: NJH * 8 16-byte pieces of this CTA's W half per stage
-    static constexpr int ITEMS = NJH * 8;
+    // builders: NJH * 8 16-byte pieces of this CTA's W half per stage (none
+    // for the dense product)
+    static constexpr int ITEMS = NM == 0 ? 0 : NJH * 8;
     // one item per builder thread where that takes at most 10 warps, else two
     static constexpr int NBW = ITEMS / 32 <= 10 ? ITEMS / 32 : 8;
     static constexpr int EC = NJH % Cfg<NM>::EC == 0 ? Cfg<NM>::EC : 8;
@@ -64,6 +65,9 @@ struct PairCfg {
     static_assert(STAGES >= 3, "ring too shallow");
     static_assert(SMEM <= 227 * 1024, "shared memory");
     static_assert(ITEMS % 32 == 0 && ITEMS <= 2 * 32 * NBW, "builder items");
+    // the dense product's W tiles, like the x tiles, complete on CTA 0's
+    // barrier: the MMA waits for nothing else
+    static constexpr uint32_t LEADER_TX = NM == 0 ? 2u * (A_BYTES + W_TX) : 2u * A_BYTES;
 };
 
 template <int NM, int I>
@@ -118,7 +122,7 @@ __global__ void __launch_bounds__(PairCfg<NM>::NTHREADS, 1)
             mbar_init(&xfull[s], 1);
             mbar_init(&wfull[s], 1);
             mbar_init(&mfull[s], 1);
-            mbar_init(&built[s], 2 * C::NBW);
+            mbar_init(&built[s], C::NBW > 0 ? 2 * C::NBW : 1);  // unused by the dense product
             mbar_init(&empty[s], 1);
         }
         for (int b = 0; b < 2; ++b) {
@@ -165,22 +169,29 @@ __global__ void __launch_bounds__(PairCfg<NM>::NTHREADS, 1)
                     }
                     uint8_t *st = smem + s * C::STAGE;
                     if (rank == 0)
-                        mbar_arrive_expect_tx(&xfull[s], 2 * C::A_BYTES);  // both CTAs' x tiles
+                        mbar_arrive_expect_tx(&xfull[s], C::LEADER_TX);  // both CTAs' x (and dense W) tiles
                     tma_load_2d_pair(st, &tm_x, cluster_addr(&xfull[s], 0), kb * BK, m0);
-                    mbar_arrive_expect_tx(&wfull[s], C::W_TX);
-                    tma_load_2d(st + C::A_BYTES, &tm_w, &wfull[s], kb * BK, n0);
-                    const int mc = (kb * BK * NM / 8) / C::MB * C::MB;  // 16-byte aligned column
-                    mbar_arrive_expect_tx(&mfull[s], C::M_BYTES);
-                    tma_load_2d(st + C::A_BYTES + C::B_BYTES, &tm_m, &mfull[s], mc, n0);
+                    if constexpr (NM == 0) {
+                        tma_load_2d_pair(st + C::A_BYTES, &tm_w, cluster_addr(&xfull[s], 0), kb * BK, n0);
+                    } else {
+                        mbar_arrive_expect_tx(&wfull[s], C::W_TX);
+                        tma_load_2d(st + C::A_BYTES, &tm_w, &wfull[s], kb * BK, n0);
+                        const int mc = (kb * BK * NM / 8) / C::MB * C::MB;  // 16-byte aligned column
+                        mbar_arrive_expect_tx(&mfull[s], C::M_BYTES);
+                        tma_load_2d(st + C::A_BYTES + C::B_BYTES, &tm_m, &mfull[s], mc, n0);
+                    }
                 }
             }
             // Before the CTA may exit, every load issued has landed: its own W
-            // and mask tiles, and (counted on CTA 0's barrier) both x tiles.
+            // and mask tiles, and (counted on CTA 0's barrier, which CTA 0
+            // waits for before the closing cluster barrier) the pair-form loads.
             for (int j = it - C::STAGES < 0 ? 0 : it - C::STAGES; j < it; ++j) {
                 const int s = j % C::STAGES;
                 const uint32_t ph = (uint32_t)(j / C::STAGES) & 1u;
-                mbar_wait(&wfull[s], ph);
-                mbar_wait(&mfull[s], ph);
+                if constexpr (NM > 0) {
+                    mbar_wait(&wfull[s], ph);
+                    mbar_wait(&mfull[s], ph);
+                }
                 if (rank == 0)
                     mbar_wait(&xfull[s], ph);
             }
@@ -201,7 +212,7 @@ __global__ void __launch_bounds__(PairCfg<NM>::NTHREADS, 1)
                 for (int kb = 0; kb < nkb; ++kb, ++it) {
                     const int s = it % C::STAGES;
                     const uint32_t ph = (uint32_t)(it / C::STAGES) & 1u;
-                    if (!mbar_wait(&built[s], ph) || !mbar_wait(&xfull[s], ph)) {
+                    if ((NM > 0 && !mbar_wait(&built[s], ph)) || !mbar_wait(&xfull[s], ph)) {
                         ok = false;
                         break;
                     }
@@ -224,6 +235,7 @@ __global__ void __launch_bounds__(PairCfg<NM>::NTHREADS, 1)
         __syncwarp();
     } else if (warp < 2 + C::NBW) {
         // ---------------------------------------------------------- builders (both CTAs)
+        if constexpr (NM > 0) {
         const int bt = threadIdx.x - 64;  // 0 .. 32 * NBW - 1
         constexpr int MAXI = (C::ITEMS + 32 * C::NBW - 1) / (32 * C::NBW);
         const uint32_t built0 = cluster_addr(built, 0);
@@ -259,6 +271,7 @@ __global__ void __launch_bounds__(PairCfg<NM>::NTHREADS, 1)
                     mbar_arrive_cluster(built0 + (uint32_t)(s * 8));
             }
         }
+        }
     } else {
         // ---------------------------------------------------------- epilogue (both CTAs)
         const int q = warp & 3;  // TMEM lane quadrant this warp may access
@@ -279,6 +292,34 @@ __global__ void __launch_bounds__(PairCfg<NM>::NTHREADS, 1)
                 grad_epilogue<NM, C::NJH, C::NJH>(tbase, tok, T, rows, n0, act, dout, gout);
                 grad_epilogue<NM, C::NJH, C::NJH>(tbase + (uint32_t)C::NH, tok, T, rows, n0 + C::NJH, act, dout,
                                                   gout);
+            } else if constexpr (NM == 0) {
+                // the dense product: out = D
+                __nv_bfloat16 *orow = out + (int64_t)tok * rows;
+#pragma unroll 1
+                for (int half = 0; half < 2; ++half) {
+#pragma unroll 1
+                    for (int jc = 0; jc < C::NJH; jc += C::EC) {
+                        uint32_t dv[C::EC];
+#pragma unroll
+                        for (int h8 = 0; h8 < C::EC / 8; ++h8)
+                            tmem_ld_x8(tbase + (uint32_t)(half * C::NH + jc + 8 * h8),
+                                       *reinterpret_cast<uint32_t(*)[8]>(&dv[8 * h8]));
+                        tmem_wait_ld();
+                        const int j = n0 + half * C::NJH + jc;
+                        if (tok < T) {
+#pragma unroll
+                            for (int e = 0; e < C::EC; e += 8) {
+                                float v8[8];
+#pragma unroll
+                                for (int z = 0; z < 8; ++z)
+                                    v8[z] = __uint_as_float(dv[e + z]);
+                                const int nv = rows - (j + e) < 8 ? (rows - (j + e) > 0 ? rows - (j + e) : 0) : 8;
+                                if (nv > 0)
+                                    store8_bf16(orow + j + e, v8, nv, (rows & 7) == 0);
+                            }
+                        }
+                    }
+                }
             } else {
             float wt[NM];
 #pragma unroll

@@ -365,7 +365,7 @@ def test_widths_multiple_of_8(n_m, T, d, h):
     assert_close(got, ref, "bf16", f"d%8 n_m={n_m} T={T} d={d} h={h}")
 
 
-@pytest.mark.parametrize("T,h,d", [(1, 200, 40), (9, 72, 136), (40, 200, 72)])
+@pytest.mark.parametrize("T,h,d", [(1, 200, 40), (9, 72, 136), (40, 200, 72), (300, 200, 136)])
 def test_down_proj_h_multiple_of_8(T, h, d):
     rng = np.random.default_rng(1500 + T + h + d)
     hid = inputs.normal(rng, (T, h), 1.0, "bf16")
