@@ -150,6 +150,29 @@ def test_prefill_pair_parity(n_m, T, d, h):
     assert_close(got, ref, "bf16", f"prefill pair n_m={n_m} T={T} d={d} h={h}")
 
 
+@pytest.mark.parametrize("n_m,T,d,h", [(4, 1536, 1024, 3000), (8, 1024, 512, 2000), (1, 2048, 512, 1024)])
+def test_prefill_pair_repeatable(n_m, T, d, h):
+    """The CTA pairs hand data and accumulators across CTAs through mbarriers;
+    any missing ordering shows up as a run that differs.  Thirty back-to-back
+    runs must be bit-identical, and the first must match the oracle on an
+    exact sample of elements."""
+    case = inputs.make_case(T, d, h, n_m, seed=360 + n_m)
+    x, W, packed, _ = device_case(case)
+    first = torch.empty((T, h), dtype=torch.bfloat16, device="cuda")
+    mglu.forward(x, W, packed, n_m, "swish", out=first)
+    out = torch.empty_like(first)
+    for rep in range(30):
+        mglu.forward(x, W, packed, n_m, "swish", out=out)
+        torch.cuda.synchronize()
+        assert torch.equal(out, first), f"pair prefill n_m={n_m} repeat {rep} differs"
+    assert mglu.last_device_status() == 0
+    rng = np.random.default_rng(361 + n_m)
+    b = rng.integers(0, T, 2000)
+    j = rng.integers(0, h, 2000)
+    ref, _ = oracle.forward_elems(case.x.values, case.W.values, oracle_packed(case), n_m, ACT["swish"], b, j)
+    assert_close(to_f64(first)[b, j], ref, "bf16", f"pair prefill n_m={n_m} sampled")
+
+
 @pytest.mark.parametrize("T,want", [(40, {1}), (200, {1}), (1, {1, 2})])
 def test_kernel_launch_counter(T, want):
     """One tensor-core launch per forward (one CTA or a CTA pair); the decode
