@@ -25,6 +25,9 @@
 // the built stages (built, one arrival per builder warp of both CTAs) and the
 // drained accumulators (acc_empty, one arrival per epilogue warp of both).
 // The MMA's commits arrive on both CTAs' stage and accumulator barriers.
+// The dense instance (NM = 0) has no builders: both CTAs' W halves, like the
+// x tiles, come by the 2-SM TMA form onto CTA 0's barrier.  The GRAD instance
+// runs the training path's gradient epilogue on each half of the tile.
 #pragma once
 #include <cstdint>
 #include <cuda_bf16.h>
