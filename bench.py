@@ -456,8 +456,10 @@ def measure(args, dist, w, dev, *, sample_clocks):
         if ev is not None:
             ev[0].record()
         if routed:
-            mglu.route_topk(x, Wr, w["route_k"], "hard", weights=mw, scores=msc)
-            mglu.forward_weighted(x, Ws[r], pks[r], nm, mw, w["act"], out=out, scratch=scratch)
+            # the router and the weighted forward in one call (on the decode
+            # kernel the router runs inside it)
+            mglu.forward_routed(x, Ws[r], pks[r], nm, Wr, w["route_k"], "hard", w["act"], out=out, weights=mw,
+                                scores=msc, scratch=scratch)
         else:
             mglu.forward(x, Ws[r], pks[r], nm, w["act"], out=out, scratch=scratch)
         if ev is not None:

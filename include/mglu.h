@@ -192,6 +192,26 @@ int mglu_forward_weighted(const void *x, int64_t T, int64_t d, const void *W,
                           void *scratch, size_t scratch_bytes, void *stream);
 
 /*
+ * The routed forward in one call: the router of mglu_route_topk (same
+ * scores, same selection, same weights, bit for bit), then
+ * mglu_forward_weighted with those weights.  On the decode kernel (T up to
+ * the decode limit, MGLU_BF16) the router runs inside the forward kernel:
+ * every CTA routes the call's tokens itself while its first weight copies
+ * are in flight, so the step is one launch (plus the row-block finisher)
+ * instead of two; otherwise the two calls run in turn.
+ *   W_r [n_m][d], k, mode: as mglu_route_topk;
+ *   weights [T][n_m] float (required), scores [T][n_m] float (or NULL):
+ *   written, as mglu_route_topk writes them;
+ *   other arguments as mglu_forward_weighted.
+ * Errors: as mglu_route_topk and mglu_forward_weighted.
+ */
+int mglu_forward_routed(const void *x, int64_t T, int64_t d, const void *W,
+                        int64_t h, const uint8_t *packed, int n_m,
+                        const void *W_r, int k, int mode, int act, int dtype,
+                        float *weights, float *scores, void *out,
+                        void *scratch, size_t scratch_bytes, void *stream);
+
+/*
  * The partial sums behind mglu_forward's output, for checking the
  * decomposition ("Masked Gated Linear Unit", "Approach": each mask splits W
  * into a gate part M_i . W and a value part (1 - M_i) . W):

@@ -42,6 +42,7 @@
 
 #include "common.cuh"
 #include "ptx.cuh"
+#include "route.cuh"
 #include "sched.cuh"
 
 namespace mglu {
@@ -420,6 +421,18 @@ __global__ void __launch_bounds__(32) split_kernel(int rows, int d, int step, in
     }
 }
 
+// In-kernel routing (ROUTED instances).  When Wr is not NULL the kernel
+// scores and routes every token itself, with the arithmetic of route_kernel
+// (route_partial / route_select, so the weights equal mglu_route_topk's bit
+// for bit), before its stream starts; every CTA keeps its own copy of the
+// weights in shared memory, and CTA 0 also stores them (and the scores) for
+// the caller and for split_kernel.
+struct Router {
+    const __nv_bfloat16 *Wr;  // [NM][d]; NULL: the weights come in mw
+    int k, mode, vec;         // kept masks, ROUTE_HARD / ROUTE_SOFTMAX, 16-byte rows
+    float *weights, *scores;  // [T][NM] outputs (scores may be NULL)
+};
+
 // The decode kernel.  Scratch (global, caller-provided): this CTA's sums of
 // the first and the last row block of its range when other CTAs also hold
 // units of them (read by split_kernel); it needs no initialization.
@@ -432,7 +445,7 @@ template <int NM, int TT, bool ROUTED = false, int NW_ = DefaultShape<NM, TT>::N
 __global__ void __launch_bounds__(Layout<NM, TT, NW_>::NTHREADS, 1)
     decode_kernel(const __nv_bfloat16 *__restrict__ x, const __nv_bfloat16 *__restrict__ W,
                   const uint8_t *__restrict__ packed, int T, int rows, int d, int act, float *__restrict__ ws_part,
-                  __nv_bfloat16 *__restrict__ out, const float *__restrict__ mw, float *__restrict__ gv)
+                  __nv_bfloat16 *__restrict__ out, const float *__restrict__ mw, float *__restrict__ gv, Router ro)
 {
     using L = Layout<NM, TT, NW_>;
     constexpr int NT = L::NT;
@@ -456,14 +469,12 @@ __global__ void __launch_bounds__(Layout<NM, TT, NW_>::NTHREADS, 1)
     Shifts<NM> sh;
     sh.init(1u + ((uint32_t)act >> 16));  // act < 2^16: the value is 1
 
+    // the mask weights the epilogue reads: mw, or the kernel's own routing
+    // (computed below, after the first copies of the stream are issued)
+    __shared__ float s_mw[ROUTED ? 16 * (NM > 0 ? NM : 1) : 1];
+    const float *mwk = mw;
     // masks some token of the call weights
     uint32_t used = (1u << NM) - 1u;
-    if constexpr (ROUTED) {
-        uint32_t u = 0;
-        for (int e = lane; e < T * NM; e += 32)
-            u |= (mw[e] != 0.0f ? 1u : 0u) << (e % NM);
-        used = __reduce_or_sync(0xffffffffu, u);
-    }
 
     // Unit (rb, s) covers k = s * STEP + 32 u + [0, 32) for MMA units u of
     // rows rb * ROWS + [0, 16); this lane's 8 weights of MMA unit u start at
@@ -655,7 +666,7 @@ __global__ void __launch_bounds__(Layout<NM, TT, NW_>::NTHREADS, 1)
 #pragma unroll
                     for (int v = 0; v <= NM; ++v)
                         sums[v] = acc[v][t][r];
-                    write_output<NM, ROUTED>(sums, rb, row, tok, act, T, rows, out, mw, gv);
+                    write_output<NM, ROUTED>(sums, rb, row, tok, act, T, rows, out, mwk, gv);
                 }
             }
     };
@@ -679,6 +690,46 @@ __global__ void __launch_bounds__(Layout<NM, TT, NW_>::NTHREADS, 1)
             load_narrow(nmask, rb_c, s_c);
     }
 
+    // routing in the kernel, while the first copies are in flight
+    if constexpr (ROUTED) {
+        if (ro.Wr) {
+            // the token groups' warp sums go to the head slots, which no warp
+            // writes before its first segment ends
+            float(*part)[8][8] = reinterpret_cast<float(*)[8][8]>(slots);
+            constexpr int G = L::NTHREADS / 256;  // groups of 256 threads, one token each at a time
+            const int vt = threadIdx.x & 255, grp = threadIdx.x >> 8;
+            if (grp < G) {
+#pragma unroll 1
+                for (int t = grp; t < T; t += G) {
+                    float a8[8];
+                    route_partial<__nv_bfloat16>(x + (int64_t)t * d, d, ro.Wr, NM, ro.vec, vt, a8);
+                    if ((vt & 31) == 0)
+#pragma unroll
+                        for (int i = 0; i < 8; ++i)
+                            part[t][vt >> 5][i] = a8[i];
+                }
+            }
+            __syncthreads();
+            if (threadIdx.x < T) {
+                const int t = threadIdx.x;
+                route_select(part[t], NM, ro.k, ro.mode, &s_mw[t * NM],
+                             blockIdx.x == 0 && ro.scores ? ro.scores + (int64_t)t * NM : nullptr);
+                if (blockIdx.x == 0)
+#pragma unroll
+                    for (int i = 0; i < NM; ++i)
+                        ro.weights[(int64_t)t * NM + i] = s_mw[t * NM + i];
+            }
+            __syncthreads();
+            mwk = s_mw;
+        }
+    }
+
+    if constexpr (ROUTED) {
+        uint32_t u = 0;
+        for (int e = lane; e < T * NM; e += 32)
+            u |= (mwk[e] != 0.0f ? 1u : 0u) << (e % NM);
+        used = __reduce_or_sync(0xffffffffu, u);
+    }
     bool tail = false;  // the last segment is partial: its sums stay in acc
     for (int i = 0; i < n; ++i) {
         uint4 xv[L::UPW][NT];
@@ -754,7 +805,7 @@ __global__ void __launch_bounds__(Layout<NM, TT, NW_>::NTHREADS, 1)
     const int rb_last = pl.last_rb(blockIdx.x);
 #pragma unroll 1
     for (int rb = pl.first_rb(blockIdx.x) + warp; rb <= rb_last; rb += L::NW)
-        combine_cta<NM, TT, ROUTED>(rb, pl, slots, tails, act, T, rows, ws_part, out, mw, gv);
+        combine_cta<NM, TT, ROUTED>(rb, pl, slots, tails, act, T, rows, ws_part, out, mwk, gv);
 }
 
 // Scratch bytes of the decode kernel: two partial slots per CTA.

@@ -219,7 +219,7 @@ int launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, int smem, cudaSt
 // ------------------------------------------------------------------ decode
 template <int NM, int TT, bool ROUTED>
 int launch_decode(const void *x, int64_t T, int64_t d, const void *W, int64_t rows, const uint8_t *packed, int act,
-                  void *out, void *ws, cudaStream_t s, const float *mw, float *gv)
+                  void *out, void *ws, cudaStream_t s, const float *mw, float *gv, mglu::dec::Router ro)
 {
     using L = mglu::dec::Layout<NM, TT>;
     const int64_t rb = (rows + mglu::dec::ROWS - 1) / mglu::dec::ROWS;
@@ -241,7 +241,7 @@ int launch_decode(const void *x, int64_t T, int64_t d, const void *W, int64_t ro
     if ((rc = launch_pdl(mglu::dec::decode_kernel<NM, TT, ROUTED>, dim3((unsigned)grid), dim3(L::NTHREADS), L::SMEM, s,
                          "decode launch", reinterpret_cast<const __nv_bfloat16 *>(x),
                          reinterpret_cast<const __nv_bfloat16 *>(W), packed, (int)T, (int)rows, (int)d, act, ws_part, o,
-                         mw, gv)))
+                         mw, gv, ro)))
         return rc;
     // row blocks whose units several CTAs hold are finished by split_kernel
     mglu::dec::Plan pl;
@@ -256,32 +256,44 @@ int launch_decode(const void *x, int64_t T, int64_t d, const void *W, int64_t ro
     }
     if (!shared)
         return MGLU_OK;
+    // with routing in the kernel, CTA 0 has stored the weights for this kernel
+    const float *mw_split = ro.Wr ? ro.weights : mw;
     return launch_pdl(mglu::dec::split_kernel<NM, TT, ROUTED>, dim3((unsigned)grid), dim3(32), 0, s, "split launch",
-                      (int)rows, (int)d, L::STEP, (int)grid, L::NW, (int)T, act, (const float *)ws_part, o, mw, gv);
+                      (int)rows, (int)d, L::STEP, (int)grid, L::NW, (int)T, act, (const float *)ws_part, o, mw_split,
+                      gv);
 }
 
 // Token capacity by T: 2, 8 or 16 (the slots and the finisher's work follow
 // the call's T; the capacity fixes the MMA column blocks and shared memory).
 template <int NM, bool ROUTED>
 int decode_tt(const void *x, int64_t T, int64_t d, const void *W, int64_t rows, const uint8_t *packed, int act,
-              void *out, void *ws, cudaStream_t s, const float *mw, float *gv)
+              void *out, void *ws, cudaStream_t s, const float *mw, float *gv, mglu::dec::Router ro)
 {
     if (T <= 2)
-        return launch_decode<NM, 2, ROUTED>(x, T, d, W, rows, packed, act, out, ws, s, mw, gv);
+        return launch_decode<NM, 2, ROUTED>(x, T, d, W, rows, packed, act, out, ws, s, mw, gv, ro);
     if (T <= 8)
-        return launch_decode<NM, 8, ROUTED>(x, T, d, W, rows, packed, act, out, ws, s, mw, gv);
-    return launch_decode<NM, 16, ROUTED>(x, T, d, W, rows, packed, act, out, ws, s, mw, gv);
+        return launch_decode<NM, 8, ROUTED>(x, T, d, W, rows, packed, act, out, ws, s, mw, gv, ro);
+    return launch_decode<NM, 16, ROUTED>(x, T, d, W, rows, packed, act, out, ws, s, mw, gv, ro);
 }
 
 template <int NM>
 int decode_nt(const void *x, int64_t T, int64_t d, const void *W, int64_t rows, const uint8_t *packed, int act,
-              void *out, void *ws, cudaStream_t s, const float *mw, float *gv = nullptr)
+              void *out, void *ws, cudaStream_t s, const float *mw, float *gv = nullptr,
+              mglu::dec::Router ro = mglu::dec::Router{nullptr, 0, 0, 0, nullptr, nullptr})
 {
     if constexpr (NM > 0) {
-        if (mw)
-            return decode_tt<NM, true>(x, T, d, W, rows, packed, act, out, ws, s, mw, gv);
+        if (mw || ro.Wr)
+            return decode_tt<NM, true>(x, T, d, W, rows, packed, act, out, ws, s, mw, gv, ro);
     }
-    return decode_tt<NM, false>(x, T, d, W, rows, packed, act, out, ws, s, nullptr, gv);
+    return decode_tt<NM, false>(x, T, d, W, rows, packed, act, out, ws, s, nullptr, gv, ro);
+}
+
+// The routed forward on the decode kernel with the router inside it.
+template <int NM>
+int decode_routed(const void *x, int64_t T, int64_t d, const void *W, int64_t rows, const uint8_t *packed, int act,
+                  void *out, void *ws, cudaStream_t s, mglu::dec::Router ro)
+{
+    return decode_nt<NM>(x, T, d, W, rows, packed, act, out, ws, s, nullptr, nullptr, ro);
 }
 
 // ------------------------------------------------------------------ prefill
@@ -883,14 +895,50 @@ int mglu_route_topk(const void *x, int64_t T, int64_t d, const void *W_r, int n_
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     const int vec = d % 8 == 0 && aligned(x, 16) && aligned(W_r, 16);
     if (dtype == MGLU_BF16)
-        mglu::route_kernel<__nv_bfloat16><<<(unsigned)T, 256, 0, s>>>(
-            reinterpret_cast<const __nv_bfloat16 *>(x), T, d, reinterpret_cast<const __nv_bfloat16 *>(W_r), n_m, k,
-            mode, vec, weights, scores);
-    else
-        mglu::route_kernel<float><<<(unsigned)T, 256, 0, s>>>(reinterpret_cast<const float *>(x), T, d,
-                                                               reinterpret_cast<const float *>(W_r), n_m, k, mode, 0,
-                                                               weights, scores);
-    return check_launch("route launch");
+        return launch_pdl(mglu::route_kernel<__nv_bfloat16>, dim3((unsigned)T), dim3(256), 0, s, "route launch",
+                          reinterpret_cast<const __nv_bfloat16 *>(x), T, d,
+                          reinterpret_cast<const __nv_bfloat16 *>(W_r), n_m, k, mode, vec, weights, scores);
+    return launch_pdl(mglu::route_kernel<float>, dim3((unsigned)T), dim3(256), 0, s, "route launch",
+                      reinterpret_cast<const float *>(x), T, d, reinterpret_cast<const float *>(W_r), n_m, k, mode,
+                      0, weights, scores);
+}
+
+int mglu_forward_routed(const void *x, int64_t T, int64_t d, const void *W, int64_t h, const uint8_t *packed,
+                        int n_m, const void *W_r, int k, int mode, int act, int dtype, float *weights, float *scores,
+                        void *out, void *scratch, size_t scratch_bytes_, void *stream)
+{
+    int rc = check_forward(x, T, d, W, h, packed, n_m, act, dtype, out);
+    if (rc)
+        return rc;
+    if (mode != MGLU_ROUTE_HARD && mode != MGLU_ROUTE_SOFTMAX)
+        return MGLU_ERR_INVALID;
+    if (k < 0 || k > n_m)
+        return MGLU_ERR_INVALID;
+    if (T == 0)
+        return MGLU_OK;
+    if (!W_r || !weights)
+        return MGLU_ERR_INVALID;
+    const uintptr_t es = dtype == MGLU_BF16 ? 2 : 4;
+    if (!aligned(W_r, es) || !aligned(weights, 4) || (scores && !aligned(scores, 4)))
+        return MGLU_ERR_ALIGN;
+    if ((rc = check_scratch(T, dtype, h, scratch, scratch_bytes_)))
+        return rc;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (path_for(T, dtype) != MGLU_PATH_DECODE) {
+        // the router, then the weighted forward
+        if ((rc = mglu_route_topk(x, T, d, W_r, n_m, k, mode, dtype, weights, scores, stream)))
+            return rc;
+        return run_product(x, T, d, W, h, packed, n_m, act, dtype, out, scratch, s, weights);
+    }
+    const mglu::dec::Router ro{reinterpret_cast<const __nv_bfloat16 *>(W_r), k, mode,
+                               d % 8 == 0 && aligned(x, 16) && aligned(W_r, 16) ? 1 : 0, weights, scores};
+    switch (n_m) {
+    case 1: return decode_routed<1>(x, T, d, W, h, packed, act, out, scratch, s, ro);
+    case 2: return decode_routed<2>(x, T, d, W, h, packed, act, out, scratch, s, ro);
+    case 4: return decode_routed<4>(x, T, d, W, h, packed, act, out, scratch, s, ro);
+    case 8: return decode_routed<8>(x, T, d, W, h, packed, act, out, scratch, s, ro);
+    default: return MGLU_ERR_UNSUPPORTED;
+    }
 }
 
 int mglu_down_proj(const void *hid, int64_t T, int64_t h, const void *W_down, int64_t d, int dtype, void *y,

@@ -14,6 +14,8 @@
 #include <cstdint>
 #include <cuda_bf16.h>
 
+#include "ptx.cuh"
+
 namespace mglu {
 
 enum { ROUTE_HARD = 0, ROUTE_SOFTMAX = 1 };
@@ -36,19 +38,19 @@ __device__ __forceinline__ void acc8(float (&acc)[8], int n_m, const float (&xv)
         }
 }
 
+// The n_m partial scores of one token held by thread tid of a group of 256
+// (tid = 0..255; thread tid takes k8 = tid, tid + 256, ... of the 8-value
+// chunks, or k = tid, tid + 256, ... of single values), each summed
+// over the 32 lanes of its warp by a fixed xor tree (every lane ends with
+// its warp's sums).  The callers keep this order so that every copy of the
+// router gives the same scores bit for bit.
 template <typename E>
-__global__ void __launch_bounds__(256) route_kernel(const E *__restrict__ x, int64_t T, int64_t d,
-                                                    const E *__restrict__ Wr, int n_m, int k, int mode, int vec,
-                                                    float *__restrict__ weights, float *__restrict__ scores)
+__device__ __forceinline__ void route_partial(const E *__restrict__ xr, int64_t d, const E *__restrict__ Wr, int n_m,
+                                              int vec, int tid, float (&acc)[8])
 {
-    __shared__ float part[8][8];  // [warp][mask]
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int64_t t = blockIdx.x;
-    float acc[8];
 #pragma unroll
     for (int i = 0; i < 8; ++i)
         acc[i] = 0.0f;
-    const E *xr = x + t * d;
     if constexpr (sizeof(E) == 2) {
         if (vec) {  // d % 8 == 0 and 16-byte aligned rows: 8 values per load
             for (int64_t k8 = tid; k8 < d / 8; k8 += 256) {
@@ -85,18 +87,19 @@ __global__ void __launch_bounds__(256) route_kernel(const E *__restrict__ x, int
 #pragma unroll
         for (int i = 0; i < 8; ++i)
             acc[i] += __shfl_xor_sync(0xffffffffu, acc[i], off);
-    if (lane == 0)
-#pragma unroll
-        for (int i = 0; i < 8; ++i)
-            part[warp][i] = acc[i];
-    __syncthreads();
-    if (tid != 0)
-        return;
+}
+
+// From the 8 warps' sums part[w][i] of one token: the scores (summed over
+// the warps in order), the k kept masks and the token's mask weights w[i]
+// (scores into sc_out when not NULL).
+__device__ __forceinline__ void route_select(const float (*part)[8], int n_m, int k, int mode, float *w,
+                                             float *sc_out)
+{
     float sc[8];
     for (int i = 0; i < 8; ++i) {
         float v = 0.0f;
-        for (int w = 0; w < 8; ++w)
-            v += part[w][i];
+        for (int ww = 0; ww < 8; ++ww)
+            v += part[ww][i];
         sc[i] = v;
     }
     uint32_t sel = 0;
@@ -116,11 +119,35 @@ __global__ void __launch_bounds__(256) route_kernel(const E *__restrict__ x, int
     }
     for (int i = 0; i < n_m; ++i) {
         const bool kept = (sel >> i) & 1u;
-        const float w = !kept ? 0.0f : mode == ROUTE_SOFTMAX ? expf(sc[i] - m) / den : 1.0f;
-        weights[t * n_m + i] = w;
-        if (scores)
-            scores[t * n_m + i] = sc[i];
+        w[i] = !kept ? 0.0f : mode == ROUTE_SOFTMAX ? expf(sc[i] - m) / den : 1.0f;
+        if (sc_out)
+            sc_out[i] = sc[i];
     }
+}
+
+template <typename E>
+__global__ void __launch_bounds__(256) route_kernel(const E *__restrict__ x, int64_t T, int64_t d,
+                                                    const E *__restrict__ Wr, int n_m, int k, int mode, int vec,
+                                                    float *__restrict__ weights, float *__restrict__ scores)
+{
+    __shared__ float part[8][8];  // [warp][mask]
+    // The next kernel in the stream (the routed forward) may launch and set
+    // up now; it waits for this grid to complete before it reads anything.
+    // This grid in turn waits for the previous kernel before reading x.
+    pdl_launch_dependents();
+    pdl_wait();
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int64_t t = blockIdx.x;
+    float acc[8];
+    route_partial<E>(x + t * d, d, Wr, n_m, vec, tid, acc);
+    if (lane == 0)
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+            part[warp][i] = acc[i];
+    __syncthreads();
+    if (tid != 0)
+        return;
+    route_select(part, n_m, k, mode, weights + t * n_m, scores ? scores + t * n_m : nullptr);
 }
 
 }  // namespace mglu

@@ -62,6 +62,7 @@ def lib() -> ctypes.CDLL:
             "mglu_route_topk": (I32, [P, I64, I64, P, I32, I32, I32, I32, P, P, P]),
             "mglu_forward_weighted": (I32, [P, I64, I64, P, I64, P, I32, I32, I32, P, P, P, SZ, P]),
             "mglu_forward_partials": (I32, [P, I64, I64, P, I64, P, I32, P, P, SZ, P]),
+            "mglu_forward_routed": (I32, [P, I64, I64, P, I64, P, I32, P, I32, I32, I32, I32, P, P, P, P, SZ, P]),
             "mglu_workspace_bytes": (SZ, [I64, I64, I64, I32, I32]),
             "mglu_forward_down": (I32, [P, I64, I64, P, I64, P, I32, I32, I32, P, P, SZ, P, P]),
             "mglu_forward_decode_static": (I32, [P, I64, I64, P, I64, P, I32, I32, P, P]),
@@ -241,6 +242,33 @@ def forward_weighted(x: torch.Tensor, W: torch.Tensor, packed: torch.Tensor, n_m
                                        _ptr(mask_weights), _ptr(out), _ptr(scratch), _nbytes(scratch),
                                        _stream(stream)), "mglu_forward_weighted")
     return out
+
+
+def forward_routed(x: torch.Tensor, W: torch.Tensor, packed: torch.Tensor, n_m: int, W_r: torch.Tensor, k: int,
+                   mode="hard", act="swish", out: Optional[torch.Tensor] = None,
+                   weights: Optional[torch.Tensor] = None, scores: Optional[torch.Tensor] = None,
+                   scratch: Optional[torch.Tensor] = None, stream=None):
+    """route_topk then forward_weighted in one call (on the decode kernel the
+    router runs inside the forward kernel).  Returns (out, weights, scores)."""
+    T, d = x.shape
+    h = W.shape[0]
+    if W.shape[1] != d or W.dtype != x.dtype:
+        raise ValueError("W must be [h][d] with x's dtype")
+    if W_r.shape != (n_m, d) or W_r.dtype != x.dtype:
+        raise ValueError("W_r must be [n_m][d] with x's dtype")
+    if out is None:
+        out = torch.empty((T, h), dtype=x.dtype, device=x.device)
+    if weights is None:
+        weights = torch.empty((T, n_m), dtype=torch.float32, device=x.device)
+    if scores is None:
+        scores = torch.empty((T, n_m), dtype=torch.float32, device=x.device)
+    if scratch is None:
+        scratch = default_scratch(h, x.device)
+    _check(lib().mglu_forward_routed(_ptr(x), T, d, _ptr(W), h, _ptr(packed), n_m, _ptr(W_r), int(k),
+                                     ROUTE_MODES.get(mode, mode), _act(act), _dtype(x), _ptr(weights), _ptr(scores),
+                                     _ptr(out), _ptr(scratch), _nbytes(scratch), _stream(stream)),
+           "mglu_forward_routed")
+    return out, weights, scores
 
 
 def forward_partials(x: torch.Tensor, W: torch.Tensor, packed: torch.Tensor, n_m: int,

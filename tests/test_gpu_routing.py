@@ -95,3 +95,31 @@ def test_routed_forward_end_to_end(T, k, mode):
     want_w = routed.route_weights(s.cpu().numpy().astype(np.float64), k, mode)
     ref = routed.forward_weighted(case.x.values, case.W.values, case.masks, train.ACT_SWISH, want_w)
     assert_close(to_f64(out), ref, "bf16", f"routed T={T} k={k} {mode}")
+
+
+@pytest.mark.parametrize("n_m,T,d,h,k,mode", [(4, 1, 512, 160, 2, "hard"), (8, 2, 4096, 300, 2, "hard"),
+                                              (8, 5, 1024, 200, 1, "softmax"), (2, 16, 256, 96, 1, "hard"),
+                                              (1, 9, 200, 64, 1, "softmax"), (4, 40, 512, 160, 2, "softmax"),
+                                              (8, 1, 4096, 14336, 2, "hard")])
+def test_forward_routed_equals_router_then_weighted_forward(n_m, T, d, h, k, mode):
+    """The routed forward in one call (on the decode kernel: the router inside
+    the forward kernel, every CTA routing the tokens itself) gives the same
+    weights, scores and output, bit for bit, as mglu_route_topk followed by
+    mglu_forward_weighted; and the output matches the oracle's routed forward
+    with those weights."""
+    case = inputs.make_case(T, d, h, n_m, seed=2800 + n_m + T)
+    _, Wr = _router_case(T, d, n_m, seed=2801 + T)
+    x, W, packed, _ = device_case(case)
+    Wr_d = to_device(Wr)
+    w_ref, s_ref = mglu.route_topk(x, Wr_d, k, mode)
+    out_ref = mglu.forward_weighted(x, W, packed, n_m, w_ref)
+    out, w, s = mglu.forward_routed(x, W, packed, n_m, Wr_d, k, mode)
+    torch.cuda.synchronize()
+    assert mglu.last_device_status() == 0
+    assert torch.equal(w, w_ref), "weights differ from mglu_route_topk"
+    assert torch.equal(s, s_ref), "scores differ from mglu_route_topk"
+    assert torch.equal(out, out_ref), "output differs from the two-call routed forward"
+    if h * d <= 1 << 22:
+        ref = routed.forward_weighted(case.x.values, case.W.values, case.masks, train.ACT_SWISH,
+                                      w.cpu().numpy().astype(np.float64))
+        assert_close(to_f64(out), ref, "bf16", f"forward_routed n_m={n_m} T={T}")
