@@ -694,7 +694,8 @@ __global__ void __launch_bounds__(Layout<NM, TT, NW_>::NTHREADS, 1)
     if constexpr (ROUTED) {
         if (ro.Wr) {
             // the token groups' warp sums go to the head slots, which no warp
-            // writes before its first segment ends
+            // writes before its first segment ends (T * 64 floats; the slots
+            // hold NW * (NM + 1) * 16 * TT >= 256 * TT of them)
             float(*part)[8][8] = reinterpret_cast<float(*)[8][8]>(slots);
             constexpr int G = L::NTHREADS / 256;  // groups of 256 threads, one token each at a time
             const int vt = threadIdx.x & 255, grp = threadIdx.x >> 8;
