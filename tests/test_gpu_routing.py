@@ -123,3 +123,24 @@ def test_forward_routed_equals_router_then_weighted_forward(n_m, T, d, h, k, mod
         ref = routed.forward_weighted(case.x.values, case.W.values, case.masks, train.ACT_SWISH,
                                       w.cpu().numpy().astype(np.float64))
         assert_close(to_f64(out), ref, "bf16", f"forward_routed n_m={n_m} T={T}")
+
+
+@pytest.mark.parametrize("T,k,dtype", [(3, 0, "bf16"), (4, 4, "bf16"), (40, 2, "bf16"), (5, 2, "f32")])
+def test_forward_routed_edges(T, k, dtype):
+    """k = 0 (no mask kept: every output 0), k = n_m (every mask kept), the
+    tensor-core path (T = 40) and the fp32 path: the one call equals the
+    router followed by the weighted forward."""
+    n_m, d, h = 4, 256, 96
+    case = inputs.make_case(T, d, h, n_m, seed=2900 + T + k, dtype=dtype)
+    _, Wr = _router_case(T, d, n_m, seed=2901 + T, dtype=dtype)
+    x, W, packed, _ = device_case(case)
+    Wr_d = to_device(Wr)
+    w_ref, s_ref = mglu.route_topk(x, Wr_d, k, "softmax")
+    out_ref = mglu.forward_weighted(x, W, packed, n_m, w_ref)
+    out, w, s = mglu.forward_routed(x, W, packed, n_m, Wr_d, k, "softmax")
+    torch.cuda.synchronize()
+    assert mglu.last_device_status() == 0
+    assert torch.equal(w, w_ref) and torch.equal(s, s_ref)
+    assert torch.equal(out, out_ref)
+    if k == 0:
+        assert not torch.any(out.float() != 0)
