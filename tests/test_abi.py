@@ -109,6 +109,27 @@ def test_forward_rejects_bad_arguments(L):
     assert L.mglu_scratch_bytes(14336) == L.mglu_scratch_bytes(16)
 
 
+def routed(L, x=A, T=1, d=128, W=A, h=16, pk=A, n_m=8, Wr=A, k=2, mode=0, act=0, dtype=0, w=A, sc=A, out=A, ws=A,
+           wsb=1 << 30):
+    return L.mglu_forward_routed(x, T, d, W, h, pk, n_m, Wr, k, mode, act, dtype, w, sc, out, ws, wsb, None)
+
+
+def test_forward_routed_rejects_bad_arguments(L):
+    """Every call below fails validation before any launch."""
+    assert routed(L, n_m=3) == mglu.ERR_UNSUPPORTED
+    assert routed(L, mode=2) == mglu.ERR_INVALID
+    assert routed(L, k=9) == mglu.ERR_INVALID
+    assert routed(L, k=-1) == mglu.ERR_INVALID
+    assert routed(L, Wr=None) == mglu.ERR_INVALID
+    assert routed(L, w=None) == mglu.ERR_INVALID
+    assert routed(L, x=None) == mglu.ERR_INVALID
+    assert routed(L, Wr=A + 1) == mglu.ERR_ALIGN
+    assert routed(L, w=A + 2) == mglu.ERR_ALIGN
+    assert routed(L, sc=A + 2) == mglu.ERR_ALIGN
+    assert routed(L, ws=None) == mglu.ERR_INVALID   # the decode path needs its scratch
+    assert routed(L, T=0) == mglu.OK                # nothing to do
+
+
 def test_forward_zero_tokens_is_a_noop(L):
     # T == 0 returns before any device work, even with no x / out
     assert fwd(L, T=0, x=None, out=None) == mglu.OK
