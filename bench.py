@@ -78,6 +78,8 @@ def parse_args(argv=None):
     ap.add_argument("--no-comparisons", action="store_true",
                     help="skip the torch.matmul baselines (dense SwiGLU, naive MGLU) timed after the run")
     ap.add_argument("--no-suite", action="store_true", help="time the headline workload only")
+    ap.add_argument("--backward-only", action="store_true",
+                    help="time only the training backward on the prefill layer and print its record")
     ap.add_argument("--tstar-sweep", action="store_true",
                     help="also time the FFN block for T in 8..64 with the decode kernel allowed up to 16 tokens "
                          "and with every T on the tensor-core kernel")
@@ -790,6 +792,13 @@ def run_mglu(args, dist):
     mglu.lib()
     mglu.set_decode_max_tokens(16)
 
+    if args.backward_only:
+        rec = measure_backward(args, dist, dev)
+        if dist.rank == 0:
+            print(json.dumps(dict(rec, metric="MGLU training backward TFLOP/s vs B200 bf16 roofline",
+                                  n_gpus=dist.world, steps=args.steps, warmup=args.warmup)), flush=True)
+        dist.close()
+        return
     w = workload_shape(args.workload, args.tokens, args.act, args.p)
     rec, extra = measure(args, dist, w, dev, sample_clocks=True)
     line = {"metric": METRIC, "value": rec["value"], "unit": "tok/s", "n_gpus": dist.world, "steps": args.steps,
