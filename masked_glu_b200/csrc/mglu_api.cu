@@ -304,7 +304,7 @@ template <int NM, bool GRAD>
 int launch_prefill_pair(const void *x, int64_t T, int64_t d, const void *W, int64_t rows, const uint8_t *packed,
                         int act, void *out, cudaStream_t s, const float *mw, int dev, const void *dout, void *gout)
 {
-    using C = mglu::pf::PairCfg<NM>;
+    using C = mglu::pf::PairCfg<NM, GRAD>;
     CUtensorMap tx, tw, tm;
     int rc;
     if ((rc = make_map(&tx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, x, d, T, d * 2, mglu::pf::BK, mglu::pf::BM,

@@ -16,8 +16,9 @@
 //
 // The MMA's N columns are CTA 0's half-blocks followed by CTA 1's:
 //   [D_a, g_1a, ..., g_NMa, D_b, g_1b, ..., g_NMb],  a / b = rows n0 + [0, NJ/2)
-// and n0 + [NJ/2, NJ) of W; each CTA's TMEM holds those N columns for its 128
-// tokens, and its epilogue writes its tokens' outputs for all NJ columns.
+// and n0 + [NJ/2, NJ) of W (each half padded with zero rows to whole 8-row
+// swizzle atoms); each CTA's TMEM holds those N columns for its 128 tokens,
+// and its epilogue writes its tokens' outputs for all NJ columns.
 //
 // Roles per CTA (warp 0 TMA producer, warp 1 TMEM and, in CTA 0, the MMA
 // issuer, NBW builder warps, 4 epilogue warps).  Barriers that both CTAs
@@ -39,15 +40,24 @@
 namespace mglu {
 namespace pf {
 
-template <int NM>
+template <int NM, bool GRAD = false>
 struct PairCfg {
-    static constexpr int NJ = Cfg<NM>::NJ;       // weight rows of a column tile (both CTAs)
+    // weight rows of a column tile (both CTAs).  At n_m = 8 the forward takes
+    // 28: nine blocks of 14 rows per CTA, padded by two zero rows, fill
+    // N = 256.  With the 1-CTA kernel's 16 rows the MMA is only N = 144 wide
+    // and the x tile, whose shared-memory writes and reads are fixed per k16
+    // step, dominates the shared-memory traffic.  The gradient epilogue reads
+    // 8-column blocks and keeps 16.
+    static constexpr int NJ = NM == 8 && !GRAD ? 28 : Cfg<NM>::NJ;
     static constexpr int NJH = NJ / 2;           // this CTA's half
-    static constexpr int N = (NM + 1) * NJ;      // MMA columns
     static constexpr int NH = (NM + 1) * NJH;    // B rows in this CTA
+    static constexpr int NHP = (NH + 7) / 8 * 8; // ... padded to whole 8-row swizzle atoms
+    static constexpr int N = 2 * NHP;            // MMA columns
+    // the variant blocks do not start on 8-column (TMEM) / 8-row boundaries
+    static constexpr bool RAGGED = NJH % 8 != 0;
     static constexpr int BM2 = 2 * BM;           // tokens of a pair tile
     static constexpr int A_BYTES = BM * BK * 2;  // 16 KB
-    static constexpr int B_BYTES = NH * BK * 2;
+    static constexpr int B_BYTES = NHP * BK * 2;
     static constexpr int MB = Cfg<NM>::MB;       // mask bytes per row per stage (0: the dense product)
     static constexpr int M_BYTES = NJH * MB;
     static constexpr int STAGE = (A_BYTES + B_BYTES + M_BYTES + 1023) / 1024 * 1024;
@@ -59,22 +69,25 @@ struct PairCfg {
     // for the dense product)
     static constexpr int ITEMS = NM == 0 ? 0 : NJH * 8;
     // one item per builder thread where that takes at most 10 warps, else two
-    static constexpr int NBW = ITEMS / 32 <= 10 ? ITEMS / 32 : 8;
+    static constexpr int NBW = (ITEMS + 31) / 32 <= 10 ? (ITEMS + 31) / 32 : 8;
     static constexpr int EC = NJH % Cfg<NM>::EC == 0 ? Cfg<NM>::EC : 8;
     static constexpr int NTHREADS = (2 + NBW + 4) * 32;
-    static_assert(NJH % 8 == 0, "a half block starts on a swizzle atom");
+    static_assert(!RAGGED || (NM > 0 && !GRAD), "only the forward act-sum epilogue reads ragged blocks");
+    static_assert(RAGGED || NJH % EC == 0, "epilogue chunking");
     static_assert(N <= 256 && N % 16 == 0, "UMMA shape for M = 256");
-    static_assert(NJH % EC == 0, "epilogue chunking");
     static_assert(STAGES >= 3, "ring too shallow");
     static_assert(SMEM <= 227 * 1024, "shared memory");
-    static_assert(ITEMS % 32 == 0 && ITEMS <= 2 * 32 * NBW, "builder items");
+    static_assert(ITEMS <= 2 * 32 * NBW, "builder items");
     // the dense product's W tiles, like the x tiles, complete on CTA 0's
     // barrier: the MMA waits for nothing else
     static constexpr uint32_t LEADER_TX = NM == 0 ? 2u * (A_BYTES + W_TX) : 2u * A_BYTES;
 };
 
-template <int NM, int I>
-__device__ __forceinline__ void build_variants_pair(uint8_t *B, int off, uint4 w, uint32_t lo, uint32_t hi)
+// Variant I of W piece (r, c) goes to stacked row (1 + I) * NJH + r, at the
+// 16-byte column its row's 128-byte swizzle gives (the stage is 1024-byte
+// aligned, so the swizzle row is the stacked row mod 8).
+template <int NM, int NJH, int I>
+__device__ __forceinline__ void build_variants_pair(uint8_t *B, int r, int c, uint4 w, uint32_t lo, uint32_t hi)
 {
     if constexpr (I < NM) {
         uint4 m;
@@ -82,8 +95,9 @@ __device__ __forceinline__ void build_variants_pair(uint8_t *B, int off, uint4 w
         m.y = w.y & pair_mask<NM, 1, I>(lo, hi);
         m.z = w.z & pair_mask<NM, 2, I>(lo, hi);
         m.w = w.w & pair_mask<NM, 3, I>(lo, hi);
-        *reinterpret_cast<uint4 *>(B + (1 + I) * PairCfg<NM>::NJH * 128 + off) = m;
-        build_variants_pair<NM, I + 1>(B, off, w, lo, hi);
+        const int R = (1 + I) * NJH + r;
+        *reinterpret_cast<uint4 *>(B + R * 128 + ((c ^ (R & 7)) << 4)) = m;
+        build_variants_pair<NM, NJH, I + 1>(B, r, c, w, lo, hi);
     }
 }
 
@@ -92,13 +106,13 @@ __device__ __forceinline__ void build_variants_pair(uint8_t *B, int off, uint4 w
 // GRAD: the training path's epilogue (see grad_epilogue) into gout from the
 // loss gradient dout, instead of the forward's output.
 template <int NM, bool GRAD = false>
-__global__ void __launch_bounds__(PairCfg<NM>::NTHREADS, 1)
+__global__ void __launch_bounds__(PairCfg<NM, GRAD>::NTHREADS, 1)
     prefill_pair_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_w,
                         const __grid_constant__ CUtensorMap tm_m, int T, int rows, int d, int act,
                         __nv_bfloat16 *__restrict__ out, const float *__restrict__ mw,
                         const __nv_bfloat16 *__restrict__ dout, __nv_bfloat16 *__restrict__ gout)
 {
-    using C = PairCfg<NM>;
+    using C = PairCfg<NM, GRAD>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t *xfull = reinterpret_cast<uint64_t *>(smem + C::BAR_OFF);  // CTA 0's: both x tiles landed
@@ -134,6 +148,16 @@ __global__ void __launch_bounds__(PairCfg<NM>::NTHREADS, 1)
         }
         mbar_init(drain, 1);
         fence_mbar_init();
+    }
+    if constexpr (C::NHP > C::NH) {
+        // the pad rows of the stacked operand are never loaded or built:
+        // zero them once, for the tensor core (async proxy) to read
+        constexpr int PIECES = (C::NHP - C::NH) * 8;
+        for (int i = threadIdx.x; i < C::STAGES * PIECES; i += C::NTHREADS) {
+            uint8_t *B = smem + (i / PIECES) * C::STAGE + C::A_BYTES;
+            *reinterpret_cast<uint4 *>(B + (C::NH + (i % PIECES) / 8) * 128 + (i % 8) * 16) = make_uint4(0, 0, 0, 0);
+        }
+        fence_proxy_async_smem();
     }
     if (warp == 1) {
         tmem_alloc_pair(tmem_slot, TMEM_COLS);
@@ -261,11 +285,10 @@ __global__ void __launch_bounds__(PairCfg<NM>::NTHREADS, 1)
                     const int item = bt + q * 32 * C::NBW;
                     if (item < C::ITEMS) {
                         const int r = item >> 3, c = item & 7;
-                        const int off = r * 128 + ((c ^ (r & 7)) << 4);
-                        const uint4 w = *reinterpret_cast<const uint4 *>(B + off);
+                        const uint4 w = *reinterpret_cast<const uint4 *>(B + r * 128 + ((c ^ (r & 7)) << 4));
                         uint32_t lo, hi;
                         load_mask_bytes<NM>(Mt + r * C::MB + moff + c * NM, lo, hi);
-                        build_variants_pair<NM, 0>(B, off, w, lo, hi);
+                        build_variants_pair<NM, C::NJH, 0>(B, r, c, w, lo, hi);
                     }
                 }
                 fence_proxy_async_smem();  // generic-proxy writes -> visible to the tensor core
@@ -293,7 +316,7 @@ __global__ void __launch_bounds__(PairCfg<NM>::NTHREADS, 1)
             if constexpr (GRAD) {
                 // both halves of the tile: CTA 0's weight rows, then CTA 1's
                 grad_epilogue<NM, C::NJH, C::NJH>(tbase, tok, T, rows, n0, act, dout, gout);
-                grad_epilogue<NM, C::NJH, C::NJH>(tbase + (uint32_t)C::NH, tok, T, rows, n0 + C::NJH, act, dout,
+                grad_epilogue<NM, C::NJH, C::NJH>(tbase + (uint32_t)C::NHP, tok, T, rows, n0 + C::NJH, act, dout,
                                                   gout);
             } else if constexpr (NM == 0) {
                 // the dense product: out = D
@@ -305,7 +328,7 @@ __global__ void __launch_bounds__(PairCfg<NM>::NTHREADS, 1)
                         uint32_t dv[C::EC];
 #pragma unroll
                         for (int h8 = 0; h8 < C::EC / 8; ++h8)
-                            tmem_ld_x8(tbase + (uint32_t)(half * C::NH + jc + 8 * h8),
+                            tmem_ld_x8(tbase + (uint32_t)(half * C::NHP + jc + 8 * h8),
                                        *reinterpret_cast<uint32_t(*)[8]>(&dv[8 * h8]));
                         tmem_wait_ld();
                         const int j = n0 + half * C::NJH + jc;
@@ -331,9 +354,51 @@ __global__ void __launch_bounds__(PairCfg<NM>::NTHREADS, 1)
             __nv_bfloat16 *orow = out + (int64_t)tok * rows;
             const bool dense_gate = (act & GATE_DENSE) != 0;
             const int a = act & ACT_MASK;
+            if constexpr (C::RAGGED) {
+#pragma unroll 1
+                for (int half = 0; half < 2; ++half) {
+                    // all NHP columns of the half in one round of loads: a
+                    // TMEM load waited for while the tensor core fills the
+                    // other accumulator takes long, and one wait per variant
+                    // block made this epilogue, not the MMA, set the pace
+                    const uint32_t hbase = tbase + (uint32_t)(half * C::NHP);
+                    uint32_t cols[C::NHP];
+#pragma unroll
+                    for (int c = 0; c < C::NHP / 8; ++c)
+                        tmem_ld_x8(hbase + (uint32_t)(8 * c), *reinterpret_cast<uint32_t(*)[8]>(&cols[8 * c]));
+                    tmem_wait_ld();
+                    float o[C::NJH];
+#pragma unroll
+                    for (int e = 0; e < C::NJH; ++e) {
+                        const float D = __uint_as_float(cols[e]);
+                        float acc = 0.f;
+#pragma unroll
+                        for (int i = 0; i < NM; ++i) {
+                            const float gi = __uint_as_float(cols[(1 + i) * C::NJH + e]);
+                            acc += wt[i] * (act_fn(a, dense_gate ? D : gi) * (D - gi));
+                        }
+                        o[e] = acc;
+                    }
+                    const int j = n0 + half * C::NJH;  // even: NJ and NJH are
+                    if (tok < T) {
+                        if ((rows & 1) == 0 && j + C::NJH <= rows &&
+                            (reinterpret_cast<uintptr_t>(orow) & 3) == 0) {
+#pragma unroll
+                            for (int e = 0; e < C::NJH; e += 2)
+                                *reinterpret_cast<__nv_bfloat162 *>(orow + j + e) =
+                                    __floats2bfloat162_rn(o[e], o[e + 1]);
+                        } else {
+#pragma unroll
+                            for (int e = 0; e < C::NJH; ++e)
+                                if (j + e < rows)
+                                    orow[j + e] = __float2bfloat16_rn(o[e]);
+                        }
+                    }
+                }
+            } else {
 #pragma unroll 1
             for (int half = 0; half < 2; ++half) {
-                const uint32_t hbase = tbase + (uint32_t)(half * C::NH);
+                const uint32_t hbase = tbase + (uint32_t)(half * C::NHP);
 #pragma unroll 1
                 for (int jc = 0; jc < C::NJH; jc += C::EC) {
                     float o[C::EC];
@@ -379,6 +444,7 @@ __global__ void __launch_bounds__(PairCfg<NM>::NTHREADS, 1)
                         }
                     }
                 }
+            }
             }
             }
             tc_fence_before();

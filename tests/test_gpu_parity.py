@@ -135,6 +135,12 @@ def test_prefill_parity(n_m, T, d, h):
 # per CTA pair.
 PAIR_CASES = [
     (8, 257, 256, 50),
+    # n_m = 8 pairs take 28 weight rows per tile (14 per CTA, padded to 16):
+    # a whole tile, one CTA's rows only, a 2-row tail, an odd h
+    (8, 300, 192, 28),
+    (8, 260, 64, 14),
+    (8, 513, 320, 30),
+    (8, 400, 128, 57),
     (4, 385, 192, 121),
     (2, 700, 128, 97),
     (1, 640, 320, 200),
@@ -432,6 +438,7 @@ def test_relu_is_homogeneous_of_degree_two(n_m, T):
 # ------------------------------------------------------------------ dense-gate ablation
 @pytest.mark.parametrize("n_m,T,d,h,dtype", [(4, 1, 512, 200, "bf16"), (8, 9, 256, 96, "bf16"),
                                              (4, 150, 384, 200, "bf16"), (1, 40, 256, 64, "bf16"),
+                                             (8, 300, 256, 90, "bf16"),
                                              (2, 5, 100, 37, "f32")])
 @pytest.mark.parametrize("act", ["swish", "gelu", "relu"])
 def test_dense_gate_matches_oracle(n_m, T, d, h, dtype, act):
