@@ -378,8 +378,12 @@ int launch_prefill(const void *x, int64_t T, int64_t d, const void *W, int64_t r
     // a tensor map needs 16-byte row strides; other packed rows are read by
     // the builder warps directly
     const int mask_direct = NM > 0 && (d * NM / 8) % 16 != 0;
+    // CTA pairs from two 128-token tiles on; the dense product (the
+    // down-projection) at any T: its pair kernel was faster on B200 at
+    // T = 24 and T = 128 as well (79 against 88 and 91 us at h = 14336,
+    // d = 4096), with the same accumulation order per k16 step
     if constexpr (NM > 0 || !GRAD) {
-        if (!mask_direct && T > mglu::pf::BM)
+        if (!mask_direct && (NM == 0 || T > mglu::pf::BM))
             return launch_prefill_pair<NM, GRAD>(x, T, d, W, rows, packed, act, out, s, mw, dev, dout, gout);
     }
     if (NM > 0 && !mask_direct) {
