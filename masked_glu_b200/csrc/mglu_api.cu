@@ -18,6 +18,7 @@
 #include "pack.cuh"
 #include "prefill.cuh"
 #include "prefill_pair.cuh"
+#include "prefill_wm.cuh"
 #include "ptx.cuh"
 #include "route.cuh"
 #include "simt.cuh"
@@ -359,6 +360,32 @@ int launch_prefill_pair(const void *x, int64_t T, int64_t d, const void *W, int6
     return check_launch("prefill pair launch");
 }
 
+template <int NM>
+int launch_prefill_wm(const void *x, int64_t T, int64_t d, const void *W, int64_t rows, const uint8_t *packed, int act,
+                      void *out, cudaStream_t s, const float *mw, int dev)
+{
+    using C = mglu::pf::WmCfg<NM>;
+    const int NT = (int)((T + 15) / 16 * 16);  // the MMA's N: tokens rounded up to 16
+    CUtensorMap tx, tw, tm;
+    int rc;
+    if ((rc = make_map(&tx, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, x, d, T, d * 2, mglu::pf::BK, NT,
+                       CU_TENSOR_MAP_SWIZZLE_128B)))
+        return rc;
+    if ((rc = make_map(&tw, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, W, d, rows, d * 2, mglu::pf::BK, C::NJ,
+                       CU_TENSOR_MAP_SWIZZLE_128B)))
+        return rc;
+    if ((rc = make_map(&tm, CU_TENSOR_MAP_DATA_TYPE_UINT8, packed, d * NM / 8, rows, d * NM / 8, C::MB, C::NJ,
+                       CU_TENSOR_MAP_SWIZZLE_NONE)))
+        return rc;
+    if ((rc = ensure_smem<mglu::pf::prefill_wm_kernel<NM>>(C::SMEM, dev)))
+        return rc;
+    const int64_t tiles = (rows + C::NJ - 1) / C::NJ;
+    const int grid = (int)(tiles < sm_count(dev) ? tiles : sm_count(dev));
+    return launch_pdl(mglu::pf::prefill_wm_kernel<NM>, dim3((unsigned)grid), dim3(C::NTHREADS), C::SMEM, s,
+                      "prefill wm launch", tx, tw, tm, (int)T, NT, (int)rows, (int)d, act,
+                      reinterpret_cast<__nv_bfloat16 *>(out), mw);
+}
+
 template <int NM, bool GRAD = false>
 int launch_prefill(const void *x, int64_t T, int64_t d, const void *W, int64_t rows, const uint8_t *packed, int act,
                    void *out, void *, cudaStream_t s, const float *mw, const void *dout = nullptr,
@@ -382,6 +409,14 @@ int launch_prefill(const void *x, int64_t T, int64_t d, const void *W, int64_t r
     // down-projection) at any T: its pair kernel was faster on B200 at
     // T = 24 and T = 128 as well (79 against 88 and 91 us at h = 14336,
     // d = 4096), with the same accumulation order per k16 step
+    // up to 128 tokens the n_m = 8 forward puts the weight rows on the MMA's
+    // M side and the tokens on N (at d=4096, h=14336: 195-201 us against
+    // 241 us for T = 24..128 on B200); at n_m <= 4 the token-major kernel
+    // was as fast or faster, so it keeps that range
+    if constexpr (NM == 8 && !GRAD) {
+        if (!mask_direct && T <= mglu::pf::WM_MAX_T)
+            return launch_prefill_wm<NM>(x, T, d, W, rows, packed, act, out, s, mw, dev);
+    }
     if constexpr (NM > 0 || !GRAD) {
         if (!mask_direct && (NM == 0 || T > mglu::pf::BM))
             return launch_prefill_pair<NM, GRAD>(x, T, d, W, rows, packed, act, out, s, mw, dev, dout, gout);

@@ -179,6 +179,57 @@ def test_prefill_pair_repeatable(n_m, T, d, h):
     assert_close(to_f64(first)[b, j], ref, "bf16", f"pair prefill n_m={n_m} sampled")
 
 
+# up to 128 tokens at n_m = 8: the weights-on-M kernel (weight rows on the
+# MMA's M side, tokens on N): ragged token counts (NT = T rounded up to 16),
+# 14-row weight tiles with ragged last tiles, several tiles per CTA, a ragged
+# last k-stage; at n_m <= 4 the same shapes take the token-major kernel
+WM_CASES = [
+    (8, 17, 256, 100),
+    (8, 40, 512, 14),
+    (8, 128, 384, 300),
+    (8, 96, 256, 4000),
+    (8, 50, 144, 60),
+    (8, 113, 320, 29),
+    (4, 33, 256, 101),
+    (4, 100, 640, 25),
+    (2, 64, 384, 170),
+    (2, 120, 256, 42),
+    (1, 48, 256, 130),
+    (1, 128, 512, 64),
+    (4, 70, 160, 77),
+]
+
+
+@pytest.mark.parametrize("n_m,T,d,h", WM_CASES)
+def test_prefill_wm_parity(n_m, T, d, h):
+    case = inputs.make_case(T, d, h, n_m, seed=370 + n_m + T + d + h)
+    got = run_forward(case, "swish")
+    ref, _ = oracle.forward(case.x.values, case.W.values, oracle_packed(case), n_m, ACT["swish"])
+    assert_close(got, ref, "bf16", f"prefill wm n_m={n_m} T={T} d={d} h={h}")
+
+
+@pytest.mark.parametrize("n_m,T,d,h", [(8, 100, 1024, 3000), (8, 24, 2048, 1000)])
+def test_prefill_wm_repeatable(n_m, T, d, h):
+    """The epilogue hands a staging buffer between its four warps through two
+    mbarriers, chunk after chunk; thirty runs must be bit-identical, and the
+    first must match the oracle on an exact sample of elements."""
+    case = inputs.make_case(T, d, h, n_m, seed=380 + n_m)
+    x, W, packed, _ = device_case(case)
+    first = torch.empty((T, h), dtype=torch.bfloat16, device="cuda")
+    mglu.forward(x, W, packed, n_m, "swish", out=first)
+    out = torch.empty_like(first)
+    for rep in range(30):
+        mglu.forward(x, W, packed, n_m, "swish", out=out)
+        torch.cuda.synchronize()
+        assert torch.equal(out, first), f"wm prefill n_m={n_m} repeat {rep} differs"
+    assert mglu.last_device_status() == 0
+    rng = np.random.default_rng(381 + n_m)
+    b = rng.integers(0, T, 2000)
+    j = rng.integers(0, h, 2000)
+    ref, _ = oracle.forward_elems(case.x.values, case.W.values, oracle_packed(case), n_m, ACT["swish"], b, j)
+    assert_close(to_f64(first)[b, j], ref, "bf16", f"wm prefill n_m={n_m} sampled")
+
+
 @pytest.mark.parametrize("T,want", [(40, {1}), (200, {1}), (1, {1, 2})])
 def test_kernel_launch_counter(T, want):
     """One tensor-core launch per forward (one CTA or a CTA pair); the decode

@@ -2,7 +2,9 @@
 in a test-only build of the library (libmglu_testhooks.so): there, every
 mbarrier wait gives up after 20 ms, and mglu_test_set_stall(1) makes the
 kernel's producer stop after the loads of its first stage (T = 300: the kernel
-on CTA pairs, both producers stop; T = 40: the one-CTA kernel).  Every load it did
+on CTA pairs, both producers stop; T = 40: the weights-on-M kernel; d = 200:
+the one-CTA token-major kernel, whose builders load the mask bytes
+themselves).  Every load it did
 issue still lands and is waited for, every MMA issued is drained before TMEM
 is released, and every other wait of the CTA runs out, records
 MGLU_ERR_TIMEOUT in the device status word and returns.  No trap, no fault,
@@ -45,7 +47,7 @@ def _forward(L, x, W, packed, n_m, out):
                           None, 0, s)
 
 
-@pytest.mark.parametrize("n_m,T,d,h", [(4, 300, 512, 200), (8, 40, 256, 96)])
+@pytest.mark.parametrize("n_m,T,d,h", [(4, 300, 512, 200), (8, 40, 256, 96), (4, 40, 200, 96)])
 def test_stalled_producer_times_out_and_the_next_call_is_correct(hooks, n_m, T, d, h):
     L = hooks
     case = inputs.make_case(T, d, h, n_m, seed=1800 + n_m + T)
