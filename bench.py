@@ -716,7 +716,7 @@ def measure_backward(args, dist, dev):
 
 
 def tstar_sweep(args, dist, dev):
-    """Device time of the FFN block (up + down) at T = 8..64 with the decode
+    """Device time of the FFN block (up + down) at T = 8..128 with the decode
     kernel allowed up to 16 tokens and with every T on the tensor-core kernel:
     where the two cross is the dispatch point."""
     import numpy as np
@@ -724,14 +724,14 @@ def tstar_sweep(args, dist, dev):
 
     from masked_glu_b200 import inputs, mglu
 
-    w = workload_shape("ffn_d4096_h14336_nm8", 64)
+    w = workload_shape("ffn_d4096_h14336_nm8", 128)
     d, h, nm = w["d"], w["h"], w["n_m"]
-    case = inputs.make_case(64, d, h, nm, seed=w["seed"], with_down=True)
+    case = inputs.make_case(128, d, h, nm, seed=w["seed"], with_down=True)
 
     def up(t):
         return torch.from_numpy(t.storage.view(np.int16)).view(torch.bfloat16).to(dev)
 
-    x64, W0, Wd0 = up(case.x), up(case.W), up(case.W_down)
+    x128, W0, Wd0 = up(case.x), up(case.W), up(case.W_down)
     pk0 = mglu.pack_masks(torch.from_numpy(case.masks).to(dev))
     del case
     l2 = torch.cuda.get_device_properties(dev).L2_cache_size
@@ -743,8 +743,8 @@ def tstar_sweep(args, dist, dev):
     rows = []
     prev = mglu.set_decode_max_tokens(16)
     try:
-        for T in (8, 12, 16, 24, 32, 48, 64):
-            x = x64[:T].contiguous()
+        for T in (8, 12, 16, 24, 32, 48, 64, 128):
+            x = x128[:T].contiguous()
             hid = torch.empty((T, h), dtype=torch.bfloat16, device=dev)
             yy = torch.empty((T, d), dtype=torch.bfloat16, device=dev)
             row = {"T": T}
