@@ -43,8 +43,13 @@ struct WmCfg {
     static_assert(NM > 0, "the masked product only");
     static constexpr int NJ = 128 / (NM + 1);       // weight rows per tile: 64 / 42 / 25 / 14
     static constexpr int MR = (NM + 1) * NJ;        // stacked rows in use (<= 128)
-    static constexpr int A_BYTES = 128 * BK * 2;    // stacked operand, 128 rows
-    static constexpr int MB = Cfg<NM>::MB;          // mask bytes per row per stage
+    // a stage spans KA 64-k swizzle atoms, so each load fetches KA
+    // neighbouring 128-byte runs of every W row and the hand-offs per k halve
+    static constexpr int KA = 2;
+    static constexpr int BKS = KA * BK;             // k per stage
+    static constexpr int ATOM = 128 * BK * 2;       // one atom of the stacked operand, 128 rows
+    static constexpr int A_BYTES = KA * ATOM;
+    static constexpr int MB = BKS * NM / 8 < 16 ? 16 : BKS * NM / 8;  // mask bytes per row per stage
     static constexpr int M_BYTES = NJ * MB;
     static constexpr int SROW = 33;                 // staging row stride (floats)
     static constexpr int S_BYTES = 128 * SROW * 4;  // 32 token columns of 128 lanes
@@ -59,20 +64,20 @@ struct WmCfg {
     // stream in flight
     static __host__ __device__ constexpr int stage_bytes(int NT)
     {
-        return (A_BYTES + NT * BK * 2 + M_BYTES + 1023) / 1024 * 1024;
+        return (A_BYTES + KA * NT * BK * 2 + M_BYTES + 1023) / 1024 * 1024;
     }
     static __host__ __device__ constexpr int stages(int NT)
     {
         return REGION / stage_bytes(NT) > MAXST ? MAXST : REGION / stage_bytes(NT);
     }
-    static constexpr uint32_t W_TX = NJ * BK * 2;
-    static constexpr int ITEMS = NJ * 8;            // 16-byte pieces of a W tile
+    static constexpr uint32_t W_TX = KA * NJ * BK * 2;
+    static constexpr int ITEMS = KA * NJ * 8;       // 16-byte pieces of a stage's W tile
     // builder groups: where one item per thread takes at most 7 warps, two
     // groups of that many build alternate stages, so two stages are built at
     // once (a stage's build is a chain of waits, loads, stores and proxy
     // fences that one group cannot overlap with the next stage's)
     static constexpr int IW = (ITEMS + 31) / 32;
-    static constexpr int BG = IW <= 7 ? 2 : 1;
+    static constexpr int BG = IW <= 4 ? 2 : 1;
     static constexpr int GW = BG == 2 ? IW : (IW <= 10 ? IW : 8);  // warps per group
     static constexpr int NBW = BG * GW;
     static constexpr int NTHREADS = (2 + NBW + 4) * 32;
@@ -108,8 +113,8 @@ __global__ void __launch_bounds__(WmCfg<NM>::NTHREADS, 1)
     pdl_launch_dependents();
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int num_tiles = (rows + C::NJ - 1) / C::NJ;
-    const int nkb = (d + BK - 1) / BK;
-    const uint32_t x_tx = (uint32_t)NT * BK * 2;
+    const int nkb = (d + C::BKS - 1) / C::BKS;
+    const uint32_t x_tx = (uint32_t)NT * BK * 2;  // one atom of the x tile
     const int STG = C::stage_bytes(NT), NST = C::stages(NT);
     uint8_t *stages = smem + C::ST_OFF;
 
@@ -134,8 +139,8 @@ __global__ void __launch_bounds__(WmCfg<NM>::NTHREADS, 1)
         // the stacked operand's pad rows are never loaded or built: zero them
         // once, for the tensor core (async proxy) to read
         constexpr int PIECES = (128 - C::MR) * 8;
-        for (int i = threadIdx.x; i < NST * PIECES; i += C::NTHREADS) {
-            uint8_t *A = stages + (i / PIECES) * STG;
+        for (int i = threadIdx.x; i < NST * C::KA * PIECES; i += C::NTHREADS) {
+            uint8_t *A = stages + (i / (C::KA * PIECES)) * STG + ((i / PIECES) % C::KA) * C::ATOM;
             *reinterpret_cast<uint4 *>(A + (C::MR + (i % PIECES) / 8) * 128 + (i % 8) * 16) = make_uint4(0, 0, 0, 0);
         }
         fence_proxy_async_smem();
@@ -174,12 +179,16 @@ __global__ void __launch_bounds__(WmCfg<NM>::NTHREADS, 1)
                     }
                     uint8_t *st = stages + s * STG;
                     mbar_arrive_expect_tx(&wfull[s], C::W_TX);
-                    tma_load_2d(st, &tm_w, &wfull[s], kb * BK, n0);  // block 0 of the stacked operand
-                    const int mc = (kb * BK * NM / 8) / C::MB * C::MB;  // 16-byte aligned column
+#pragma unroll
+                    for (int a = 0; a < C::KA; ++a)  // block 0 of each atom of the stacked operand
+                        tma_load_2d(st + a * C::ATOM, &tm_w, &wfull[s], kb * C::BKS + a * BK, n0);
+                    const int mc = (kb * C::BKS * NM / 8) / C::MB * C::MB;  // 16-byte aligned column
                     mbar_arrive_expect_tx(&mfull[s], C::M_BYTES);
-                    tma_load_2d(st + C::A_BYTES + x_tx, &tm_m, &mfull[s], mc, n0);
-                    mbar_arrive_expect_tx(&xfull[s], x_tx);
-                    tma_load_2d(st + C::A_BYTES, &tm_x, &xfull[s], kb * BK, 0);
+                    tma_load_2d(st + C::A_BYTES + C::KA * x_tx, &tm_m, &mfull[s], mc, n0);
+                    mbar_arrive_expect_tx(&xfull[s], C::KA * x_tx);
+#pragma unroll
+                    for (int a = 0; a < C::KA; ++a)
+                        tma_load_2d(st + C::A_BYTES + a * x_tx, &tm_x, &xfull[s], kb * C::BKS + a * BK, 0);
                 }
             }
             // every load issued has landed before the CTA may exit
@@ -214,9 +223,12 @@ __global__ void __launch_bounds__(WmCfg<NM>::NTHREADS, 1)
                     const uint32_t a_addr = smem_u32(stages + s * STG);
                     const uint32_t b_addr = a_addr + C::A_BYTES;
 #pragma unroll
-                    for (int k16 = 0; k16 < BK / 16; ++k16)
-                        umma_f16_ss(d_tmem, sw128_kmajor_desc(a_addr + k16 * 32), sw128_kmajor_desc(b_addr + k16 * 32),
-                                    idesc, (kb | k16) != 0 ? 1u : 0u);
+                    for (int a = 0; a < C::KA; ++a)
+#pragma unroll
+                        for (int k16 = 0; k16 < BK / 16; ++k16)
+                            umma_f16_ss(d_tmem, sw128_kmajor_desc(a_addr + a * C::ATOM + k16 * 32),
+                                        sw128_kmajor_desc(b_addr + a * x_tx + k16 * 32), idesc,
+                                        (kb | a | k16) != 0 ? 1u : 0u);
                     umma_commit(&empty[s]);
                 }
                 if (ok)
@@ -243,17 +255,18 @@ __global__ void __launch_bounds__(WmCfg<NM>::NTHREADS, 1)
                 }
                 fence_proxy_async_smem();  // TMA-written tiles are read with ordinary loads below
                 uint8_t *A = stages + s * STG;
-                const uint8_t *Mt = A + C::A_BYTES + x_tx;
-                const int moff = (kb * BK * NM / 8) % C::MB;  // nonzero only when NM = 1
+                const uint8_t *Mt = A + C::A_BYTES + C::KA * x_tx;
 #pragma unroll
                 for (int q = 0; q < MAXI; ++q) {
                     const int item = bt + q * 32 * C::GW;
                     if (item < C::ITEMS) {
-                        const int r = item >> 3, c = item & 7;
-                        const uint4 w = *reinterpret_cast<const uint4 *>(A + r * 128 + ((c ^ (r & 7)) << 4));
+                        const int a = item / (C::NJ * 8), rem = item % (C::NJ * 8);
+                        const int r = rem >> 3, c = rem & 7;
+                        uint8_t *Aa = A + a * C::ATOM;
+                        const uint4 w = *reinterpret_cast<const uint4 *>(Aa + r * 128 + ((c ^ (r & 7)) << 4));
                         uint32_t lo, hi;
-                        load_mask_bytes<NM>(Mt + r * C::MB + moff + c * NM, lo, hi);
-                        build_variants_pair<NM, C::NJ, 0>(A, r, c, w, lo, hi);
+                        load_mask_bytes<NM>(Mt + r * C::MB + a * (BK * NM / 8) + c * NM, lo, hi);
+                        build_variants_pair<NM, C::NJ, 0>(Aa, r, c, w, lo, hi);
                     }
                 }
                 fence_proxy_async_smem();  // generic-proxy writes -> visible to the tensor core
