@@ -489,7 +489,7 @@ def test_relu_is_homogeneous_of_degree_two(n_m, T):
 # ------------------------------------------------------------------ dense-gate ablation
 @pytest.mark.parametrize("n_m,T,d,h,dtype", [(4, 1, 512, 200, "bf16"), (8, 9, 256, 96, "bf16"),
                                              (4, 150, 384, 200, "bf16"), (1, 40, 256, 64, "bf16"),
-                                             (8, 300, 256, 90, "bf16"),
+                                             (8, 300, 256, 90, "bf16"), (8, 64, 256, 50, "bf16"),
                                              (2, 5, 100, 37, "f32")])
 @pytest.mark.parametrize("act", ["swish", "gelu", "relu"])
 def test_dense_gate_matches_oracle(n_m, T, d, h, dtype, act):

@@ -60,7 +60,7 @@ def test_route_ties_go_to_the_lower_index():
 
 @pytest.mark.parametrize("n_m,T,d,h", [(4, 1, 512, 200), (8, 3, 256, 96), (8, 9, 256, 96), (4, 16, 384, 130),
                                        (4, 40, 256, 100), (8, 200, 384, 72), (2, 5, 96, 40),
-                                       (8, 390, 256, 86)])
+                                       (8, 390, 256, 86), (8, 70, 256, 60)])
 def test_weighted_forward_matches_oracle(n_m, T, d, h):
     case = inputs.make_case(T, d, h, n_m, seed=2400 + n_m + T + d)
     x, W, packed, _ = device_case(case)
