@@ -409,12 +409,13 @@ int launch_prefill(const void *x, int64_t T, int64_t d, const void *W, int64_t r
     // down-projection) at any T: its pair kernel was faster on B200 at
     // T = 24 and T = 128 as well (79 against 88 and 91 us at h = 14336,
     // d = 4096), with the same accumulation order per k16 step
-    // up to 128 tokens the n_m = 8 forward puts the weight rows on the MMA's
-    // M side and the tokens on N (at d=4096, h=14336: 195-201 us against
-    // 241 us for T = 24..128 on B200); at n_m <= 4 the token-major kernel
-    // was as fast or faster, so it keeps that range
-    if constexpr (NM == 8 && !GRAD) {
-        if (!mask_direct && T <= mglu::pf::WM_MAX_T)
+    // up to 128 tokens at n_m = 8 and up to 96 at n_m = 4 the forward puts
+    // the weight rows on the MMA's M side and the tokens on N.  On B200 at
+    // d=4096, h=14336: n_m = 8 143-200 us against 241 us (T = 24..128);
+    // n_m = 4 89-121 us against 127-130 us (T = 17..96), at T = 128 about
+    // equal.  At n_m <= 2 the token-major kernel keeps the range
+    if constexpr ((NM == 8 || NM == 4) && !GRAD) {
+        if (!mask_direct && T <= (NM == 8 ? mglu::pf::WM_MAX_T : 96))
             return launch_prefill_wm<NM>(x, T, d, W, rows, packed, act, out, s, mw, dev);
     }
     if constexpr (NM > 0 || !GRAD) {

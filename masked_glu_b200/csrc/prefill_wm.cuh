@@ -1,6 +1,6 @@
 // prefill_wm.cuh -- the MGLU up-projection for 17 to 128 tokens with the
 // weights on the MMA's M side and the tokens on N (the library runs it for
-// n_m = 8; the template takes any n_m >= 1).
+// n_m = 8 and, up to 96 tokens, n_m = 4).
 //
 // The token-major kernels (prefill.cuh, prefill_pair.cuh) multiply a whole
 // 128- or 256-token tile whatever T is, so below a full tile their cost does

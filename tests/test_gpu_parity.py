@@ -179,10 +179,11 @@ def test_prefill_pair_repeatable(n_m, T, d, h):
     assert_close(to_f64(first)[b, j], ref, "bf16", f"pair prefill n_m={n_m} sampled")
 
 
-# up to 128 tokens at n_m = 8: the weights-on-M kernel (weight rows on the
-# MMA's M side, tokens on N): ragged token counts (NT = T rounded up to 16),
-# 14-row weight tiles with ragged last tiles, several tiles per CTA, a ragged
-# last k-stage; at n_m <= 4 the same shapes take the token-major kernel
+# up to 128 tokens at n_m = 8 and 96 at n_m = 4: the weights-on-M kernel
+# (weight rows on the MMA's M side, tokens on N): ragged token counts (NT = T
+# rounded up to 16), 14- and 25-row weight tiles with ragged last tiles,
+# several tiles per CTA, a ragged last k-stage; at n_m <= 2 (and n_m = 4
+# above 96 tokens) the same shapes take the token-major kernel
 WM_CASES = [
     (8, 17, 256, 100),
     (8, 40, 512, 14),
@@ -197,6 +198,8 @@ WM_CASES = [
     (1, 48, 256, 130),
     (1, 128, 512, 64),
     (4, 70, 160, 77),
+    (4, 96, 384, 260),
+    (4, 17, 128, 50),
 ]
 
 
@@ -208,7 +211,7 @@ def test_prefill_wm_parity(n_m, T, d, h):
     assert_close(got, ref, "bf16", f"prefill wm n_m={n_m} T={T} d={d} h={h}")
 
 
-@pytest.mark.parametrize("n_m,T,d,h", [(8, 100, 1024, 3000), (8, 24, 2048, 1000)])
+@pytest.mark.parametrize("n_m,T,d,h", [(8, 100, 1024, 3000), (8, 24, 2048, 1000), (4, 64, 2048, 1000)])
 def test_prefill_wm_repeatable(n_m, T, d, h):
     """The epilogue hands a staging buffer between its four warps through two
     mbarriers, chunk after chunk; thirty runs must be bit-identical, and the
