@@ -409,13 +409,14 @@ int launch_prefill(const void *x, int64_t T, int64_t d, const void *W, int64_t r
     // down-projection) at any T: its pair kernel was faster on B200 at
     // T = 24 and T = 128 as well (79 against 88 and 91 us at h = 14336,
     // d = 4096), with the same accumulation order per k16 step
-    // up to 128 tokens at n_m = 8 and up to 96 at n_m = 4 the forward puts
-    // the weight rows on the MMA's M side and the tokens on N.  On B200 at
-    // d=4096, h=14336: n_m = 8 143-200 us against 241 us (T = 24..128);
-    // n_m = 4 89-121 us against 127-130 us (T = 17..96), at T = 128 about
-    // equal.  At n_m <= 2 the token-major kernel keeps the range
-    if constexpr ((NM == 8 || NM == 4) && !GRAD) {
-        if (!mask_direct && T <= (NM == 8 ? mglu::pf::WM_MAX_T : 96))
+    // up to 128 tokens at n_m = 8, 96 at n_m = 4 and 32 at n_m <= 2 the
+    // forward puts the weight rows on the MMA's M side and the tokens on N.
+    // On B200 at d=4096, h=14336: n_m = 8 143-200 us against 241 us
+    // (T = 24..128); n_m = 4 89-121 us against 127-130 us (T = 17..96), about
+    // equal at T = 128; n_m = 2 68-70 us against 88 us (T = 17..32), slower
+    // from T = 96 (at d=2048, h=8192 already from T = 64)
+    if constexpr (NM > 0 && !GRAD) {
+        if (!mask_direct && T <= (NM == 8 ? mglu::pf::WM_MAX_T : NM == 4 ? 96 : 32))
             return launch_prefill_wm<NM>(x, T, d, W, rows, packed, act, out, s, mw, dev);
     }
     if constexpr (NM > 0 || !GRAD) {

@@ -1,6 +1,6 @@
 // prefill_wm.cuh -- the MGLU up-projection for 17 to 128 tokens with the
-// weights on the MMA's M side and the tokens on N (the library runs it for
-// n_m = 8 and, up to 96 tokens, n_m = 4).
+// weights on the MMA's M side and the tokens on N (the library runs it up
+// to 128 tokens at n_m = 8, 96 at n_m = 4 and 32 at n_m <= 2).
 //
 // The token-major kernels (prefill.cuh, prefill_pair.cuh) multiply a whole
 // 128- or 256-token tile whatever T is, so below a full tile their cost does
@@ -78,7 +78,8 @@ struct WmCfg {
     // fences that one group cannot overlap with the next stage's)
     static constexpr int IW = (ITEMS + 31) / 32;
     static constexpr int BG = IW <= 4 ? 2 : 1;
-    static constexpr int GW = BG == 2 ? IW : (IW <= 10 ? IW : 8);  // warps per group
+    // warps per group: one piece per thread up to 10 warps, else two
+    static constexpr int GW = BG == 2 ? IW : (IW <= 10 ? IW : ((IW + 1) / 2 > 8 ? (IW + 1) / 2 : 8));
     static constexpr int NBW = BG * GW;
     static constexpr int NTHREADS = (2 + NBW + 4) * 32;
     static_assert(stages(WM_MAX_T) >= 3, "ring too shallow");

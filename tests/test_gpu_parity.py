@@ -179,11 +179,12 @@ def test_prefill_pair_repeatable(n_m, T, d, h):
     assert_close(to_f64(first)[b, j], ref, "bf16", f"pair prefill n_m={n_m} sampled")
 
 
-# up to 128 tokens at n_m = 8 and 96 at n_m = 4: the weights-on-M kernel
-# (weight rows on the MMA's M side, tokens on N): ragged token counts (NT = T
-# rounded up to 16), 14- and 25-row weight tiles with ragged last tiles,
-# several tiles per CTA, a ragged last k-stage; at n_m <= 2 (and n_m = 4
-# above 96 tokens) the same shapes take the token-major kernel
+# up to 128 tokens at n_m = 8, 96 at n_m = 4 and 32 at n_m <= 2: the
+# weights-on-M kernel (weight rows on the MMA's M side, tokens on N): ragged
+# token counts (NT = T rounded up to 16), 14-, 25-, 42- and 64-row weight
+# tiles with ragged last tiles, several tiles per CTA, a ragged last
+# k-stage; above those token counts the same shapes take the token-major
+# kernels
 WM_CASES = [
     (8, 17, 256, 100),
     (8, 40, 512, 14),
@@ -200,6 +201,10 @@ WM_CASES = [
     (4, 70, 160, 77),
     (4, 96, 384, 260),
     (4, 17, 128, 50),
+    (2, 20, 256, 90),
+    (2, 32, 320, 200),
+    (1, 32, 384, 130),
+    (1, 17, 256, 64),
 ]
 
 
@@ -211,7 +216,8 @@ def test_prefill_wm_parity(n_m, T, d, h):
     assert_close(got, ref, "bf16", f"prefill wm n_m={n_m} T={T} d={d} h={h}")
 
 
-@pytest.mark.parametrize("n_m,T,d,h", [(8, 100, 1024, 3000), (8, 24, 2048, 1000), (4, 64, 2048, 1000)])
+@pytest.mark.parametrize("n_m,T,d,h", [(8, 100, 1024, 3000), (8, 24, 2048, 1000), (4, 64, 2048, 1000),
+                                       (1, 32, 2048, 1000)])
 def test_prefill_wm_repeatable(n_m, T, d, h):
     """The epilogue hands a staging buffer between its four warps through two
     mbarriers, chunk after chunk; thirty runs must be bit-identical, and the
